@@ -1,0 +1,357 @@
+#!/usr/bin/env python
+"""Benchmark of the QK-RMSNorm sliding-window attention core on B200.
+
+One step = forward + backward of every layer of the 8-layer "SSSL" attention
+stack (B=8, T=2048, H=4, D=128; layers 0-2 and 4-6 window 1024, layers 3 and 7
+full causal), each layer on its own seeded bf16 inputs, all enqueued back to
+back on one stream through the C ABI (libar_attn.so).
+
+Metric: TFLOP/s counted on unmasked (query, key) pairs only, 4*D FLOPs per pair
+forward and 2.5x that backward; also reported as a fraction of the measured
+dense bf16 tensor-core peak.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+
+With N > 1 (under torchrun) every rank runs the same workload on its own GPU
+(replicas: the core has no cross-GPU data flow); the time is the max over
+ranks and the value the sum of all ranks' FLOPs over that time.
+--impl reference times the fp64 CPU oracle on a bounded sample instead.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attn fwd+bwd TFLOP/s (unmasked) at T=2048 SSSL; % of B200 BF16 peak"
+D = 128
+FWD_FLOPS_PER_PAIR = 4 * D
+BWD_FACTOR = 2.5
+
+WORKLOADS = {
+    "stack8": dict(config=3, B=8, T=2048, H=4, n_layer=8, pattern="SSSL",
+                   name="8-layer SSSL attention stack fwd+bwd, B=8 T=2048 H=4 D=128 (windows 1024/full)"),
+    "stack12": dict(config=5, B=8, T=2048, H=6, n_layer=12, pattern="SSSL",
+                    name="12-layer SSSL attention stack fwd+bwd, B=8 T=2048 H=6 D=128 (windows 1024/full)"),
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="stack8")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def windows_for(wl):
+    from oracle.stack import layer_windows  # pure-Python rule, used only for FLOP counting here
+    return layer_windows(wl["n_layer"], wl["T"], wl["pattern"])
+
+
+def pairs(T, w):
+    w = T if (w < 0 or w >= T - 1) else w
+    n1 = min(w + 1, T)
+    return n1 * (n1 + 1) // 2 + (T - n1) * (w + 1)
+
+
+def step_flops(wl):
+    """(forward, backward) counted FLOPs of one step of the workload."""
+    f = sum(wl["B"] * wl["H"] * pairs(wl["T"], w) * FWD_FLOPS_PER_PAIR for w in windows_for(wl))
+    return f, BWD_FACTOR * f
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(bf16_burst=d["bf16_tflops"], bf16_sustained=d["bf16_tflops_sustained"], hbm=d["hbm_gbs"],
+                    source="measured")
+    return dict(bf16_burst=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the GPU is timed."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.samples = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_id), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [s for (t, s) in self.samples if t0 <= t <= t1] or [s for (_, s) in self.samples]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 5 + i and "Active" == r[5 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((num(r[3]) or 0.0) for r in rows)}
+
+
+# ---------------------------------------------------------------- oracle (CPU baseline and reference arm)
+_INPUT_CACHE = {}
+
+
+def _layer_inputs_cached(wl, layer):
+    from sliding_window_attention_rmsnorm_b200 import synth
+    key = (wl["config"], layer)
+    if key not in _INPUT_CACHE:
+        _INPUT_CACHE[key] = synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], wl["H"], D)
+    return _INPUT_CACHE[key]
+
+
+def oracle_sample(wl, seconds, seed_layer_offset=0):
+    """Run the fp64 oracle fwd+bwd on whole heads of the workload's layers,
+    cycling through layers, for about `seconds`; returns (flops, secs, desc, threads)."""
+    from oracle import oracle as orc
+    ws = windows_for(wl)
+    B, T, H = wl["B"], wl["T"], wl["H"]
+    flops, heads_done, t_total, n = 0.0, [], 0.0, 0
+    while t_total < seconds or n == 0:
+        layer = (n + seed_layer_offset) % wl["n_layer"]
+        head = (7 * n + 3) % (B * H)
+        b, h = divmod(head, H)
+        x = _layer_inputs_cached(wl, layer)
+        xs = {r: t[b:b + 1, :, h:h + 1].contiguous() for r, t in x.items()}
+        t0 = time.perf_counter()
+        orc.attn_fwd(xs["q"], xs["k"], xs["v"], ws[layer])
+        orc.attn_bwd(xs["q"], xs["k"], xs["v"], xs["dO"], ws[layer])
+        t_total += time.perf_counter() - t0
+        flops += pairs(T, ws[layer]) * FWD_FLOPS_PER_PAIR * (1 + BWD_FACTOR)
+        heads_done.append((layer, head))
+        n += 1
+    desc = "%d whole heads (T=%d) of the workload's layers, fwd+bwd in fp64 C/OpenMP" % (n, T)
+    return flops, t_total, desc, orc.num_threads()
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    from oracle import oracle as orc
+    per_step = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(wl, 0.0)
+    flops, secs, desc, threads = 0.0, 0.0, "", orc.num_threads()
+    for s in range(args.steps):
+        f, t, desc, threads = oracle_sample(wl, per_step, seed_layer_offset=s)
+        flops += f
+        secs += t
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl["name"], "global_batch": wl["B"], "seq_len": wl["T"], "heads": wl["H"],
+                   "layers": wl["n_layer"], "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": "per step: " + desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our CUDA path
+def run_ours(args, wl, rank, world, dist):
+    import torch
+    from sliding_window_attention_rmsnorm_b200 import attn, build, stack, synth
+
+    dev = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(dev)
+    build.build()
+    B, T, H, L = wl["B"], wl["T"], wl["H"], wl["n_layer"]
+    host = [synth.layer_inputs(wl["config"], l, B, T, H, D) for l in range(L)]
+    layers = [{r: t.to("cuda", non_blocking=False) for r, t in x.items()} for x in host]
+    st = stack.Stack(layers, wl["pattern"])
+    fwd_f, bwd_f = step_flops(wl)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        st.step()
+    attn.sync_status()
+
+    visible = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+    sampler = ClockSampler(visible[dev] if dev < len(visible) else dev) if rank == 0 else None
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    attn.timing_enable(True)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        st.step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier()
+    attn.timing_enable(False)
+    attn.sync_status()
+    ms = e0.elapsed_time(e1) / args.steps
+    kern = attn.timing_read()
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    clocks = None
+    if sampler is not None:
+        sampler.stop()
+        clocks = sampler.summary(t_wall0, t_wall1)
+
+    value = world * (fwd_f + bwd_f) / (ms * 1e-3) / 1e12
+    peaks = measured_peaks()
+
+    # roofline of the dominant kernel: counted FLOPs per launch over its event-timed mean duration
+    per_kind_flops = {"fwd": fwd_f / L, "bwd": bwd_f / L}
+    dom = max(("fwd", "bwd"), key=lambda k: kern[k][0])
+    tot_ms, n_launch = kern[dom]
+    achieved = (per_kind_flops[dom] * n_launch) / (tot_ms * 1e-3) / 1e12
+    roof = {"kernel": dom + "_kernel", "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_sustained"],
+            "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"], "traffic": None,
+            "peak_kind": "bf16 sustained (%s)" % peaks["source"]}
+    kernels = {k: {"ms_per_launch": (v[0] / v[1]) if v[1] else None, "launches": v[1],
+                   "share": v[0] / max(1e-9, sum(x[0] for x in kern.values()))} for k, v in kern.items()}
+    for k in ("fwd", "bwd"):
+        if kern[k][1]:
+            kernels[k]["tflops"] = per_kind_flops[k] * kern[k][1] / (kern[k][0] * 1e-3) / 1e12
+    # memory-bound helpers: algorithmic bytes per launch
+    tok = B * T * H
+    algo_bytes = {"fwd_prep": tok * D * 2 + tok * 4,
+                  "bwd_prep": 3 * tok * D * 2 + tok * 4 * 4 + tok * D * 4,
+                  "dq_post": tok * D * 4 + tok * D * 2 * 2}
+    for k, by in algo_bytes.items():
+        if kern[k][1]:
+            kernels[k]["gbs"] = by * kern[k][1] / (kern[k][0] * 1e-3) / 1e9
+            kernels[k]["hbm_frac"] = kernels[k]["gbs"] / peaks["hbm"]
+
+    # end to end: inputs from pinned host memory, results back to host, all inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        pinned = [{r: t.pin_memory() for r, t in x.items()} for x in host]
+        outs_h = [{n: torch.empty(st.out[l][n].shape, dtype=st.out[l][n].dtype, pin_memory=True)
+                   for n in ("o", "dq", "dk", "dv")} for l in range(L)]
+        def e2e_step():
+            for l in range(L):
+                for r in ("q", "k", "v", "dO"):
+                    layers[l][r].copy_(pinned[l][r], non_blocking=True)
+            st.step()
+            for l in range(L):
+                for n in ("o", "dq", "dk", "dv"):
+                    outs_h[l][n].copy_(st.out[l][n], non_blocking=True)
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = a0.elapsed_time(a1) / args.e2e_steps
+        if dist is not None:
+            t = torch.tensor([ms_e2e], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        h2d = sum(t.numel() * t.element_size() for x in pinned for t in x.values())
+        d2h = sum(t.numel() * t.element_size() for x in outs_h for t in x.values())
+        e2e = {"value": world * (fwd_f + bwd_f) / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, secs, desc, threads = oracle_sample(wl, args.cpu_seconds)
+        cpu = {"value": f / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl["name"], "global_batch": B * world, "seq_len": T, "heads": H,
+                       "layers": L, "windows": windows_for(wl), "parallelism": "replicas x%d" % world,
+                       "l2": "inputs larger than L2 (%.0f MB of q,k,v,dO per step)" % (4 * L * tok * D * 2 / 1e6)},
+            "pct_of_bf16_peak": {"sustained": value / world / peaks["bf16_sustained"],
+                                 "burst": value / world / peaks["bf16_burst"], "source": peaks["source"]},
+            "roofline": roof,
+            "kernels": kernels,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": int(sum(v[1] for v in kern.values())),
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    wl = WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if args.impl == "ours":
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        if args.impl == "reference":
+            run_reference(args, wl, rank, world)
+        else:
+            run_ours(args, wl, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,128 @@
+/*
+ * ar_attn.h - C ABI of the QK-RMSNorm sliding-window attention core (sm_100a).
+ *
+ * The operation (per batch b and head h, queries i and keys j of one sequence):
+ *
+ *   qhat_i = q_i / sqrt(mean_d q_id^2 + eps),  khat_j likewise     (RMSNorm, no gain)
+ *   s_ij   = scale * qhat_i . khat_j          for 0 <= i - j <= window, else masked
+ *   lse_i  = log sum_j exp(s_ij),   o_i = sum_j exp(s_ij - lse_i) v_j
+ *
+ * and its exact gradient with respect to q, k and v.  Sources on the reference
+ * pages: the "autoresearch" README (gitee), section 7.3 "CausalSelfAttention"
+ * (norm(x) = F.rms_norm(x, (x.size(-1),)) applied to q and k, no weight) and
+ * sections 5.2.1-5.2.2 (FlashAttention-3 with window_size = (window, 0); the
+ * "SSSL" pattern: S = seq_len/2, L = seq_len, last layer forced to L); the
+ * web3.okx.com code review, paragraphs on the QK norm and on the window pattern.
+ *
+ * Conventions shared by every entry point
+ *   - q, k, v, o, dO, dq, dk, dv: bf16, layout [B, T, H, D] contiguous, D = 128.
+ *   - lse: fp32 [B, H, T], natural logarithm.
+ *   - window: a key j is visible to query i iff 0 <= i - j <= window.  window < 0
+ *     or window >= T - 1 means full causal attention.  window = 0: each query
+ *     sees only itself.
+ *   - eps >= 0 and finite; scale > 0 and finite (usually 1/sqrt(D)).
+ *   - All pointers are DEVICE pointers of the current CUDA device, 16-byte
+ *     aligned (the kernels read them with TMA).  The caller owns every buffer;
+ *     the library never frees or retains caller memory.
+ *   - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls only enqueue work and return; results are ready when the stream is.
+ *   - Return value: AR_OK (0) or a negative AR_ERR_* code.  No exception or
+ *     abort crosses the ABI.  Argument errors are detected before any work is
+ *     enqueued.  A device-side wait that gives up (AR_ERR_TIMEOUT) is reported
+ *     by ar_attn_sync_status().
+ *   - Workspace: if `workspace` is NULL the library allocates it stream-ordered
+ *     (cudaMallocAsync / cudaFreeAsync on `stream`); otherwise it must hold at
+ *     least the bytes returned by the matching *_workspace_bytes() call and be
+ *     256-byte aligned.  It is scratch: its contents on entry do not matter.
+ */
+#ifndef AR_ATTN_H
+#define AR_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  AR_OK = 0,
+  AR_ERR_NULL = -1,        /* a required pointer is NULL */
+  AR_ERR_SHAPE = -2,       /* B, T or H <= 0, or sizes overflow the index range */
+  AR_ERR_UNSUPPORTED = -3, /* D != 128 */
+  AR_ERR_ALIGN = -4,       /* a pointer is not 16-byte aligned (workspace: 256) */
+  AR_ERR_ARG = -5,         /* eps < 0, scale <= 0, or either is not finite */
+  AR_ERR_DEVICE = -6,      /* current device is not compute capability 10.0 (B200) */
+  AR_ERR_CUDA = -7,        /* a CUDA runtime call failed */
+  AR_ERR_TIMEOUT = -8,     /* a device-side wait gave up (reported by sync_status) */
+  AR_ERR_WORKSPACE = -9    /* workspace given but smaller than required */
+};
+
+/* Bytes of scratch ar_attn_fwd needs: one fp32 per (b, h, t) rounded up to
+ * whole 128-token tiles (the per-key norm factors).  0 on invalid sizes. */
+size_t ar_attn_fwd_workspace_bytes(int B, int T, int H, int D);
+
+/* Forward pass.  Inputs q, k, v; outputs o [B,T,H,D] bf16 and lse [B,H,T] fp32
+ * (lse is what ar_attn_bwd needs).  Launches a per-key norm pre-pass and the
+ * fused attention kernel on `stream`. */
+int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                int B, int T, int H, int D, int window, float eps, float scale,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of scratch ar_attn_bwd needs: an fp32 [B,T,H,D] dq accumulator plus
+ * three fp32 per-(b, h, t) vectors.  0 on invalid sizes. */
+size_t ar_attn_bwd_workspace_bytes(int B, int T, int H, int D);
+
+/* Backward pass.  Inputs q, k, v, the forward's o and lse, and the upstream
+ * gradient dO; outputs dq, dk, dv [B,T,H,D] bf16 (overwritten, not added to).
+ * window, eps and scale must be the forward's.  Launches, on `stream`: the
+ * pre-pass (delta = rowsum(dO * o), 1/rms(q), accumulator reset), the fused
+ * backward kernel (dk, dv, dq accumulation), and the dq RMSNorm post-pass. */
+int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                const float* lse, void* dq, void* dk, void* dv,
+                int B, int T, int H, int D, int window, float eps, float scale,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears this device's status word.
+ * Returns AR_OK, AR_ERR_TIMEOUT if a kernel abandoned a wait since the last
+ * call, or AR_ERR_CUDA if the synchronisation itself failed. */
+int ar_attn_sync_status(void* stream);
+
+/* Static, human-readable text for a status code (never NULL). */
+const char* ar_attn_strerror(int status);
+
+/* Window of layer `layer` in a stack of n_layer layers following `pattern`
+ * (characters 'S' and 'L', case-insensitive; layer l uses pattern[l mod len]):
+ * 'L' -> seq_len, 'S' -> seq_len / 2, and the last layer always seq_len.
+ * Returns a negative AR_ERR_* code on invalid arguments. */
+int ar_attn_layer_window(int layer, int n_layer, int seq_len, const char* pattern);
+
+/* Number of visible (query, key) pairs of one head: sum_i (min(i, w) + 1),
+ * w = window as above.  Used to count the FLOPs the attention really does. */
+long long ar_attn_unmasked_pairs(int T, int window);
+
+/* Kernel timing for measurement.  Kernel kinds, in launch order: */
+enum {
+  AR_KERNEL_FWD_PREP = 0, /* per-key norm factors (memory-bound) */
+  AR_KERNEL_FWD = 1,      /* fused forward attention (tensor-core bound) */
+  AR_KERNEL_BWD_PREP = 2, /* delta, 1/rms(q), accumulator reset (memory-bound) */
+  AR_KERNEL_BWD = 3,      /* fused backward attention (tensor-core bound) */
+  AR_KERNEL_DQ_POST = 4,  /* dq RMSNorm backward (memory-bound) */
+  AR_KERNEL_KINDS = 5
+};
+
+/* on != 0: clear the record and, until called with on == 0, bracket every
+ * kernel that ar_attn_fwd / ar_attn_bwd launch with CUDA events on the call's
+ * stream (a few microseconds of host time per kernel).  on == 0 stops
+ * recording and keeps what was recorded for ar_attn_timing_read.  Returns AR_OK. */
+int ar_attn_timing_enable(int on);
+
+/* Waits for the recorded events and writes, per kernel kind, the summed device
+ * time in milliseconds (ms[AR_KERNEL_KINDS]) and the number of launches
+ * (count[AR_KERNEL_KINDS]); either pointer may be NULL.  Clears the record. */
+int ar_attn_timing_read(double* ms, long long* count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AR_ATTN_H */

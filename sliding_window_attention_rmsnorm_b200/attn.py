@@ -1,0 +1,166 @@
+"""ctypes binding of libar_attn.so (argument marshalling only).
+
+Every step of the attention core runs in the library's CUDA kernels; this
+module checks tensor dtypes/devices, allocates outputs and scratch with torch's
+caching allocator, and passes raw pointers plus torch's current CUDA stream.
+If the library is missing or cannot be loaded, the first call raises: there is
+no fallback implementation.
+"""
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libar_attn.so")
+
+AR_OK = 0
+STATUS = {
+    0: "AR_OK", -1: "AR_ERR_NULL", -2: "AR_ERR_SHAPE", -3: "AR_ERR_UNSUPPORTED", -4: "AR_ERR_ALIGN",
+    -5: "AR_ERR_ARG", -6: "AR_ERR_DEVICE", -7: "AR_ERR_CUDA", -8: "AR_ERR_TIMEOUT", -9: "AR_ERR_WORKSPACE",
+}
+
+_lib = None
+
+
+class ArAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s failed: %s (%s)" % (where, STATUS.get(status, status), strerror(status)))
+
+
+def lib():
+    """Load libar_attn.so (raises OSError if it is absent)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise OSError("libar_attn.so not built at %s; run sliding_window_attention_rmsnorm_b200.build"
+                          % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.ar_attn_fwd_workspace_bytes.argtypes = [i, i, i, i]
+        L.ar_attn_fwd_workspace_bytes.restype = sz
+        L.ar_attn_bwd_workspace_bytes.argtypes = [i, i, i, i]
+        L.ar_attn_bwd_workspace_bytes.restype = sz
+        L.ar_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, vp, sz, vp]
+        L.ar_attn_fwd.restype = i
+        L.ar_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, f, vp, sz, vp]
+        L.ar_attn_bwd.restype = i
+        L.ar_attn_sync_status.argtypes = [vp]
+        L.ar_attn_sync_status.restype = i
+        L.ar_attn_strerror.argtypes = [i]
+        L.ar_attn_strerror.restype = ctypes.c_char_p
+        L.ar_attn_layer_window.argtypes = [i, i, i, ctypes.c_char_p]
+        L.ar_attn_layer_window.restype = i
+        L.ar_attn_unmasked_pairs.argtypes = [i, i]
+        L.ar_attn_unmasked_pairs.restype = ctypes.c_longlong
+        L.ar_attn_timing_enable.argtypes = [i]
+        L.ar_attn_timing_enable.restype = i
+        L.ar_attn_timing_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
+        L.ar_attn_timing_read.restype = i
+        _lib = L
+    return _lib
+
+
+def strerror(status: int) -> str:
+    return lib().ar_attn_strerror(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != AR_OK:
+        raise ArAttnError(status, where)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check_inputs(*ts):
+    for t in ts:
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 4):
+            raise ValueError("expected contiguous bf16 CUDA tensors of shape [B, T, H, D]")
+        if t.shape != ts[0].shape:
+            raise ValueError("q, k, v (and o, dO) must have the same shape")
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)
+
+
+def fwd_workspace_bytes(B, T, H, D) -> int:
+    return int(lib().ar_attn_fwd_workspace_bytes(B, T, H, D))
+
+
+def bwd_workspace_bytes(B, T, H, D) -> int:
+    return int(lib().ar_attn_bwd_workspace_bytes(B, T, H, D))
+
+
+def fwd(q, k, v, window: int, eps: float = 1e-6, scale=None, out=None, lse=None, workspace=None):
+    """o, lse = attention(norm(q), norm(k), v) over the band 0 <= i - j <= window.
+
+    q, k, v: bf16 CUDA tensors [B, T, H, 128].  Returns o (bf16, same shape)
+    and lse (fp32 [B, H, T]).  Enqueued on torch's current stream.
+    """
+    _check_inputs(q, k, v)
+    B, T, H, D = q.shape
+    if scale is None:
+        scale = default_scale(D)
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((B, H, T), dtype=torch.float32, device=q.device) if lse is None else lse
+    if workspace is None:
+        workspace = torch.empty(max(fwd_workspace_bytes(B, T, H, D), 1), dtype=torch.uint8, device=q.device)
+    st = lib().ar_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, T, H, D, int(window),
+                           float(eps), float(scale), _ptr(workspace), workspace.numel(), _stream())
+    _check(st, "ar_attn_fwd")
+    return o, lse_t
+
+
+def bwd(q, k, v, o, dO, lse, window: int, eps: float = 1e-6, scale=None, dq=None, dk=None, dv=None,
+        workspace=None):
+    """dq, dk, dv of the forward above, given the upstream gradient dO."""
+    _check_inputs(q, k, v, o, dO)
+    B, T, H, D = q.shape
+    if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, H, T)):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, H, T]")
+    if scale is None:
+        scale = default_scale(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device=q.device)
+    st = lib().ar_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                           B, T, H, D, int(window), float(eps), float(scale), _ptr(workspace), workspace.numel(),
+                           _stream())
+    _check(st, "ar_attn_bwd")
+    return dq, dk, dv
+
+
+def sync_status():
+    """Synchronise the current stream and raise if a kernel gave up a wait."""
+    _check(lib().ar_attn_sync_status(_stream()), "ar_attn_sync_status")
+
+
+def unmasked_pairs(T: int, window: int) -> int:
+    return int(lib().ar_attn_unmasked_pairs(int(T), int(window)))
+
+
+KERNELS = ("fwd_prep", "fwd", "bwd_prep", "bwd", "dq_post")
+
+
+def timing_enable(on: bool = True):
+    """Start (clearing earlier records) or stop per-kernel event timing."""
+    _check(lib().ar_attn_timing_enable(1 if on else 0), "ar_attn_timing_enable")
+
+
+def timing_read():
+    """{kernel: (total_ms, launches)} recorded since timing_enable(True)."""
+    ms = (ctypes.c_double * len(KERNELS))()
+    n = (ctypes.c_longlong * len(KERNELS))()
+    _check(lib().ar_attn_timing_read(ms, n), "ar_attn_timing_read")
+    return {k: (ms[i], n[i]) for i, k in enumerate(KERNELS)}

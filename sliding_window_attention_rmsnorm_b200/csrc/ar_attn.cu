@@ -1,0 +1,397 @@
+// Host side of libar_attn.so: argument validation, workspace layout, TMA
+// tensor maps and kernel launches behind the C ABI declared in ar_attn.h.
+#include "ar_attn.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cctype>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "aux.cuh"
+#include "bwd.cuh"
+#include "fwd.cuh"
+#include "sm100.cuh"
+
+namespace {
+
+constexpr int kD = 128;
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int status = AR_OK;  // AR_OK or AR_ERR_DEVICE / AR_ERR_CUDA
+  int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Checks the current device once: compute capability 10.0, kernel attributes.
+int device_setup(int* sms_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return AR_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return AR_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    d.ready = true;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      d.status = AR_ERR_CUDA;
+    } else if (major != 10 || minor != 0) {
+      d.status = AR_ERR_DEVICE;
+    } else if (cudaFuncSetAttribute(ar::fwd::fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    ar::fwd::kSmemBytes) != cudaSuccess ||
+               cudaFuncSetAttribute(ar::bwd::bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    ar::bwd::kSmemBytes) != cudaSuccess) {
+      d.status = AR_ERR_CUDA;
+    }
+    if (!g_encode && d.status == AR_OK) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        d.status = AR_ERR_CUDA;
+      else
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  if (d.status != AR_OK) {
+    cudaGetLastError();  // clear any sticky-free error left by the attribute calls
+    return d.status;
+  }
+  *sms_out = d.sms;
+  return AR_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int check_shape(int B, int T, int H, int D) {
+  if (B <= 0 || T <= 0 || H <= 0) return AR_ERR_SHAPE;
+  if (D != kD) return AR_ERR_UNSUPPORTED;
+  const long long T_pad = (T + 127LL) / 128 * 128;
+  // all element indices must fit comfortably in 63 bits and unit counts in int
+  if ((long long)B * H * T_pad > (1LL << 31) / 2) return AR_ERR_SHAPE;
+  if ((long long)B * T * H * kD > (1LL << 40)) return AR_ERR_SHAPE;
+  return AR_OK;
+}
+
+int check_args(float eps, float scale) {
+  if (!std::isfinite(eps) || eps < 0.f) return AR_ERR_ARG;
+  if (!std::isfinite(scale) || scale <= 0.f) return AR_ERR_ARG;
+  return AR_OK;
+}
+
+int effective_window(int window, int T) { return (window < 0 || window >= T - 1) ? T : window; }
+
+// [B, T, H, 128] bf16 viewed as a 4-D tensor (d, h, t, b); boxes of 64 x 1 x 128 x 1
+// land as 128 rows of 128 bytes with the 128-byte swizzle the MMA descriptors expect.
+int make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
+  cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)T * H * kD * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? AR_OK : AR_ERR_CUDA;
+}
+
+size_t vec_bytes(int B, int T, int H) {
+  const size_t T_pad = round_up((size_t)T, 128);
+  return round_up((size_t)B * H * T_pad * sizeof(float), 256);
+}
+
+// ---------------------------------------------------------------- kernel timing
+struct TimingRec {
+  int kind;
+  cudaEvent_t a, b;
+};
+struct Timing {
+  std::mutex mu;
+  bool on = false;
+  std::vector<TimingRec> recs;
+  std::vector<cudaEvent_t> pool;
+} g_timing;
+
+cudaEvent_t timing_event() {
+  if (!g_timing.pool.empty()) {
+    cudaEvent_t e = g_timing.pool.back();
+    g_timing.pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Brackets one launch with events when timing is enabled.
+struct KernelTimer {
+  int kind;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  KernelTimer(int kind_, cudaStream_t s_) : kind(kind_), s(s_) {
+    std::lock_guard<std::mutex> lock(g_timing.mu);
+    if (!g_timing.on) return;
+    a = timing_event();
+    if (a) cudaEventRecord(a, s);
+  }
+  void stop() {
+    if (!a) return;
+    std::lock_guard<std::mutex> lock(g_timing.mu);
+    cudaEvent_t b = timing_event();
+    if (!b) return;
+    cudaEventRecord(b, s);
+    g_timing.recs.push_back({kind, a, b});
+    a = nullptr;
+  }
+};
+
+int prep_grid(long long rows, int sms) {
+  long long blocks = (rows + 15) / 16;  // 16 rows per 256-thread block
+  const long long cap = (long long)sms * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return (int)blocks;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ar_attn_fwd_workspace_bytes(int B, int T, int H, int D) {
+  if (check_shape(B, T, H, D) != AR_OK) return 0;
+  return vec_bytes(B, T, H);
+}
+
+size_t ar_attn_bwd_workspace_bytes(int B, int T, int H, int D) {
+  if (check_shape(B, T, H, D) != AR_OK) return 0;
+  return round_up((size_t)B * T * H * kD * sizeof(float), 256) + 3 * vec_bytes(B, T, H);
+}
+
+int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T, int H, int D,
+                int window, float eps, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse) return AR_ERR_NULL;
+  int st = check_shape(B, T, H, D);
+  if (st != AR_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return AR_ERR_ALIGN;
+  if ((st = check_args(eps, scale)) != AR_OK) return st;
+  const size_t need = ar_attn_fwd_workspace_bytes(B, T, H, D);
+  if (workspace && workspace_bytes < need) return AR_ERR_WORKSPACE;
+  if (workspace && !aligned(workspace, 256)) return AR_ERR_ALIGN;
+  int sms = 0;
+  if ((st = device_setup(&sms)) != AR_OK) return st;
+
+  CUtensorMap tq, tk, tv;
+  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, H) != AR_OK || make_map(&tv, v, B, T, H) != AR_OK)
+    return AR_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  if (!ws && cudaMallocAsync(&ws, need, s) != cudaSuccess) return AR_ERR_CUDA;
+
+  const int T_pad = (T + 127) / 128 * 128;
+  float* ck = static_cast<float*>(ws);
+  const long long rows = (long long)B * T * H;
+  const float cscale = scale * 1.4426950408889634f;
+  {
+    KernelTimer t(AR_KERNEL_FWD_PREP, s);
+    ar::fwd_prep_kernel<<<prep_grid(rows, sms), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(k), ck, B, T, H,
+                                                              T_pad, eps, cscale);
+    t.stop();
+  }
+  ar::FwdParams p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.ck = ck;
+  p.B = B;
+  p.T = T;
+  p.H = H;
+  p.T_pad = T_pad;
+  p.w = effective_window(window, T);
+  p.nqp = (T + 255) / 256;
+  p.n_units = B * H * p.nqp;
+  p.eps = eps;
+  const int grid = p.n_units < sms ? p.n_units : sms;
+  {
+    KernelTimer t(AR_KERNEL_FWD, s);
+    ar::fwd::fwd_kernel<<<grid, ar::fwd::kThreads, ar::fwd::kSmemBytes, s>>>(tq, tk, tv, p);
+    t.stop();
+  }
+  cudaError_t e = cudaGetLastError();
+  if (!workspace) cudaFreeAsync(ws, s);
+  return e == cudaSuccess ? AR_OK : AR_ERR_CUDA;
+}
+
+int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                void* dq, void* dk, void* dv, int B, int T, int H, int D, int window, float eps, float scale,
+                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return AR_ERR_NULL;
+  int st = check_shape(B, T, H, D);
+  if (st != AR_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
+    return AR_ERR_ALIGN;
+  if ((st = check_args(eps, scale)) != AR_OK) return st;
+  const size_t need = ar_attn_bwd_workspace_bytes(B, T, H, D);
+  if (workspace && workspace_bytes < need) return AR_ERR_WORKSPACE;
+  if (workspace && !aligned(workspace, 256)) return AR_ERR_ALIGN;
+  int sms = 0;
+  if ((st = device_setup(&sms)) != AR_OK) return st;
+
+  CUtensorMap tq, tk, tv, tdo;
+  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, H) != AR_OK ||
+      make_map(&tv, v, B, T, H) != AR_OK || make_map(&tdo, dO, B, T, H) != AR_OK)
+    return AR_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  if (!ws && cudaMallocAsync(&ws, need, s) != cudaSuccess) return AR_ERR_CUDA;
+
+  const int T_pad = (T + 127) / 128 * 128;
+  char* w8 = static_cast<char*>(ws);
+  float* dq_acc = reinterpret_cast<float*>(w8);
+  const size_t acc_bytes = round_up((size_t)B * T * H * kD * sizeof(float), 256);
+  const size_t vb = vec_bytes(B, T, H);
+  float* lse2 = reinterpret_cast<float*>(w8 + acc_bytes);
+  float* delta = reinterpret_cast<float*>(w8 + acc_bytes + vb);
+  float* rq = reinterpret_cast<float*>(w8 + acc_bytes + 2 * vb);
+  const long long rows = (long long)B * T * H;
+
+  {
+    KernelTimer t(AR_KERNEL_BWD_PREP, s);
+    ar::bwd_prep_kernel<<<prep_grid(rows, sms), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(o),
+        static_cast<const __nv_bfloat16*>(dO), lse, lse2, delta, rq, dq_acc, B, T, H, T_pad, eps);
+    t.stop();
+  }
+  ar::BwdParams p;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dq_acc = dq_acc;
+  p.lse2 = lse2;
+  p.delta = delta;
+  p.rq = rq;
+  p.B = B;
+  p.T = T;
+  p.H = H;
+  p.T_pad = T_pad;
+  p.w = effective_window(window, T);
+  p.nk = (T + 127) / 128;
+  p.n_units = B * H * p.nk;
+  p.eps = eps;
+  p.scale = scale;
+  const int grid = p.n_units < sms ? p.n_units : sms;
+  {
+    KernelTimer t(AR_KERNEL_BWD, s);
+    ar::bwd::bwd_kernel<<<grid, ar::bwd::kThreads, ar::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
+    t.stop();
+  }
+  {
+    KernelTimer t(AR_KERNEL_DQ_POST, s);
+    ar::dq_post_kernel<<<prep_grid(rows, sms), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q), dq_acc,
+                                                             static_cast<__nv_bfloat16*>(dq), B, T, H, eps);
+    t.stop();
+  }
+  cudaError_t e = cudaGetLastError();
+  if (!workspace) cudaFreeAsync(ws, s);
+  return e == cudaSuccess ? AR_OK : AR_ERR_CUDA;
+}
+
+int ar_attn_sync_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return AR_ERR_CUDA;
+  int flag = 0;
+  if (cudaMemcpyFromSymbol(&flag, ar::g_status, sizeof(int)) != cudaSuccess) return AR_ERR_CUDA;
+  if (flag != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(ar::g_status, &zero, sizeof(int)) != cudaSuccess) return AR_ERR_CUDA;
+    return AR_ERR_TIMEOUT;
+  }
+  return AR_OK;
+}
+
+const char* ar_attn_strerror(int status) {
+  switch (status) {
+    case AR_OK: return "ok";
+    case AR_ERR_NULL: return "a required pointer is NULL";
+    case AR_ERR_SHAPE: return "invalid shape (B, T, H must be positive and within index range)";
+    case AR_ERR_UNSUPPORTED: return "unsupported head dimension (only D = 128)";
+    case AR_ERR_ALIGN: return "misaligned pointer (tensors need 16-byte, workspace 256-byte alignment)";
+    case AR_ERR_ARG: return "invalid eps or scale (eps >= 0, scale > 0, both finite)";
+    case AR_ERR_DEVICE: return "current device is not a compute capability 10.0 (B200) GPU";
+    case AR_ERR_CUDA: return "a CUDA runtime call failed";
+    case AR_ERR_TIMEOUT: return "a device-side wait timed out; results of the affected call are invalid";
+    case AR_ERR_WORKSPACE: return "workspace smaller than the required size";
+    default: return "unknown status";
+  }
+}
+
+int ar_attn_layer_window(int layer, int n_layer, int seq_len, const char* pattern) {
+  if (!pattern) return AR_ERR_NULL;
+  const size_t len = std::strlen(pattern);
+  if (len == 0 || n_layer <= 0 || seq_len <= 0 || layer < 0 || layer >= n_layer) return AR_ERR_ARG;
+  if (layer == n_layer - 1) return seq_len;
+  const char c = (char)std::toupper((unsigned char)pattern[layer % len]);
+  if (c == 'L') return seq_len;
+  if (c == 'S') return seq_len / 2;
+  return AR_ERR_ARG;
+}
+
+int ar_attn_timing_enable(int on) {
+  std::lock_guard<std::mutex> lock(g_timing.mu);
+  if (on) {
+    for (auto& r : g_timing.recs) {
+      g_timing.pool.push_back(r.a);
+      g_timing.pool.push_back(r.b);
+    }
+    g_timing.recs.clear();
+  }
+  g_timing.on = on != 0;
+  return AR_OK;
+}
+
+int ar_attn_timing_read(double* ms, long long* count) {
+  std::lock_guard<std::mutex> lock(g_timing.mu);
+  double acc[AR_KERNEL_KINDS] = {0, 0, 0, 0, 0};
+  long long n[AR_KERNEL_KINDS] = {0, 0, 0, 0, 0};
+  int st = AR_OK;
+  for (auto& r : g_timing.recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) {
+      st = AR_ERR_CUDA;
+    } else if (r.kind >= 0 && r.kind < AR_KERNEL_KINDS) {
+      acc[r.kind] += t;
+      n[r.kind] += 1;
+    }
+    g_timing.pool.push_back(r.a);
+    g_timing.pool.push_back(r.b);
+  }
+  g_timing.recs.clear();
+  for (int i = 0; i < AR_KERNEL_KINDS; ++i) {
+    if (ms) ms[i] = acc[i];
+    if (count) count[i] = n[i];
+  }
+  return st;
+}
+
+long long ar_attn_unmasked_pairs(int T, int window) {
+  if (T <= 0) return 0;
+  const long long w = (window < 0 || window >= T - 1) ? (long long)T : (long long)window;
+  // rows i <= w see i + 1 keys, the others w + 1
+  const long long n1 = (w + 1 < T) ? (w + 1) : T;
+  long long total = n1 * (n1 + 1) / 2;
+  total += (long long)(T - n1) * (w + 1);
+  return total;
+}
+
+}  // extern "C"

@@ -1,0 +1,137 @@
+// Memory-bound passes around the two attention kernels.  One 128-element row
+// (one token of one head) is handled by 16 lanes, 8 elements (16 bytes) each.
+//
+//   fwd_prep  : ck[bh, t] = rk_t * scale * log2(e), rk_t = 1/sqrt(mean_d k_td^2 + eps)
+//   bwd_prep  : delta[bh, t] = sum_d dO_td o_td  (FlashAttention's backward pre-pass),
+//               rq[bh, t]    = 1/sqrt(mean_d q_td^2 + eps),
+//               lse2[bh, t]  = lse[bh, t] * log2(e), and dq_acc[t] = 0
+//   dq_post   : dq = rq (dqhat - qhat (dqhat . qhat) / D), qhat = rq q  (RMSNorm backward)
+// The [B*H, T_pad] vectors are zero on the padding t >= T so that every tile
+// of 128 entries can be copied whole.
+#pragma once
+#include "sm100.cuh"
+
+namespace ar {
+
+__device__ __forceinline__ float half_warp_sum(float v) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    f[2 * e] = bf16lo(w[e]);
+    f[2 * e + 1] = bf16hi(w[e]);
+  }
+}
+
+// Rows are visited in memory order (b, t, h); row r is token t = (r / H) % T of
+// head (b, h).
+__global__ void fwd_prep_kernel(const __nv_bfloat16* __restrict__ k, float* __restrict__ ck, int B, int T, int H,
+                                int T_pad, float eps, float cscale) {
+  const long long rows = (long long)B * T * H;
+  const int sub = threadIdx.x & 15;
+  const long long gstride = (long long)gridDim.x * (blockDim.x / 16);
+  for (long long r = (long long)blockIdx.x * (blockDim.x / 16) + threadIdx.x / 16; r < rows; r += gstride) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(k + r * 128) + sub);
+    float f[8];
+    unpack8(u, f);
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+    ss = half_warp_sum(ss);
+    if (sub == 0) {
+      const int h = (int)(r % H);
+      const long long bt = r / H;
+      const int t = (int)(bt % T), b = (int)(bt / T);
+      ck[((long long)b * H + h) * T_pad + t] = rsqrtf(ss * (1.0f / 128.0f) + eps) * cscale;
+    }
+  }
+  // padding entries
+  const long long pads = (long long)B * H * (T_pad - T);
+  for (long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x; x < pads; x += (long long)gridDim.x * blockDim.x) {
+    const long long bh = x / (T_pad - T);
+    const int t = T + (int)(x % (T_pad - T));
+    ck[bh * T_pad + t] = 0.f;
+  }
+}
+
+__global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ o,
+                                const __nv_bfloat16* __restrict__ dO, const float* __restrict__ lse,
+                                float* __restrict__ lse2, float* __restrict__ delta, float* __restrict__ rq,
+                                float* __restrict__ dq_acc, int B, int T, int H, int T_pad, float eps) {
+  const long long rows = (long long)B * T * H;
+  const int sub = threadIdx.x & 15;
+  const long long gstride = (long long)gridDim.x * (blockDim.x / 16);
+  const float kLog2e = 1.4426950408889634f;
+  for (long long r = (long long)blockIdx.x * (blockDim.x / 16) + threadIdx.x / 16; r < rows; r += gstride) {
+    float fq[8], fo[8], fd[8];
+    unpack8(__ldg(reinterpret_cast<const uint4*>(q + r * 128) + sub), fq);
+    unpack8(__ldg(reinterpret_cast<const uint4*>(o + r * 128) + sub), fo);
+    unpack8(__ldg(reinterpret_cast<const uint4*>(dO + r * 128) + sub), fd);
+    float ss = 0.f, dl = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      ss = fmaf(fq[e], fq[e], ss);
+      dl = fmaf(fo[e], fd[e], dl);
+    }
+    ss = half_warp_sum(ss);
+    dl = half_warp_sum(dl);
+    float4* z = reinterpret_cast<float4*>(dq_acc + r * 128) + 2 * sub;
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (sub == 0) {
+      const int h = (int)(r % H);
+      const long long bt = r / H;
+      const int t = (int)(bt % T), b = (int)(bt / T);
+      const long long bh = (long long)b * H + h;
+      delta[bh * T_pad + t] = dl;
+      rq[bh * T_pad + t] = rsqrtf(ss * (1.0f / 128.0f) + eps);
+      lse2[bh * T_pad + t] = lse[bh * T + t] * kLog2e;
+    }
+  }
+  const long long pads = (long long)B * H * (T_pad - T);
+  for (long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x; x < pads; x += (long long)gridDim.x * blockDim.x) {
+    const long long bh = x / (T_pad - T);
+    const int t = T + (int)(x % (T_pad - T));
+    delta[bh * T_pad + t] = 0.f;
+    rq[bh * T_pad + t] = 0.f;
+    lse2[bh * T_pad + t] = 0.f;
+  }
+}
+
+__global__ void dq_post_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ dq_acc,
+                               __nv_bfloat16* __restrict__ dq, int B, int T, int H, float eps) {
+  const long long rows = (long long)B * T * H;
+  const int sub = threadIdx.x & 15;
+  const long long gstride = (long long)gridDim.x * (blockDim.x / 16);
+  for (long long r = (long long)blockIdx.x * (blockDim.x / 16) + threadIdx.x / 16; r < rows; r += gstride) {
+    float fq[8];
+    unpack8(__ldg(reinterpret_cast<const uint4*>(q + r * 128) + sub), fq);
+    const float4* g4 = reinterpret_cast<const float4*>(dq_acc + r * 128) + 2 * sub;
+    const float4 ga = __ldcs(g4), gb = __ldcs(g4 + 1);
+    const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+    float ss = 0.f, gq = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      ss = fmaf(fq[e], fq[e], ss);
+      gq = fmaf(g[e], fq[e], gq);
+    }
+    ss = half_warp_sum(ss);
+    gq = half_warp_sum(gq);
+    const float r_ = rsqrtf(ss * (1.0f / 128.0f) + eps);
+    // dq = r (g - qhat (g.qhat)/D) with qhat = r q  ->  r g - r^3 q (g.q) / D
+    const float c = r_ * r_ * r_ * gq * (1.0f / 128.0f);
+    uint4 out;
+    out.x = pack_bf16(r_ * g[0] - c * fq[0], r_ * g[1] - c * fq[1]);
+    out.y = pack_bf16(r_ * g[2] - c * fq[2], r_ * g[3] - c * fq[3]);
+    out.z = pack_bf16(r_ * g[4] - c * fq[4], r_ * g[5] - c * fq[5]);
+    out.w = pack_bf16(r_ * g[6] - c * fq[6], r_ * g[7] - c * fq[7]);
+    reinterpret_cast<uint4*>(dq + r * 128)[sub] = out;
+  }
+}
+
+}  // namespace ar

@@ -1,0 +1,434 @@
+// Fused QK-RMSNorm + band-limited causal attention, forward, for sm_100a.
+//
+// Computes, per head, o_i = sum_j softmax_j(s_ij) v_j and lse_i over the keys
+// visible to query i (0 <= i - j <= w), with s_ij = scale * qhat_i . khat_j and
+// qhat = q / rms(q), khat = k / rms(k) (parameter-free RMSNorm).  Sources:
+// "autoresearch" README (gitee), section 7.3 (norm(q), norm(k) before the
+// attention product) and sections 5.2.1-5.2.2 (FlashAttention-3 call with
+// window_size = (w, 0), "SSSL" window pattern).
+//
+// The norm is folded into the logits as a rank-1 scale: the tensor core
+// multiplies the raw bf16 q and k, and the softmax warps apply
+// rq_i * (rk_j * scale * log2 e), where rq_i comes from the Q tile in shared
+// memory and rk_j from a per-key pre-pass (`ck`).  q and k are never rounded
+// after normalisation.
+//
+// CTA organisation (persistent, one CTA per SM, 320 threads):
+//   warps 0-3  softmax warpgroup 0: query tile 0 (rows r0..r0+127), one row per thread
+//   warps 4-7  softmax warpgroup 1: query tile 1 (rows r0+128..r0+255)
+//   warp 8     TMA producer: Q tiles, K and V tiles (2 stages each) and ck
+//   warp 9     MMA issuer: S_k = Q_k K^T into TMEM, O_k += P_k V with P_k read from TMEM
+// TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P_k (bf16
+// pairs) overwrites the first 64 columns of S_k.  The MMA issue order
+// S0 S1 | PV0 S0' PV1 S1' | ... lets one warpgroup's softmax run while the
+// tensor core works for the other.
+// Only key tiles that intersect the band of a query tile are visited, in
+// descending order from the diagonal tile.  Output rescaling is lazy: the
+// running max is raised only when it grows by more than 2^8.
+#pragma once
+#include "sm100.cuh"
+
+namespace ar {
+
+struct FwdParams {
+  __nv_bfloat16* o;  // [B, T, H, 128]
+  float* lse;        // [B, H, T]
+  const float* ck;   // [B*H, T_pad]: rk_j * scale * log2(e), 0 on padding
+  int B, T, H, T_pad;
+  int w;             // left window (w >= T means full causal)
+  int nqp;           // query-tile pairs per head = ceil(T / 256)
+  int n_units;       // B * H * nqp
+  float eps;
+};
+
+namespace fwd {
+constexpr int kThreads = 384;
+// Launch budget 168 registers x 384 threads; warpgroup 2 (TMA, MMA, 2 idle
+// warps) drops to 104 so warpgroups 0-1 can rise to 200: 256*200 + 128*104 = 168*384.
+constexpr int kRegsLow = 104, kRegsHigh = 200;
+static_assert(256 * kRegsHigh + 128 * kRegsLow <= 168 * kThreads, "register split exceeds the launch budget");
+constexpr uint32_t kTile = 32768, kHalf = 16384;
+constexpr uint32_t kQ = 0, kK = 2 * kTile, kV = 4 * kTile, kCK = 6 * kTile;
+enum {
+  QFULL = 0, QEMPTY, KFULL, KEMPTY = KFULL + 2, VFULL = KEMPTY + 2, VEMPTY = VFULL + 2,
+  SFULL = VEMPTY + 2, PFULL = SFULL + 2, ODONE = PFULL + 2, OFREE = ODONE + 2, FINAL = OFREE + 2, NBAR
+};
+constexpr uint32_t kBar = kCK + 1024;
+constexpr uint32_t kTmemPtr = kBar + NBAR * 8;
+constexpr uint32_t kAbort = kTmemPtr + 4;
+constexpr uint32_t kSmemBytes = kAbort + 4 + 1024;  // + slack for 1024-byte alignment
+
+struct Unit {
+  int bh, b, h;
+  int r0[2];
+  bool valid[2];
+  int lo[2], hi[2];
+  int hi_u, N;
+  __device__ bool in(int k, int n) const { return valid[k] && n >= lo[k] && n <= hi[k]; }
+};
+
+// Units are (head, query-tile pair); heavier pairs (later rows) first, dealt to
+// CTAs in snake order so each CTA's total work is balanced.
+__device__ __forceinline__ int unit_index(int cta, int round, int G) {
+  return round * G + ((round & 1) ? (G - 1 - cta) : cta);
+}
+
+__device__ __forceinline__ Unit decode(const FwdParams& p, int u) {
+  Unit U;
+  const int BH = p.B * p.H;
+  const int qp = p.nqp - 1 - u / BH;
+  U.bh = u % BH;
+  U.b = U.bh / p.H;
+  U.h = U.bh % p.H;
+  for (int k = 0; k < 2; ++k) {
+    U.r0[k] = qp * 256 + 128 * k;
+    U.valid[k] = U.r0[k] < p.T;
+    const int r1 = min(U.r0[k] + 127, p.T - 1);
+    U.lo[k] = max(0, U.r0[k] - p.w) / 128;
+    U.hi[k] = r1 / 128;
+  }
+  U.hi_u = U.valid[1] ? U.hi[1] : U.hi[0];
+  U.N = U.hi_u - U.lo[0] + 1;
+  return U;
+}
+
+__device__ __forceinline__ uint32_t bar_addr(uint32_t sbase, int i) { return sbase + kBar + 8u * i; }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kAbort);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int G = gridDim.x, cta = blockIdx.x;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NBAR; ++i) {
+      uint32_t cnt = 1;
+      if (i == PFULL || i == PFULL + 1 || i == OFREE || i == OFREE + 1) cnt = 128;
+      mbar_init(bar_addr(sbase, i), cnt);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(sbase + kTmemPtr, 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + kTmemPtr);
+
+
+  if (warp >= 8) {
+   regs_dec<kRegsLow>();
+   if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t kv = 0;
+      int uidx = 0;
+      bool ok = true;
+      int last_k_par[2] = {-1, -1}, last_v_par[2] = {-1, -1}, last_q_par = -1;
+      for (int r = 0; ok; ++r) {
+        const int u = unit_index(cta, r, G);
+        if (u >= p.n_units) break;
+        const Unit U = decode(p, u);
+        if (uidx > 0 && !mbar_wait(bar_addr(sbase, QEMPTY), (uidx - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(bar_addr(sbase, QFULL), kTile * (U.valid[1] ? 2 : 1));
+        for (int k = 0; k < 2; ++k)
+          if (U.valid[k])
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_4d(sbase + kQ + k * kTile + hf * kHalf, &tm_q, bar_addr(sbase, QFULL), hf * 64, U.h,
+                          U.r0[k], U.b);
+        last_q_par = uidx & 1;
+        for (int it = 0; it < U.N; ++it, ++kv) {
+          const int n = U.hi_u - it;
+          const int st = kv & 1, ph = (kv >> 1) & 1;
+          if (!mbar_wait(bar_addr(sbase, KEMPTY + st), ph ^ 1, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(bar_addr(sbase, KFULL + st), kTile);
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_4d(sbase + kK + st * kTile + hf * kHalf, &tm_k, bar_addr(sbase, KFULL + st), hf * 64, U.h,
+                        n * 128, U.b);
+          last_k_par[st] = ph;
+          if (!mbar_wait(bar_addr(sbase, VEMPTY + st), ph ^ 1, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(bar_addr(sbase, VFULL + st), kTile + 512);
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_4d(sbase + kV + st * kTile + hf * kHalf, &tm_v, bar_addr(sbase, VFULL + st), hf * 64, U.h,
+                        n * 128, U.b);
+          bulk_load(sbase + kCK + st * 512, p.ck + (size_t)U.bh * p.T_pad + n * 128, 512,
+                    bar_addr(sbase, VFULL + st));
+          last_v_par[st] = ph;
+        }
+        ++uidx;
+      }
+      if (*abort_flag) {
+        // Let copies still in flight land before the CTA's shared memory goes away.
+        volatile int never = 0;
+        for (int s = 0; s < 2; ++s) {
+          if (last_k_par[s] >= 0) mbar_wait(bar_addr(sbase, KFULL + s), last_k_par[s], &never);
+          if (last_v_par[s] >= 0) mbar_wait(bar_addr(sbase, VFULL + s), last_v_par[s], &never);
+        }
+        if (last_q_par >= 0) mbar_wait(bar_addr(sbase, QFULL), last_q_par, &never);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_qk = idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t id_pv = idesc_bf16(128, 128, 0, 1);
+      auto issue_s = [&](int k, int st) {
+        const uint32_t qa = sbase + kQ + k * kTile, ka = sbase + kK + st * kTile;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          mma_ss(tbase + 128 * k, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), id_qk,
+                 kk > 0);
+        }
+      };
+      auto issue_pv = [&](int k, int st, bool acc) {
+        const uint32_t va = sbase + kV + st * kTile;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tbase + 256 + 128 * k, tbase + 128 * k + kk * 8, sdesc_sw128(va + kk * 2048, kHalf, 1024), id_pv,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      uint32_t kv = 0, pcount[2] = {0, 0}, ounits[2] = {0, 0};
+      int uidx = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int u = unit_index(cta, r, G);
+        if (u >= p.n_units) break;
+        const Unit U = decode(p, u);
+        if (!mbar_wait(bar_addr(sbase, QFULL), uidx & 1, abort_flag)) break;
+        {
+          const int st = kv & 1, ph = (kv >> 1) & 1;
+          if (!mbar_wait(bar_addr(sbase, KFULL + st), ph, abort_flag)) break;
+          tc_fence_after();
+          for (int k = 0; k < 2; ++k)
+            if (U.in(k, U.hi_u)) {
+              issue_s(k, st);
+              mma_commit(bar_addr(sbase, SFULL + k));
+            }
+          mma_commit(bar_addr(sbase, KEMPTY + st));
+        }
+        bool first_pv[2] = {true, true};
+        for (int it = 0; it < U.N && ok; ++it) {
+          const int n = U.hi_u - it;
+          const uint32_t kvn = kv + it, kvx = kvn + 1;
+          const int stn = kvn & 1, phn = (kvn >> 1) & 1, stx = kvx & 1, phx = (kvx >> 1) & 1;
+          const bool has_next = it + 1 < U.N;
+          if (!mbar_wait(bar_addr(sbase, VFULL + stn), phn, abort_flag)) { ok = false; break; }
+          if (has_next && !mbar_wait(bar_addr(sbase, KFULL + stx), phx, abort_flag)) { ok = false; break; }
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            if (U.in(k, n)) {
+              if (first_pv[k] && ounits[k] > 0 &&
+                  !mbar_wait(bar_addr(sbase, OFREE + k), (ounits[k] - 1) & 1, abort_flag)) { ok = false; break; }
+              if (!mbar_wait(bar_addr(sbase, PFULL + k), pcount[k] & 1, abort_flag)) { ok = false; break; }
+              ++pcount[k];
+              tc_fence_after();
+              issue_pv(k, stn, !first_pv[k]);
+              first_pv[k] = false;
+            }
+            if (k == 1) mma_commit(bar_addr(sbase, VEMPTY + stn));
+            if (has_next && U.in(k, n - 1)) {
+              tc_fence_after();
+              issue_s(k, stx);
+              mma_commit(bar_addr(sbase, SFULL + k));
+            }
+          }
+          if (ok && has_next) mma_commit(bar_addr(sbase, KEMPTY + stx));
+        }
+        if (!ok) break;
+        for (int k = 0; k < 2; ++k)
+          if (U.valid[k]) {
+            mma_commit(bar_addr(sbase, ODONE + k));
+            ++ounits[k];
+          }
+        mma_commit(bar_addr(sbase, QEMPTY));
+        kv += U.N;
+        ++uidx;
+      }
+      // Drain: every MMA issued by this thread completes before TMEM is freed.
+      mma_commit(bar_addr(sbase, FINAL));
+      volatile int never = 0;
+      mbar_wait(bar_addr(sbase, FINAL), 0, &never);
+    }
+  }
+  } else {
+   regs_inc<kRegsHigh>();
+   {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int k = warp / 4;
+    const int row = threadIdx.x & 127;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tbase + 128 * k + lane_off;
+    const uint32_t tO = tbase + 256 + 128 * k + lane_off;
+    const float kLn2 = 0.69314718055994531f;
+    uint32_t scount = 0, ecount = 0, kv = 0;
+    int uidx = 0;
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      const int u = unit_index(cta, r, G);
+      if (u >= p.n_units) break;
+      const Unit U = decode(p, u);
+      if (!(k ? U.valid[1] : U.valid[0])) {
+        kv += U.N;
+        ++uidx;
+        continue;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, QFULL), uidx & 1, abort_flag))) break;
+      // this warpgroup's query tile, as scalars (no dynamic indexing into U)
+      const int r0k = k ? U.r0[1] : U.r0[0];
+      const int lok = k ? U.lo[1] : U.lo[0];
+      const int hik = k ? U.hi[1] : U.hi[0];
+      const int i = r0k + row;
+      // rq_i from this thread's own Q row in shared memory.
+      float rq;
+      {
+        float ss[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t qa = sbase + kQ + k * kTile;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = lds128(qa + hf * kHalf + sw128(row, c));
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float a = bf16lo(w4[e]), b2 = bf16hi(w4[e]);
+              ss[e] = fmaf(a, a, ss[e]);
+              ss[e] = fmaf(b2, b2, ss[e]);
+            }
+          }
+        rq = rsqrtf((ss[0] + ss[1] + ss[2] + ss[3]) * (1.0f / 128.0f) + p.eps);
+      }
+      float m = -INFINITY, l = 0.f;
+      bool first = true;
+      for (int n = hik; n >= lok; --n) {
+        const uint32_t kvn = kv + (U.hi_u - n);
+        const int stn = kvn & 1, phn = (kvn >> 1) & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, SFULL + k), scount & 1, abort_flag))) { ok = false; break; }
+        ++scount;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VFULL + stn), phn, abort_flag))) { ok = false; break; }
+        tc_fence_after();
+        uint32_t s[128];
+        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+        tmem_wait_ld();
+        const float4* ck4 = reinterpret_cast<const float4*>(smem + kCK + stn * 512);
+        const bool masked = (n * 128 + 127 > r0k) || (r0k + 127 - n * 128 > p.w);
+        float mx[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+#pragma unroll
+        for (int j4 = 0; j4 < 32; ++j4) {
+          const float4 c4 = ck4[j4];
+          const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = j4 * 4 + e;
+            float x = __uint_as_float(s[j]) * cc[e];
+            if (masked) {
+              const int ja = n * 128 + j;
+              if (ja > i || i - ja > p.w) x = -INFINITY;
+            }
+            s[j] = __float_as_uint(x);
+            mx[j & 7] = fmaxf(mx[j & 7], x);
+          }
+        }
+        const float mrow = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float mnew = fmaxf(m, mrow * rq);
+        if (first) {
+          m = mnew;
+          first = false;
+        } else {
+          const bool need = mnew > m + 8.0f;
+          if (__any_sync(0xffffffffu, need)) {
+            const float alpha = need ? ex2(m - mnew) : 1.0f;
+            if (need) {
+              m = mnew;
+              l *= alpha;
+            }
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t ov[32];
+              tmem_ld32(tO + 32 * c, ov);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+              tmem_st32(tO + 32 * c, ov);
+            }
+            tmem_wait_st();
+          }
+        }
+        const float negm = -m;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2(fmaf(__uint_as_float(s[32 * c + 2 * e]), rq, negm));
+            const float p1 = ex2(fmaf(__uint_as_float(s[32 * c + 2 * e + 1]), rq, negm));
+            ls[e & 3] += p0 + p1;
+            pk[e] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tS + 16 * c, pk);
+        }
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_addr(sbase, PFULL + k));
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, ODONE + k), ecount & 1, abort_flag))) break;
+      ++ecount;
+      tc_fence_after();
+      const float inv = 1.0f / l;
+      __nv_bfloat16* orow = p.o + (((size_t)U.b * p.T + i) * p.H + U.h) * 128;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(tO + 32 * c, ov);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
+        if (i < p.T) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_addr(sbase, OFREE + k));
+      if (i < p.T) p.lse[(size_t)U.bh * p.T + i] = (m + log2f(l)) * kLn2;
+      kv += U.N;
+      ++uidx;
+    }
+  }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+}  // namespace fwd
+}  // namespace ar

@@ -1,0 +1,55 @@
+"""Per-layer driver of the attention core for an "SSSL" layer stack.
+
+The window of each layer comes from the library (ar_attn_layer_window): the
+pattern repeats over layers, 'S' is half the sequence length, 'L' the full
+length, and the last layer is always global ("autoresearch" README on gitee,
+section 5.2.2; web3.okx.com review, paragraph on the SSSL pattern).  Layers here
+take independent inputs, as in the stacked workloads this core is measured on.
+"""
+from . import attn
+
+
+def layer_windows(n_layer: int, seq_len: int, pattern: str = "SSSL"):
+    out = []
+    for layer in range(n_layer):
+        w = attn.lib().ar_attn_layer_window(layer, n_layer, seq_len, pattern.encode())
+        if w < 0:
+            raise ValueError("invalid window pattern %r" % pattern)
+        out.append(w)
+    return out
+
+
+class Stack:
+    """Forward and backward of every layer, enqueued back to back on one stream.
+
+    layers: list of dicts with bf16 CUDA tensors q, k, v, dO [B, T, H, 128].
+    Outputs (o, lse, dq, dk, dv) and scratch are allocated once and reused.
+    """
+
+    def __init__(self, layers, pattern: str = "SSSL", eps: float = 1e-6, scale=None):
+        import torch
+        self.layers = layers
+        B, T, H, D = layers[0]["q"].shape
+        self.windows = layer_windows(len(layers), T, pattern)
+        self.eps, self.scale = eps, scale
+        dev = layers[0]["q"].device
+        self.out = [dict(o=torch.empty_like(L["q"]),
+                         lse=torch.empty((B, H, T), dtype=torch.float32, device=dev),
+                         dq=torch.empty_like(L["q"]), dk=torch.empty_like(L["q"]),
+                         dv=torch.empty_like(L["q"])) for L in layers]
+        self.ws_fwd = torch.empty(attn.fwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device=dev)
+        self.ws_bwd = torch.empty(attn.bwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device=dev)
+
+    def forward(self):
+        for L, O, w in zip(self.layers, self.out, self.windows):
+            attn.fwd(L["q"], L["k"], L["v"], w, self.eps, self.scale, out=O["o"], lse=O["lse"],
+                     workspace=self.ws_fwd)
+
+    def backward(self):
+        for L, O, w in zip(reversed(self.layers), reversed(self.out), reversed(self.windows)):
+            attn.bwd(L["q"], L["k"], L["v"], O["o"], L["dO"], O["lse"], w, self.eps, self.scale,
+                     dq=O["dq"], dk=O["dk"], dv=O["dv"], workspace=self.ws_bwd)
+
+    def step(self):
+        self.forward()
+        self.backward()

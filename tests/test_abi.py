@@ -1,0 +1,118 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared
+symbol, and its host-side logic (argument validation, window rule, pair
+count, workspace sizes) behaves as the header states.
+
+Validation tests always include at least one invalid argument that the
+library checks before touching the device, so no kernel is ever launched on
+the placeholder pointers used here.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from oracle import oracle as orc
+from oracle.stack import layer_windows as oracle_windows
+from sliding_window_attention_rmsnorm_b200 import attn, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return attn.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "ar_attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ar_attn_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("ar_attn_fwd", "ar_attn_bwd", "ar_attn_bwd_workspace_bytes", "ar_attn_sync_status",
+              "ar_attn_strerror"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for n in declared_functions():
+        assert hasattr(L, n), n
+
+
+def test_strerror(L):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9, 12345):
+        assert attn.strerror(code)
+    assert attn.strerror(0) == "ok"
+
+
+def test_layer_window_matches_oracle_rule(L):
+    for n_layer in (1, 2, 4, 8, 12, 13):
+        for T in (256, 2048, 8192):
+            for pat in ("SSSL", "L", "SL", "SLLL", "SSSS", "sssl"):
+                mine = [L.ar_attn_layer_window(l, n_layer, T, pat.encode()) for l in range(n_layer)]
+                assert mine == oracle_windows(n_layer, T, pat), (n_layer, T, pat)
+    assert L.ar_attn_layer_window(0, 8, 2048, b"SXSL") == 1024
+    assert L.ar_attn_layer_window(1, 8, 2048, b"SXSL") == -5
+    assert L.ar_attn_layer_window(8, 8, 2048, b"SSSL") == -5
+    assert L.ar_attn_layer_window(0, 8, 2048, None) == -1
+
+
+def test_unmasked_pairs_matches_oracle(L):
+    for T in (1, 2, 7, 128, 129, 200, 256, 2048):
+        for w in (-1, 0, 1, 5, 127, 128, 1024, T - 2, T - 1, T, 5 * T):
+            assert L.ar_attn_unmasked_pairs(T, w) == orc.unmasked_pairs(T, w if w < T - 1 else -1), (T, w)
+
+
+def test_workspace_sizes(L):
+    B, T, H, D = 8, 2048, 4, 128
+    assert attn.fwd_workspace_bytes(B, T, H, D) == B * H * T * 4
+    assert attn.bwd_workspace_bytes(B, T, H, D) == B * T * H * D * 4 + 3 * B * H * T * 4
+    # ragged T rounds the per-token vectors up to whole 128-token tiles
+    assert attn.fwd_workspace_bytes(1, 200, 1, 128) == 256 * 4
+    assert attn.fwd_workspace_bytes(1, 200, 1, 64) == 0
+    assert attn.bwd_workspace_bytes(0, 200, 1, 128) == 0
+
+
+P16 = 1 << 20  # a 16-byte aligned placeholder address; never dereferenced
+
+
+def fwd_call(L, q=P16, k=P16, v=P16, o=P16, lse=P16, B=1, T=128, H=1, D=128, window=-1, eps=1e-6,
+             scale=0.088, ws=None, ws_bytes=0):
+    vp = ctypes.c_void_p
+    return L.ar_attn_fwd(vp(q), vp(k), vp(v), vp(o), vp(lse), B, T, H, D, window, eps, scale, vp(ws),
+                         ws_bytes, None)
+
+
+def bwd_call(L, ptr=P16, dq=P16, B=1, T=128, H=1, D=128, eps=1e-6, scale=0.088, ws=None, ws_bytes=0):
+    vp = ctypes.c_void_p
+    return L.ar_attn_bwd(vp(ptr), vp(ptr), vp(ptr), vp(ptr), vp(ptr), vp(ptr), vp(dq), vp(ptr), vp(ptr),
+                         B, T, H, D, -1, eps, scale, vp(ws), ws_bytes, None)
+
+
+def test_fwd_argument_errors(L):
+    assert fwd_call(L, q=0) == -1
+    assert fwd_call(L, lse=0) == -1
+    assert fwd_call(L, B=0) == -2
+    assert fwd_call(L, T=-3) == -2
+    assert fwd_call(L, H=0) == -2
+    assert fwd_call(L, D=64) == -3
+    assert fwd_call(L, k=P16 + 8) == -4
+    assert fwd_call(L, eps=-1.0) == -5
+    assert fwd_call(L, eps=float("nan")) == -5
+    assert fwd_call(L, scale=0.0) == -5
+    assert fwd_call(L, scale=float("inf")) == -5
+    assert fwd_call(L, ws=P16, ws_bytes=4) == -9
+    assert fwd_call(L, ws=P16 + 16, ws_bytes=1 << 20) == -4
+
+
+def test_bwd_argument_errors(L):
+    assert bwd_call(L, dq=0) == -1
+    assert bwd_call(L, B=-1) == -2
+    assert bwd_call(L, D=256) == -3
+    assert bwd_call(L, dq=P16 + 4) == -4
+    assert bwd_call(L, scale=-0.5) == -5
+    assert bwd_call(L, ws=P16, ws_bytes=100) == -9

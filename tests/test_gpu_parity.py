@@ -1,0 +1,193 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Every case draws seeded bf16 inputs, runs ar_attn_fwd / ar_attn_bwd on the
+GPU, and compares element by element with the oracle on the same bits:
+  o, dq, dk, dv : max |err| <= 2e-2 and ||err||_2 / ||ref||_2 <= 5e-3
+  lse           : max |err| <= 1e-3
+Small shapes are compared whole (they span several 128-row tiles and a ragged
+tail); the full-size workloads are compared on whole sampled heads, which
+the oracle computes one by one, in the same launch configuration the
+benchmark uses.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as orc
+from oracle.stack import layer_windows as oracle_windows
+from sliding_window_attention_rmsnorm_b200 import attn, build, stack, synth
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, REL_L2, LSE_ABS = 2e-2, 5e-3, 1e-3
+EPS = 1e-6
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+    attn.lib()
+
+
+def run_gpu(x, window, eps=EPS, scale=None, D=128):
+    q, k, v, dO = (x[r].cuda() for r in ("q", "k", "v", "dO"))
+    o, lse = attn.fwd(q, k, v, window, eps, scale)
+    dq, dk, dv = attn.bwd(q, k, v, o, dO, lse, window, eps, scale)
+    attn.sync_status()
+    return {n: t.float().cpu().numpy() for n, t in dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv).items()}
+
+
+def run_oracle(x, window, eps=EPS, scale=None, heads=None):
+    o, lse = orc.attn_fwd(x["q"], x["k"], x["v"], window, eps, scale, heads=heads)
+    g = orc.attn_bwd(x["q"], x["k"], x["v"], x["dO"], window, eps, scale, heads=heads)
+    return dict(o=o, lse=lse, dq=g["dq"], dk=g["dk"], dv=g["dv"])
+
+
+def select(a, name, H, heads):
+    """Restrict an array to the listed flat heads."""
+    if heads is None:
+        return a
+    if name == "lse":
+        B = a.shape[0]
+        return np.stack([a[h // H, h % H] for h in heads])
+    return np.stack([a[h // H, :, h % H] for h in heads])
+
+
+def compare(gpu, ref, H, heads=None, tag=""):
+    for n in ("o", "dq", "dk", "dv", "lse"):
+        a = select(gpu[n], n, H, heads).astype(np.float64)
+        b = select(ref[n], n, H, heads)
+        assert np.isfinite(a).all(), (tag, n, "non-finite")
+        err = np.abs(a - b)
+        if n == "lse":
+            assert err.max() <= LSE_ABS, (tag, n, err.max())
+            continue
+        rel = np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30)
+        assert err.max() <= MAX_ABS, (tag, n, "max abs", err.max())
+        assert rel <= REL_L2, (tag, n, "rel l2", rel)
+
+
+# ------------------------------------------------------------------ whole-tensor parity
+@pytest.mark.parametrize("window", [128, -1])
+def test_small_config_whole(window):
+    """B=1, T=256, H=4: the small workload, sliding (w=128) and full causal."""
+    x = synth.layer_inputs(1, 0 if window > 0 else 1, 1, 256, 4, 128)
+    compare(run_gpu(x, window), run_oracle(x, window), 4, tag="small w=%d" % window)
+
+
+@pytest.mark.parametrize("T,window", [(1, -1), (7, -1), (7, 2), (129, -1), (129, 64), (200, 0),
+                                      (200, 5), (200, 130), (300, 255), (384, 100), (640, 256),
+                                      (1000, 511), (1024, 1023)])
+def test_ragged_and_windows(T, window):
+    B, H = 2, 3
+    x = synth.layer_inputs(7, T, B, T, H, 128)
+    compare(run_gpu(x, window), run_oracle(x, window), H, tag="T=%d w=%d" % (T, window))
+
+
+def test_peaked_logits():
+    """Keys close to their queries push logits towards the +-sqrt(D) bound."""
+    B, T, H = 1, 384, 2
+    x = synth.layer_inputs(9, 0, B, T, H, 128)
+    x["k"] = synth.peaked_keys(x["q"], 9999)
+    for w in (64, -1):
+        compare(run_gpu(x, w), run_oracle(x, w), H, tag="peaked w=%d" % w)
+
+
+def test_other_eps_and_scale():
+    B, T, H = 1, 256, 2
+    x = synth.layer_inputs(11, 0, B, T, H, 128)
+    for eps, scale in ((0.0, 0.05), (1e-2, 0.2)):
+        compare(run_gpu(x, 100, eps, scale), run_oracle(x, 100, eps, scale), H, tag="eps=%g" % eps)
+
+
+# ------------------------------------------------------------------ full-size workloads, sampled heads
+@pytest.mark.parametrize("window", [1024, 2048])
+def test_full_size_layer_sampled_heads(window):
+    """B=8, T=2048, H=4 (S layer: window 1024; L layer: full causal)."""
+    B, T, H = 8, 2048, 4
+    x = synth.layer_inputs(2, 0 if window == 1024 else 3, B, T, H, 128)
+    heads = [0, 13, B * H - 1]
+    compare(run_gpu(x, window), run_oracle(x, window, heads=heads), H, heads, tag="cfg2 w=%d" % window)
+
+
+@pytest.mark.parametrize("window", [4096, 8192])
+def test_long_context_sampled_head(window):
+    """B=2, T=8192, H=4 (window 4096, and full causal)."""
+    B, T, H = 2, 8192, 4
+    x = synth.layer_inputs(4, 0 if window == 4096 else 1, B, T, H, 128)
+    heads = [B * H - 2]
+    compare(run_gpu(x, window), run_oracle(x, window, heads=heads), H, heads, tag="cfg4 w=%d" % window)
+
+
+def test_stack_of_eight_layers_sampled():
+    """The 8-layer SSSL stack (B=8, T=2048, H=4), every layer checked on one head."""
+    B, T, H, n_layer = 8, 2048, 4, 8
+    layers = [{r: t.cuda() for r, t in synth.layer_inputs(3, l, B, T, H, 128).items()} for l in range(n_layer)]
+    st = stack.Stack(layers, "SSSL", EPS)
+    assert st.windows == oracle_windows(n_layer, T, "SSSL")
+    st.step()
+    attn.sync_status()
+    for l in range(n_layer):
+        head = [(5 * l + 3) % (B * H)]
+        xc = {r: t.cpu() for r, t in layers[l].items()}
+        gpu = {n: t.float().cpu().numpy() for n, t in st.out[l].items()}
+        compare(gpu, run_oracle(xc, st.windows[l], heads=head), H, head, tag="stack layer %d" % l)
+
+
+def test_twelve_layer_stack_shape_sampled():
+    """Depth-12 stack shape (H=6): layer 0 (S) and layer 11 (forced L) on one head each."""
+    B, T, H = 8, 2048, 6
+    ws = oracle_windows(12, T, "SSSL")
+    for l in (0, 11):
+        x = synth.layer_inputs(5, l, B, T, H, 128)
+        head = [7 * l % (B * H)]
+        compare(run_gpu(x, ws[l]), run_oracle(x, ws[l], heads=head), H, head, tag="cfg5 layer %d" % l)
+
+
+# ------------------------------------------------------------------ closed forms on the GPU
+def test_full_window_equivalence_on_gpu():
+    """window = T-1, T, 10T and -1 all mean full causal: identical tile work."""
+    B, T, H = 2, 384, 2
+    x = synth.layer_inputs(12, 0, B, T, H, 128)
+    outs = [run_gpu(x, w) for w in (T - 1, T, 10 * T, -1)]
+    for o in outs[1:]:
+        for n in ("o", "lse", "dk", "dv"):
+            assert np.array_equal(o[n], outs[0][n]), n
+        np.testing.assert_allclose(o["dq"], outs[0]["dq"], atol=1e-2)
+
+
+def test_window_zero_on_gpu():
+    """w = 0: every query sees only itself, so o = v, dv = dO and dq = dk = 0."""
+    B, T, H = 1, 300, 2
+    x = synth.layer_inputs(13, 0, B, T, H, 128)
+    g = run_gpu(x, 0)
+    assert np.array_equal(g["o"], x["v"].float().numpy())
+    assert np.array_equal(g["dv"], x["dO"].float().numpy())
+    # dS = P (dP - delta) cancels up to fp32 rounding of two different dot products
+    assert np.abs(g["dq"]).max() < 1e-3 and np.abs(g["dk"]).max() < 1e-3
+
+
+def test_lse_bound_on_gpu():
+    B, T, H = 2, 512, 2
+    x = synth.layer_inputs(14, 0, B, T, H, 128)
+    for w in (100, -1):
+        g = run_gpu(x, w)
+        ww = T if w < 0 else w
+        n = np.array([min(i, ww) + 1 for i in range(T)], dtype=np.float64)
+        assert np.all(np.abs(g["lse"] - np.log(n)) <= math.sqrt(128) + 1e-3)
+
+
+def test_masked_positions_zero_gradient_on_gpu():
+    B, T, H, i0, w = 1, 512, 1, 300, 77
+    x = synth.layer_inputs(15, 0, B, T, H, 128)
+    dO = x["dO"].clone()
+    dO[:, torch.arange(T) != i0] = 0
+    x["dO"] = dO
+    g = run_gpu(x, w)
+    outside = [j for j in range(T) if not (i0 - w <= j <= i0)]
+    assert np.all(g["dk"][:, outside] == 0) and np.all(g["dv"][:, outside] == 0)
+    assert np.all(g["dq"][:, np.arange(T) != i0] == 0)
