@@ -54,6 +54,17 @@ int device_setup(int* sms_out) {
                                     ar::bwd::kSmemBytes) != cudaSuccess) {
       d.status = AR_ERR_CUDA;
     }
+    if (d.status == AR_OK) {
+      // The kernels move registers between warpgroups with setmaxnreg; the split
+      // is sized for exactly 168 registers per thread at launch, so refuse any
+      // other build rather than launch a kernel whose register raise cannot be met.
+      cudaFuncAttributes fa, ba;
+      if (cudaFuncGetAttributes(&fa, ar::fwd::fwd_kernel) != cudaSuccess ||
+          cudaFuncGetAttributes(&ba, ar::bwd::bwd_kernel) != cudaSuccess)
+        d.status = AR_ERR_CUDA;
+      else if (fa.numRegs != ar::fwd::kLaunchRegs || ba.numRegs != ar::bwd::kLaunchRegs)
+        d.status = AR_ERR_CUDA;
+    }
     if (!g_encode && d.status == AR_OK) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;

@@ -45,8 +45,8 @@ namespace fwd {
 constexpr int kThreads = 384;
 // Launch budget 168 registers x 384 threads; warpgroup 2 (TMA, MMA, 2 idle
 // warps) drops to 104 so warpgroups 0-1 can rise to 200: 256*200 + 128*104 = 168*384.
-constexpr int kRegsLow = 104, kRegsHigh = 200;
-static_assert(256 * kRegsHigh + 128 * kRegsLow <= 168 * kThreads, "register split exceeds the launch budget");
+constexpr int kRegsLow = 104, kRegsHigh = 200, kLaunchRegs = 168;
+static_assert(256 * kRegsHigh + 128 * kRegsLow <= kLaunchRegs * kThreads, "register split exceeds the launch budget");
 constexpr uint32_t kTile = 32768, kHalf = 16384;
 constexpr uint32_t kQ = 0, kK = 2 * kTile, kV = 4 * kTile, kCK = 6 * kTile;
 enum {
