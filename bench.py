@@ -39,6 +39,14 @@ WORKLOADS = {
                    name="8-layer SSSL attention stack fwd+bwd, B=8 T=2048 H=4 D=128 (windows 1024/full)"),
     "stack12": dict(config=5, B=8, T=2048, H=6, n_layer=12, pattern="SSSL",
                     name="12-layer SSSL attention stack fwd+bwd, B=8 T=2048 H=6 D=128 (windows 1024/full)"),
+    "layer_s": dict(config=2, B=8, T=2048, H=4, n_layer=1, windows=[1024],
+                    name="single S layer fwd+bwd, B=8 T=2048 H=4 D=128, window 1024"),
+    "layer_l": dict(config=2, B=8, T=2048, H=4, n_layer=1, windows=[2048],
+                    name="single L layer fwd+bwd, B=8 T=2048 H=4 D=128, full causal"),
+    "long_s": dict(config=4, B=2, T=8192, H=4, n_layer=1, windows=[4096],
+                   name="long-context S layer fwd+bwd, B=2 T=8192 H=4 D=128, window 4096"),
+    "long_l": dict(config=4, B=2, T=8192, H=4, n_layer=1, windows=[8192],
+                   name="long-context L layer fwd+bwd, B=2 T=8192 H=4 D=128, full causal"),
 }
 
 
@@ -57,6 +65,8 @@ def parse():
 
 
 def windows_for(wl):
+    if "windows" in wl:
+        return list(wl["windows"])
     from oracle.stack import layer_windows  # pure-Python rule, used only for FLOP counting here
     return layer_windows(wl["n_layer"], wl["T"], wl["pattern"])
 
@@ -204,7 +214,7 @@ def run_ours(args, wl, rank, world, dist):
     B, T, H, L = wl["B"], wl["T"], wl["H"], wl["n_layer"]
     host = [synth.layer_inputs(wl["config"], l, B, T, H, D) for l in range(L)]
     layers = [{r: t.to("cuda", non_blocking=False) for r, t in x.items()} for x in host]
-    st = stack.Stack(layers, wl["pattern"])
+    st = stack.Stack(layers, wl.get("pattern", "SSSL"), windows=wl.get("windows"))
     fwd_f, bwd_f = step_flops(wl)
 
     def barrier():

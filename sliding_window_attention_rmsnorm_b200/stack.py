@@ -26,11 +26,11 @@ class Stack:
     Outputs (o, lse, dq, dk, dv) and scratch are allocated once and reused.
     """
 
-    def __init__(self, layers, pattern: str = "SSSL", eps: float = 1e-6, scale=None):
+    def __init__(self, layers, pattern: str = "SSSL", eps: float = 1e-6, scale=None, windows=None):
         import torch
         self.layers = layers
         B, T, H, D = layers[0]["q"].shape
-        self.windows = layer_windows(len(layers), T, pattern)
+        self.windows = list(windows) if windows is not None else layer_windows(len(layers), T, pattern)
         self.eps, self.scale = eps, scale
         dev = layers[0]["q"].device
         self.out = [dict(o=torch.empty_like(L["q"]),
