@@ -205,8 +205,9 @@ int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
   int sms = 0;
   if ((st = device_setup(&sms)) != AR_OK) return st;
 
-  CUtensorMap tq, tk, tv;
-  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, H) != AR_OK || make_map(&tv, v, B, T, H) != AR_OK)
+  CUtensorMap tq, tk, tv, to;
+  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, H) != AR_OK ||
+      make_map(&tv, v, B, T, H) != AR_OK || make_map(&to, o, B, T, H) != AR_OK)
     return AR_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   void* ws = workspace;
@@ -223,7 +224,6 @@ int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
     t.stop();
   }
   ar::FwdParams p;
-  p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.ck = ck;
   p.B = B;
@@ -237,7 +237,7 @@ int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
   const int grid = p.n_units < sms ? p.n_units : sms;
   {
     KernelTimer t(AR_KERNEL_FWD, s);
-    ar::fwd::fwd_kernel<<<grid, ar::fwd::kThreads, ar::fwd::kSmemBytes, s>>>(tq, tk, tv, p);
+    ar::fwd::fwd_kernel<<<grid, ar::fwd::kThreads, ar::fwd::kSmemBytes, s>>>(tq, tk, tv, to, p);
     t.stop();
   }
   cudaError_t e = cudaGetLastError();

@@ -13,25 +13,27 @@
 // memory and rk_j from a per-key pre-pass (`ck`).  q and k are never rounded
 // after normalisation.
 //
-// CTA organisation (persistent, one CTA per SM, 320 threads):
+// CTA organisation (persistent, one CTA per SM, 384 threads):
 //   warps 0-3  softmax warpgroup 0: query tile 0 (rows r0..r0+127), one row per thread
 //   warps 4-7  softmax warpgroup 1: query tile 1 (rows r0+128..r0+255)
 //   warp 8     TMA producer: Q tiles, K and V tiles (2 stages each) and ck
 //   warp 9     MMA issuer: S_k = Q_k K^T into TMEM, O_k += P_k V with P_k read from TMEM
+//   warps 10-11 idle (their registers go to the softmax warpgroups)
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P_k (bf16
 // pairs) overwrites the first 64 columns of S_k.  The MMA issue order
 // S0 S1 | PV0 S0' PV1 S1' | ... lets one warpgroup's softmax run while the
 // tensor core works for the other.
 // Only key tiles that intersect the band of a query tile are visited, in
 // descending order from the diagonal tile.  Output rescaling is lazy: the
-// running max is raised only when it grows by more than 2^8.
+// running max is raised only when it grows by more than 2^8.  The epilogue
+// stages the normalised O tile in the warpgroup's Q buffer and writes it with
+// one TMA store (rows past T are clipped by the tensor map).
 #pragma once
 #include "sm100.cuh"
 
 namespace ar {
 
 struct FwdParams {
-  __nv_bfloat16* o;  // [B, T, H, 128]
   float* lse;        // [B, H, T]
   const float* ck;   // [B*H, T_pad]: rk_j * scale * log2(e), 0 on padding
   int B, T, H, T_pad;
@@ -51,7 +53,8 @@ constexpr uint32_t kTile = 32768, kHalf = 16384;
 constexpr uint32_t kQ = 0, kK = 2 * kTile, kV = 4 * kTile, kCK = 6 * kTile;
 enum {
   QFULL = 0, QEMPTY, KFULL, KEMPTY = KFULL + 2, VFULL = KEMPTY + 2, VEMPTY = VFULL + 2,
-  SFULL = VEMPTY + 2, PFULL = SFULL + 2, ODONE = PFULL + 2, OFREE = ODONE + 2, FINAL = OFREE + 2, NBAR
+  SFULL = VEMPTY + 2, PFULL = SFULL + 2, ODONE = PFULL + 2, OFREE = ODONE + 2, EPI = OFREE + 2,
+  FINAL = EPI + 2, NBAR
 };
 constexpr uint32_t kBar = kCK + 1024;
 constexpr uint32_t kTmemPtr = kBar + NBAR * 8;
@@ -80,6 +83,7 @@ __device__ __forceinline__ Unit decode(const FwdParams& p, int u) {
   U.bh = u % BH;
   U.b = U.bh / p.H;
   U.h = U.bh % p.H;
+#pragma unroll
   for (int k = 0; k < 2; ++k) {
     U.r0[k] = qp * 256 + 128 * k;
     U.valid[k] = U.r0[k] < p.T;
@@ -96,7 +100,8 @@ __device__ __forceinline__ uint32_t bar_addr(uint32_t sbase, int i) { return sba
 
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+               const FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -107,7 +112,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBAR; ++i) {
       uint32_t cnt = 1;
-      if (i == PFULL || i == PFULL + 1 || i == OFREE || i == OFREE + 1) cnt = 128;
+      if (i == PFULL || i == PFULL + 1 || i == OFREE || i == OFREE + 1 || i == EPI || i == EPI + 1) cnt = 128;
+      if (i == QEMPTY) cnt = 2;  // one arrival per softmax warpgroup and unit
       mbar_init(bar_addr(sbase, i), cnt);
     }
     *abort_flag = 0;
@@ -121,18 +127,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_o);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + kTmemPtr);
 
-
   if (warp >= 8) {
-   regs_dec<kRegsLow>();
-   if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    regs_dec<kRegsLow>();
+    if (warp == 8 && lane == 0) {
+      // ---------------------------------------------------------- TMA producer
       uint32_t kv = 0;
       int uidx = 0;
       bool ok = true;
@@ -178,10 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (last_q_par >= 0) mbar_wait(bar_addr(sbase, QFULL), last_q_par, &never);
       }
-    }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 9 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t id_qk = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t id_pv = idesc_bf16(128, 128, 0, 1);
       auto issue_s = [&](int k, int st) {
@@ -212,6 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int st = kv & 1, ph = (kv >> 1) & 1;
           if (!mbar_wait(bar_addr(sbase, KFULL + st), ph, abort_flag)) break;
           tc_fence_after();
+#pragma unroll
           for (int k = 0; k < 2; ++k)
             if (U.in(k, U.hi_u)) {
               issue_s(k, st);
@@ -226,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int stn = kvn & 1, phn = (kvn >> 1) & 1, stx = kvx & 1, phx = (kvx >> 1) & 1;
           const bool has_next = it + 1 < U.N;
           if (!mbar_wait(bar_addr(sbase, VFULL + stn), phn, abort_flag)) { ok = false; break; }
-          if (has_next && !mbar_wait(bar_addr(sbase, KFULL + stx), phx, abort_flag)) { ok = false; break; }
+          bool k_next_ready = false;
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
             if (U.in(k, n)) {
@@ -240,6 +244,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (k == 1) mma_commit(bar_addr(sbase, VEMPTY + stn));
             if (has_next && U.in(k, n - 1)) {
+              if (!k_next_ready) {
+                if (!mbar_wait(bar_addr(sbase, KFULL + stx), phx, abort_flag)) { ok = false; break; }
+                k_next_ready = true;
+              }
               tc_fence_after();
               issue_s(k, stx);
               mma_commit(bar_addr(sbase, SFULL + k));
@@ -248,12 +256,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok && has_next) mma_commit(bar_addr(sbase, KEMPTY + stx));
         }
         if (!ok) break;
+#pragma unroll
         for (int k = 0; k < 2; ++k)
           if (U.valid[k]) {
             mma_commit(bar_addr(sbase, ODONE + k));
             ++ounits[k];
           }
-        mma_commit(bar_addr(sbase, QEMPTY));
         kv += U.N;
         ++uidx;
       }
@@ -262,16 +270,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       volatile int never = 0;
       mbar_wait(bar_addr(sbase, FINAL), 0, &never);
     }
-  }
   } else {
-   regs_inc<kRegsHigh>();
-   {
+    regs_inc<kRegsHigh>();
     // ------------------------------------------------------------ softmax warpgroups
     const int k = warp / 4;
     const int row = threadIdx.x & 127;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tbase + 128 * k + lane_off;
     const uint32_t tO = tbase + 256 + 128 * k + lane_off;
+    const uint32_t qa = sbase + kQ + k * kTile;
     const float kLn2 = 0.69314718055994531f;
     uint32_t scount = 0, ecount = 0, kv = 0;
     int uidx = 0;
@@ -280,22 +287,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int u = unit_index(cta, r, G);
       if (u >= p.n_units) break;
       const Unit U = decode(p, u);
-      if (!(k ? U.valid[1] : U.valid[0])) {
+      // this warpgroup's query tile, as scalars (no dynamic indexing into U)
+      const bool validk = k ? U.valid[1] : U.valid[0];
+      const int r0k = k ? U.r0[1] : U.r0[0];
+      const int lok = k ? U.lo[1] : U.lo[0];
+      const int hik = k ? U.hi[1] : U.hi[0];
+      if (!validk) {
+        if (row == 0) mbar_arrive(bar_addr(sbase, QEMPTY));  // nothing of ours in the Q buffers
         kv += U.N;
         ++uidx;
         continue;
       }
       if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, QFULL), uidx & 1, abort_flag))) break;
-      // this warpgroup's query tile, as scalars (no dynamic indexing into U)
-      const int r0k = k ? U.r0[1] : U.r0[0];
-      const int lok = k ? U.lo[1] : U.lo[0];
-      const int hik = k ? U.hi[1] : U.hi[0];
       const int i = r0k + row;
       // rq_i from this thread's own Q row in shared memory.
       float rq;
       {
         float ss[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint32_t qa = sbase + kQ + k * kTile;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
@@ -311,14 +319,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         rq = rsqrtf((ss[0] + ss[1] + ss[2] + ss[3]) * (1.0f / 128.0f) + p.eps);
       }
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l0 = 0.f, l1 = 0.f;
       bool first = true;
       for (int n = hik; n >= lok; --n) {
         const uint32_t kvn = kv + (U.hi_u - n);
         const int stn = kvn & 1, phn = (kvn >> 1) & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, SFULL + k), scount & 1, abort_flag))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, SFULL + k), scount & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
         ++scount;
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VFULL + stn), phn, abort_flag))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VFULL + stn), phn, abort_flag))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         uint32_t s[128];
         tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
@@ -327,28 +341,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
         tmem_wait_ld();
         const float4* ck4 = reinterpret_cast<const float4*>(smem + kCK + stn * 512);
-        const bool masked = (n * 128 + 127 > r0k) || (r0k + 127 - n * 128 > p.w);
-        float mx[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+        // x_j = S_j * ck_j (two at a time), running max three at a time
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
         for (int j4 = 0; j4 < 32; ++j4) {
           const float4 c4 = ck4[j4];
-          const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = j4 * 4 + e;
-            float x = __uint_as_float(s[j]) * cc[e];
-            if (masked) {
-              const int ja = n * 128 + j;
-              if (ja > i || i - ja > p.w) x = -INFINITY;
-            }
-            s[j] = __float_as_uint(x);
-            mx[j & 7] = fmaxf(mx[j & 7], x);
+          float x0, x1, x2, x3;
+          fmul2(x0, x1, __uint_as_float(s[4 * j4]), __uint_as_float(s[4 * j4 + 1]), c4.x, c4.y);
+          fmul2(x2, x3, __uint_as_float(s[4 * j4 + 2]), __uint_as_float(s[4 * j4 + 3]), c4.z, c4.w);
+          s[4 * j4] = __float_as_uint(x0);
+          s[4 * j4 + 1] = __float_as_uint(x1);
+          s[4 * j4 + 2] = __float_as_uint(x2);
+          s[4 * j4 + 3] = __float_as_uint(x3);
+          if ((j4 & 1) == 0) {
+            mx0 = fmax3(mx0, x0, x1);
+            mx1 = fmax3(mx1, x2, x3);
+          } else {
+            mx2 = fmax3(mx2, x0, x1);
+            mx3 = fmax3(mx3, x2, x3);
           }
         }
-        const float mrow = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        // masking only on tiles that cross the diagonal or the window edge
+        if ((n * 128 + 127 > r0k) || (r0k + 127 - n * 128 > p.w)) {
+          const int hi_c = i - n * 128;        // keys j <= hi_c are causal
+          const int lo_c = i - p.w - n * 128;  // keys j >= lo_c are inside the window
+          mx0 = mx1 = mx2 = mx3 = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < 128; ++j) {
+            float x = __uint_as_float(s[j]);
+            x = (j > hi_c || j < lo_c) ? -INFINITY : x;
+            s[j] = __float_as_uint(x);
+            if ((j & 1) == 0) mx0 = fmaxf(mx0, x);
+            else mx1 = fmaxf(mx1, x);
+          }
+        }
+        const float mrow = fmaxf(fmax3(mx0, mx1, mx2), mx3);
         const float mnew = fmaxf(m, mrow * rq);
         if (first) {
           m = mnew;
@@ -359,7 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float alpha = need ? ex2(m - mnew) : 1.0f;
             if (need) {
               m = mnew;
-              l *= alpha;
+              l0 *= alpha;
+              l1 *= alpha;
             }
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
@@ -367,27 +395,33 @@ __global__ void __launch_bounds__(kThreads, 1)
               tmem_ld32(tO + 32 * c, ov);
               tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+              for (int e = 0; e < 32; e += 2) {
+                float a0, a1;
+                fmul2(a0, a1, __uint_as_float(ov[e]), __uint_as_float(ov[e + 1]), alpha, alpha);
+                ov[e] = __float_as_uint(a0);
+                ov[e + 1] = __float_as_uint(a1);
+              }
               tmem_st32(tO + 32 * c, ov);
             }
             tmem_wait_st();
           }
         }
+        // p_j = 2^(x_j rq - m), packed to bf16 pairs into the S columns of TMEM
         const float negm = -m;
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2(fmaf(__uint_as_float(s[32 * c + 2 * e]), rq, negm));
-            const float p1 = ex2(fmaf(__uint_as_float(s[32 * c + 2 * e + 1]), rq, negm));
-            ls[e & 3] += p0 + p1;
+            float t0, t1;
+            ffma2(t0, t1, __uint_as_float(s[32 * c + 2 * e]), __uint_as_float(s[32 * c + 2 * e + 1]), rq, rq, negm,
+                  negm);
+            const float p0 = ex2(t0), p1 = ex2(t1);
+            fadd2(l0, l1, p0, p1);
             pk[e] = pack_bf16(p0, p1);
           }
           tmem_st16(tS + 16 * c, pk);
         }
-        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar_addr(sbase, PFULL + k));
@@ -397,8 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, ODONE + k), ecount & 1, abort_flag))) break;
       ++ecount;
       tc_fence_after();
+      const float l = l0 + l1;
       const float inv = 1.0f / l;
-      __nv_bfloat16* orow = p.o + (((size_t)U.b * p.T + i) * p.H + U.h) * 128;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t ov[32];
@@ -406,21 +440,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
-        if (i < p.T) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+        for (int e = 0; e < 16; ++e) {
+          float a0, a1;
+          fmul2(a0, a1, __uint_as_float(ov[2 * e]), __uint_as_float(ov[2 * e + 1]), inv, inv);
+          pk[e] = pack_bf16(a0, a1);
+        }
+        // columns 32c..32c+31 = 16-byte chunks 4c..4c+3 of the row, in the Q buffer's layout
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        for (int e = 0; e < 4; ++e) {
+          const int chunk = 4 * c + e;
+          sts128(qa + (chunk >> 3) * kHalf + sw128(row, chunk & 7),
+                 make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]));
         }
       }
       tc_fence_before();
       mbar_arrive(bar_addr(sbase, OFREE + k));
+      fence_proxy_async_smem();
+      mbar_arrive(bar_addr(sbase, EPI + k));
       if (i < p.T) p.lse[(size_t)U.bh * p.T + i] = (m + log2f(l)) * kLn2;
+      if (row == 0) {
+        // one thread stores the tile once every row is staged, then frees the Q buffer
+        if (mbar_wait(bar_addr(sbase, EPI + k), (ecount - 1) & 1, abort_flag)) {
+          tma_store_4d(&tm_o, qa, 0, U.h, r0k, U.b);
+          tma_store_4d(&tm_o, qa + kHalf, 64, U.h, r0k, U.b);
+          bulk_commit();
+          bulk_wait_read();
+        }
+        mbar_arrive(bar_addr(sbase, QEMPTY));
+      }
       kv += U.N;
       ++uidx;
     }
-  }
+    if (row == 0) bulk_wait_all();  // the last output tile has reached global memory
   }
   tc_fence_before();
   __syncthreads();
