@@ -290,6 +290,7 @@ int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, cons
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.dq_acc = dq_acc;
+  p.k = static_cast<const __nv_bfloat16*>(k);
   p.lse2 = lse2;
   p.delta = delta;
   p.rq = rq;
@@ -311,7 +312,7 @@ int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, cons
   {
     KernelTimer t(AR_KERNEL_DQ_POST, s);
     ar::dq_post_kernel<<<prep_grid(rows, sms), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q), dq_acc,
-                                                             static_cast<__nv_bfloat16*>(dq), B, T, H, eps);
+                                                             static_cast<__nv_bfloat16*>(dq), B, T, H, eps, scale);
     t.stop();
   }
   cudaError_t e = cudaGetLastError();

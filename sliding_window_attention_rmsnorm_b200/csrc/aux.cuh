@@ -5,7 +5,8 @@
 //   bwd_prep  : delta[bh, t] = sum_d dO_td o_td  (FlashAttention's backward pre-pass),
 //               rq[bh, t]    = 1/sqrt(mean_d q_td^2 + eps),
 //               lse2[bh, t]  = lse[bh, t] * log2(e), and dq_acc[t] = 0
-//   dq_post   : dq = rq (dqhat - qhat (dqhat . qhat) / D), qhat = rq q  (RMSNorm backward)
+//   dq_post   : dq = rq (dqhat - qhat (dqhat . qhat) / D), qhat = rq q  (RMSNorm backward),
+//               from the accumulator rq dqhat / scale of the backward kernel
 // The [B*H, T_pad] vectors are zero on the padding t >= T so that every tile
 // of 128 entries can be copied whole.
 #pragma once
@@ -103,8 +104,10 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_
   }
 }
 
+// dq from the fp32 accumulator acc_i = sum_j G_ij k_j = rq_i dqhat_i / scale:
+//   dq = rq (dqhat - qhat (dqhat . qhat) / D) = scale (acc - rq^2 q (acc . q) / D)
 __global__ void dq_post_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ dq_acc,
-                               __nv_bfloat16* __restrict__ dq, int B, int T, int H, float eps) {
+                               __nv_bfloat16* __restrict__ dq, int B, int T, int H, float eps, float scale) {
   const long long rows = (long long)B * T * H;
   const int sub = threadIdx.x & 15;
   const long long gstride = (long long)gridDim.x * (blockDim.x / 16);
@@ -122,14 +125,12 @@ __global__ void dq_post_kernel(const __nv_bfloat16* __restrict__ q, const float*
     }
     ss = half_warp_sum(ss);
     gq = half_warp_sum(gq);
-    const float r_ = rsqrtf(ss * (1.0f / 128.0f) + eps);
-    // dq = r (g - qhat (g.qhat)/D) with qhat = r q  ->  r g - r^3 q (g.q) / D
-    const float c = r_ * r_ * r_ * gq * (1.0f / 128.0f);
+    const float c = gq * (1.0f / 128.0f) / (ss * (1.0f / 128.0f) + eps);
     uint4 out;
-    out.x = pack_bf16(r_ * g[0] - c * fq[0], r_ * g[1] - c * fq[1]);
-    out.y = pack_bf16(r_ * g[2] - c * fq[2], r_ * g[3] - c * fq[3]);
-    out.z = pack_bf16(r_ * g[4] - c * fq[4], r_ * g[5] - c * fq[5]);
-    out.w = pack_bf16(r_ * g[6] - c * fq[6], r_ * g[7] - c * fq[7]);
+    out.x = pack_bf16(scale * (g[0] - c * fq[0]), scale * (g[1] - c * fq[1]));
+    out.y = pack_bf16(scale * (g[2] - c * fq[2]), scale * (g[3] - c * fq[3]));
+    out.z = pack_bf16(scale * (g[4] - c * fq[4]), scale * (g[5] - c * fq[5]));
+    out.w = pack_bf16(scale * (g[6] - c * fq[6]), scale * (g[7] - c * fq[7]));
     reinterpret_cast<uint4*>(dq + r * 128)[sub] = out;
   }
 }

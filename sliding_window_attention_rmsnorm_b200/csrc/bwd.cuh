@@ -9,32 +9,42 @@
 // The RMSNorm enters as the rank-1 factor rq_i rk_j: the tensor core works on
 // raw bf16 q and k, and one bf16 matrix G_ij = dS_ij rq_i rk_j feeds both
 // gradient products, dK_acc = G^T Q = rk_j dkhat_j / scale and
-// dQ_acc = G K = rq_i dqhat_i / scale, which the epilogues correct per row.
-// The key-side RMSNorm backward (dk = rk (dkhat - khat (dkhat.khat)/D)) runs in
-// this kernel's epilogue; dqhat is accumulated in fp32 in global memory and
-// finished by the dq post-pass.
+// dQ_acc = G K = rq_i dqhat_i / scale.  The key-side RMSNorm backward
+// (dk = rk (dkhat - khat (dkhat.khat)/D)) runs in this kernel's epilogue;
+// dQ_acc is accumulated in fp32 in global memory and finished (the factor
+// scale / rq_i and the query-side norm backward) by the dq post-pass.
 //
-// CTA organisation (persistent, one CTA per SM, 320 threads):
-//   warps 0-3  compute warpgroup: one key row per thread; P^T, dS^T, epilogue
-//   warps 4-7  dQ warpgroup: one query row per thread; reads dQ from TMEM and
-//              adds it to the fp32 accumulator with vector reductions
-//   warp 8     TMA producer: K, V per unit; Q, dO per query tile (2 stages)
-//   warp 9     MMA issuer
-// TMEM: S^T (cols 0-127, P^T overwrites 0-63) | dP^T (128-255, later dQ) | dV | dK.
-// Shared memory: K, V, Q[2], dO[2], G^T (all 128x128 bf16, 128-byte swizzled),
-// plus the per-query vectors (lse*log2 e, delta, rq) of the current tile.
+// Each 128-query tile is handled as two 64-query halves a = 0, 1, one per
+// compute warpgroup, and the MMAs are software-pipelined so that the tensor
+// core computes half a of the next tile while the warpgroups finish this one:
+//   grad(0,i) dP_0(i+1) S_0(i+1) | grad(1,i) dP_1(i+1) S_1(i+1) | grad(0,i+1) ...
+// with grad(a,i) = dV += P_a^T dO_a, dK += G_a^T Q_a, dQ_a^T = K^T G_a^T.
+// dQ is produced transposed (TMEM lane = feature d, column = query), so its
+// fp32 reductions into global memory are coalesced across a warp.
+//
+// CTA organisation (persistent, one CTA per SM, 512 threads):
+//   warps 0-3   compute warpgroup 0: query half 0; one key row per thread
+//   warps 4-7   compute warpgroup 1: query half 1
+//   warps 8-11  dQ/epilogue warpgroup: dQ^T read-out and reduction; dK, dV epilogue
+//   warp 12     TMA producer: K, V per unit; Q, dO per query tile (2 stages)
+//   warp 13     MMA issuer;  warps 14-15 idle
+// TMEM (512 columns): S_0 | S_1 (64 each; P_a^T overwrites the first 32, then
+// dQ_a^T the whole slot) | dP_0 | dP_1 (64 each) | dV (128) | dK (128).
+// Shared memory: K, V, Q[2], dO[2], G^T (all 128x128 bf16, 128-byte swizzled,
+// G^T half a = query columns 64a..64a+63), plus per-half query vectors.
 #pragma once
 #include "sm100.cuh"
 
 namespace ar {
 
 struct BwdParams {
-  __nv_bfloat16* dk;   // [B, T, H, 128]
-  __nv_bfloat16* dv;   // [B, T, H, 128]
-  float* dq_acc;       // [B, T, H, 128] fp32 dqhat accumulator (zeroed by the pre-pass)
-  const float* lse2;   // [B*H, T_pad] lse * log2(e), 0 on padding
-  const float* delta;  // [B*H, T_pad] rowsum(dO * o), 0 on padding
-  const float* rq;     // [B*H, T_pad] 1/rms(q_i), 0 on padding
+  __nv_bfloat16* dk;       // [B, T, H, 128]
+  __nv_bfloat16* dv;       // [B, T, H, 128]
+  float* dq_acc;           // [B, T, H, 128] fp32 sum_j G_ij k_j (zeroed by the pre-pass)
+  const __nv_bfloat16* k;  // [B, T, H, 128] raw keys, for the dk epilogue
+  const float* lse2;       // [B*H, T_pad] lse * log2(e), 0 on padding
+  const float* delta;      // [B*H, T_pad] rowsum(dO * o), 0 on padding
+  const float* rq;         // [B*H, T_pad] 1/rms(q_i), 0 on padding
   int B, T, H, T_pad;
   int w;        // left window (w >= T means full causal)
   int nk;       // key tiles per head = ceil(T / 128)
@@ -43,21 +53,22 @@ struct BwdParams {
 };
 
 namespace bwd {
-constexpr int kThreads = 384;
-// Launch budget 168 registers x 384 threads; warpgroup 2 (TMA, MMA, 2 idle
-// warps) drops to 104 so warpgroups 0-1 can rise to 200: 256*200 + 128*104 = 168*384.
-constexpr int kRegsLow = 104, kRegsHigh = 200, kLaunchRegs = 168;
-static_assert(256 * kRegsHigh + 128 * kRegsLow <= kLaunchRegs * kThreads, "register split exceeds the launch budget");
+constexpr int kThreads = 512;
+// 128 registers per thread for every role (65536 / 512); no register moves.
+constexpr int kLaunchRegs = 128;
 constexpr uint32_t kTile = 32768, kHalf = 16384;
-constexpr uint32_t kK = 0, kV = kTile, kQ = 2 * kTile, kDO = 4 * kTile, kDS = 6 * kTile, kVec = 7 * kTile;
+constexpr uint32_t kK = 0, kV = kTile, kQ = 2 * kTile, kDO = 4 * kTile, kG = 6 * kTile, kVec = 7 * kTile;
 enum {
-  KVFULL = 0, KVEMPTY, QFULL, QEMPTY = QFULL + 2, SFULL = QEMPTY + 2, DSREADY, DSFREE, DQFULL, DQFREE,
-  DKDVDONE, ACCFREE, VECFULL, VECEMPTY, FINAL, NBAR
+  KVFULL = 0, KVEMPTY, QFULL, QEMPTY = QFULL + 2, SFULL = QEMPTY + 2, DSREADY = SFULL + 2, DSFREE = DSREADY + 2,
+  DQFULL = DSFREE + 2, DQFREE = DQFULL + 2, VECFULL = DQFREE + 2, VECEMPTY = VECFULL + 2, DKDVDONE = VECEMPTY + 2,
+  ACCFREE, FINAL, NBAR
 };
-constexpr uint32_t kBar = kVec + 3 * 512;
+constexpr uint32_t kVecHalf = 3 * 64 * 4;  // lse2, delta, rq for 64 queries
+constexpr uint32_t kBar = kVec + 2 * kVecHalf;
 constexpr uint32_t kTmemPtr = kBar + NBAR * 8;
 constexpr uint32_t kAbort = kTmemPtr + 4;
 constexpr uint32_t kSmemBytes = kAbort + 4 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Unit {
   int bh, b, h, kt, qlo, N;
@@ -84,6 +95,10 @@ __device__ __forceinline__ Unit decode(const BwdParams& p, int u) {
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t sbase, int i) { return sbase + kBar + 8u * i; }
 
+__device__ __forceinline__ void red_add_f32(float* gaddr, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(gaddr), "f"(v) : "memory");
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -98,18 +113,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBAR; ++i) {
       uint32_t cnt = 1;
-      if (i == DSREADY || i == DQFREE || i == ACCFREE || i == VECFULL || i == VECEMPTY) cnt = 128;
-      if (i == KVEMPTY) cnt = 129;  // the MMA commit + every compute thread after its epilogue
+      if (i == DSREADY || i == DSREADY + 1 || i == DQFREE || i == DQFREE + 1 || i == VECFULL || i == VECFULL + 1 ||
+          i == VECEMPTY || i == VECEMPTY + 1 || i == ACCFREE)
+        cnt = 128;
+      if (i == KVEMPTY) cnt = 1 + 256;  // the MMA commit + every compute thread once rk is read
       mbar_init(bar_addr(sbase, i), cnt);
     }
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(sbase + kTmemPtr, 512);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == 12 && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
@@ -119,14 +136,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + kTmemPtr);
-
   const float kLog2e = 1.4426950408889634f;
 
-  if (warp >= 8) {
-   regs_dec<kRegsLow>();
-   if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+  if (warp >= 12) {
+    if (warp == 12 && lane == 0) {
+      // ---------------------------------------------------------- TMA producer
       uint32_t qc = 0;
       int uidx = 0;
       bool ok = true;
@@ -163,14 +177,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 2; ++s)
           if (last_q_par[s] >= 0) mbar_wait(bar_addr(sbase, QFULL + s), last_q_par[s], &never);
       }
-    }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);  // both operands K-major
-      constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);  // A K-major, B MN-major
-      constexpr uint32_t id_nn = idesc_bf16(128, 128, 1, 1);  // both MN-major
-      const uint32_t tS = tbase, tDP = tbase + 128, tDV = tbase + 256, tDK = tbase + 384;
+    } else if (warp == 13 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t id_s = idesc_bf16(128, 64, 0, 0);     // S^T, dP^T: both K-major, N = 64 queries
+      constexpr uint32_t id_acc = idesc_bf16(128, 128, 0, 1);  // dV, dK: A K-major, B MN-major
+      constexpr uint32_t id_dq = idesc_bf16(128, 64, 1, 1);    // dQ^T: both MN-major
+      const uint32_t tDV = tbase + 256, tDK = tbase + 384;
+      auto issue_s = [&](int a, int st) {  // S_a^T = K Q_a^T
+        const uint32_t qa = sbase + kQ + st * kTile + a * 64 * 128;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          mma_ss(tbase + 64 * a, sdesc_sw128(sbase + kK + off, 16, 1024), sdesc_sw128(qa + off, 16, 1024), id_s,
+                 kk > 0);
+        }
+      };
+      auto issue_dp = [&](int a, int st) {  // dP_a^T = V dO_a^T
+        const uint32_t da = sbase + kDO + st * kTile + a * 64 * 128;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          mma_ss(tbase + 128 + 64 * a, sdesc_sw128(sbase + kV + off, 16, 1024), sdesc_sw128(da + off, 16, 1024),
+                 id_s, kk > 0);
+        }
+      };
+      auto issue_grad = [&](int a, int st, bool first) {
+        const uint32_t qrow = sbase + kQ + st * kTile + a * 64 * 128;
+        const uint32_t drow = sbase + kDO + st * kTile + a * 64 * 128;
+        const uint32_t ga = sbase + kG + a * kHalf;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // dV += P_a^T dO_a   (P_a^T from TMEM, 16 queries per step)
+          mma_ts(tDV, tbase + 64 * a + kk * 8, sdesc_sw128(drow + kk * 2048, kHalf, 1024), id_acc,
+                 (first && kk == 0) ? 0u : 1u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // dK += G_a^T Q_a
+          mma_ss(tDK, sdesc_sw128(ga + kk * 32, 16, 1024), sdesc_sw128(qrow + kk * 2048, kHalf, 1024), id_acc,
+                 (first && kk == 0) ? 0u : 1u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // dQ_a^T = K^T G_a^T  (16 keys per step), into slot S_a
+          mma_ss(tbase + 64 * a, sdesc_sw128(sbase + kK + kk * 2048, kHalf, 1024),
+                 sdesc_sw128(ga + kk * 2048, kHalf, 1024), id_dq, kk > 0);
+      };
       uint32_t qc = 0;
       int uidx = 0;
       bool ok = true;
@@ -179,272 +226,298 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
         if (!mbar_wait(bar_addr(sbase, KVFULL), uidx & 1, abort_flag)) break;
-        for (int it = 0; it < U.N; ++it, ++qc) {
+        {  // prologue: S and dP of both halves of the first tile
           const int st = qc & 1, ph = (qc >> 1) & 1;
-          const uint32_t qa = sbase + kQ + st * kTile, da = sbase + kDO + st * kTile;
-          if (!mbar_wait(bar_addr(sbase, QFULL + st), ph, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          // S^T = K Q^T
+          if (!mbar_wait(bar_addr(sbase, QFULL + st), ph, abort_flag)) break;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            mma_ss(tS, sdesc_sw128(sbase + kK + off, 16, 1024), sdesc_sw128(qa + off, 16, 1024), id_kk, kk > 0);
+          for (int a = 0; a < 2; ++a) {
+            if (qc > 0 && !mbar_wait(bar_addr(sbase, DQFREE + a), (qc - 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(a, st);
+            issue_dp(a, st);
+            mma_commit(bar_addr(sbase, SFULL + a));
           }
-          // dP^T = V dO^T, once the previous dQ has left TMEM
-          if (qc > 0 && !mbar_wait(bar_addr(sbase, DQFREE), (qc - 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
+          if (!ok) break;
+        }
+        for (int it = 0; it < U.N && ok; ++it) {
+          const uint32_t q = qc + it, q1 = q + 1;
+          const int st = q & 1, st1 = q1 & 1, ph1 = (q1 >> 1) & 1;
+          const bool has_next = it + 1 < U.N;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            mma_ss(tDP, sdesc_sw128(sbase + kV + off, 16, 1024), sdesc_sw128(da + off, 16, 1024), id_kk, kk > 0);
+          for (int a = 0; a < 2; ++a) {
+            if (!mbar_wait(bar_addr(sbase, DSREADY + a), q & 1, abort_flag)) { ok = false; break; }
+            if (it == 0 && a == 0 && uidx > 0 &&
+                !mbar_wait(bar_addr(sbase, ACCFREE), (uidx - 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_grad(a, st, it == 0 && a == 0);
+            mma_commit(bar_addr(sbase, DQFULL + a));
+            mma_commit(bar_addr(sbase, DSFREE + a));
+            if (a == 1) mma_commit(bar_addr(sbase, QEMPTY + st));
+            if (has_next) {
+              if (a == 0 && !mbar_wait(bar_addr(sbase, QFULL + st1), ph1, abort_flag)) { ok = false; break; }
+              tc_fence_after();
+              issue_dp(a, st1);
+              if (!mbar_wait(bar_addr(sbase, DQFREE + a), q & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after();
+              issue_s(a, st1);
+              mma_commit(bar_addr(sbase, SFULL + a));
+            }
           }
-          mma_commit(bar_addr(sbase, SFULL));
-          if (!mbar_wait(bar_addr(sbase, DSREADY), qc & 1, abort_flag)) { ok = false; break; }
-          if (it == 0 && uidx > 0 && !mbar_wait(bar_addr(sbase, ACCFREE), (uidx - 1) & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          // dV += P^T dO   (P^T from TMEM)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tDV, tS + kk * 8, sdesc_sw128(da + kk * 2048, kHalf, 1024), id_kn, (it > 0 || kk > 0) ? 1u : 0u);
-          // dK += G^T Q
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            mma_ss(tDK, sdesc_sw128(sbase + kDS + off, 16, 1024), sdesc_sw128(qa + kk * 2048, kHalf, 1024), id_kn,
-                   (it > 0 || kk > 0) ? 1u : 0u);
-          }
-          // dQ = G K   (into the dP^T columns)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tDP, sdesc_sw128(sbase + kDS + kk * 2048, kHalf, 1024),
-                   sdesc_sw128(sbase + kK + kk * 2048, kHalf, 1024), id_nn, kk > 0);
-          mma_commit(bar_addr(sbase, DQFULL));
-          mma_commit(bar_addr(sbase, DSFREE));
-          mma_commit(bar_addr(sbase, QEMPTY + st));
         }
         if (!ok) break;
         mma_commit(bar_addr(sbase, DKDVDONE));
         mma_commit(bar_addr(sbase, KVEMPTY));
+        qc += U.N;
         ++uidx;
       }
       mma_commit(bar_addr(sbase, FINAL));
       volatile int never = 0;
       mbar_wait(bar_addr(sbase, FINAL), 0, &never);
     }
-  }
   } else {
-   regs_inc<kRegsHigh>();
-   if (warp < 4) {
-    // ------------------------------------------------------------ compute warpgroup (key rows)
-    const int row = threadIdx.x;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const uint32_t tS = tbase + lane_off, tDP = tbase + 128 + lane_off;
-    const uint32_t tDV = tbase + 256 + lane_off, tDK = tbase + 384 + lane_off;
-    float* vec = reinterpret_cast<float*>(smem + kVec);  // [0..127] lse2, [128..255] delta, [256..383] rq
-    uint32_t qc = 0;
-    int uidx = 0;
-    bool ok = true;
-    for (int r = 0; ok; ++r) {
-      const int u = unit_index(cta, r, G);
-      if (u >= p.n_units) break;
-      const Unit U = decode(p, u);
-      const int j = U.kt * 128 + row;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, KVFULL), uidx & 1, abort_flag))) break;
-      float rk;
-      {
-        float ss[4] = {0.f, 0.f, 0.f, 0.f};
+    if (warp < 8) {
+      // ---------------------------------------------------------- compute warpgroups (key rows)
+      const int a = warp / 4;  // query half
+      const int row = threadIdx.x & 127;
+      const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+      const uint32_t tS = tbase + 64 * a + lane_off, tDP = tbase + 128 + 64 * a + lane_off;
+      float* vec = reinterpret_cast<float*>(smem + kVec + a * kVecHalf);  // [0,64) lse2 [64,128) delta [128,192) rq
+      const uint32_t ga = sbase + kG + a * kHalf;
+      uint32_t qc = 0;
+      int uidx = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int u = unit_index(cta, r, G);
+        if (u >= p.n_units) break;
+        const Unit U = decode(p, u);
+        const int j = U.kt * 128 + row;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, KVFULL), uidx & 1, abort_flag))) break;
+        float rk;
+        {
+          float ss[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
+          for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 v = lds128(sbase + kK + hf * kHalf + sw128(row, c));
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            for (int c = 0; c < 8; ++c) {
+              const uint4 v = lds128(sbase + kK + hf * kHalf + sw128(row, c));
+              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float a = bf16lo(w4[e]), b2 = bf16hi(w4[e]);
-              ss[e] = fmaf(a, a, ss[e]);
-              ss[e] = fmaf(b2, b2, ss[e]);
-            }
-          }
-        rk = rsqrtf((ss[0] + ss[1] + ss[2] + ss[3]) * (1.0f / 128.0f) + p.eps);
-      }
-      const float Cj = rk * p.scale * kLog2e;
-      const size_t vbase = (size_t)U.bh * p.T_pad;
-      for (int it = 0; it < U.N; ++it, ++qc) {
-        const int qt = U.qlo + it;
-        // Per-query vectors of this tile, staged through shared memory: every
-        // thread writes one entry once all threads are done with the previous tile.
-        const float v_lse2 = p.lse2[vbase + qt * 128 + row];
-        const float v_delta = p.delta[vbase + qt * 128 + row];
-        const float v_rq = p.rq[vbase + qt * 128 + row];
-        if (qc > 0 &&
-            !__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VECEMPTY), (qc - 1) & 1, abort_flag))) {
-          ok = false;
-          break;
-        }
-        vec[row] = v_lse2;
-        vec[128 + row] = v_delta;
-        vec[256 + row] = v_rq;
-        mbar_arrive(bar_addr(sbase, VECFULL));
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VECFULL), qc & 1, abort_flag))) { ok = false; break; }
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, SFULL), qc & 1, abort_flag))) { ok = false; break; }
-        if (qc > 0 &&
-            !__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DSFREE), (qc - 1) & 1, abort_flag))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const bool masked = (qt == U.kt) || (qt * 128 + 127 - U.kt * 128 > p.w) || (qt * 128 + 127 >= p.T);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sv[32], dp[32];
-          tmem_ld32(tS + 32 * c, sv);
-          tmem_ld32(tDP + 32 * c, dp);
-          tmem_wait_ld();
-          uint32_t pk[16], gk[16];
-#pragma unroll
-          for (int e2 = 0; e2 < 16; ++e2) {
-            float pp[2], gg[2];
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int e = 2 * e2 + h2;
-              const int ii = 32 * c + e;
-              const float rqi = vec[256 + ii];
-              float P = ex2(fmaf(__uint_as_float(sv[e]) * rqi, Cj, -vec[ii]));
-              if (masked) {
-                const int i = qt * 128 + ii;
-                if (i < j || i - j > p.w || i >= p.T) P = 0.f;
+              for (int e = 0; e < 4; ++e) {
+                const float x0 = bf16lo(w4[e]), x1 = bf16hi(w4[e]);
+                ss[e] = fmaf(x0, x0, ss[e]);
+                ss[e] = fmaf(x1, x1, ss[e]);
               }
-              const float dS = P * (__uint_as_float(dp[e]) - vec[128 + ii]);
-              pp[h2] = P;
-              gg[h2] = dS * rqi * rk;
             }
-            pk[e2] = pack_bf16(pp[0], pp[1]);
-            gk[e2] = pack_bf16(gg[0], gg[1]);
+          rk = rsqrtf((ss[0] + ss[1] + ss[2] + ss[3]) * (1.0f / 128.0f) + p.eps);
+        }
+        mbar_arrive(bar_addr(sbase, KVEMPTY));  // done reading K from shared memory
+        const float Cj = rk * p.scale * kLog2e;
+        const size_t vbase = (size_t)U.bh * p.T_pad;
+        for (int it = 0; it < U.N; ++it, ++qc) {
+          const int qt = U.qlo + it;
+          const int i0 = qt * 128 + 64 * a;  // first query of this half
+          // per-query vectors of this half, staged through shared memory
+          const int vsel = row >> 6, vq = row & 63;
+          const float v0 = vsel == 0 ? p.lse2[vbase + i0 + vq] : p.rq[vbase + i0 + vq];
+          const float v1 = vsel == 0 ? p.delta[vbase + i0 + vq] : 0.f;
+          if (qc > 0 &&
+              !__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VECEMPTY + a), (qc - 1) & 1, abort_flag))) {
+            ok = false;
+            break;
           }
-          tmem_st16(tS + 16 * c, pk);
-          // G^T row j, queries 32c..32c+31: region c/2, 16-byte chunks 4*(c&1)..+3
-          const uint32_t ga = sbase + kDS + (c >> 1) * kHalf;
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            sts128(ga + sw128(row, 4 * (c & 1) + q4),
-                   make_uint4(gk[4 * q4], gk[4 * q4 + 1], gk[4 * q4 + 2], gk[4 * q4 + 3]));
-        }
-        tmem_wait_st();
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(bar_addr(sbase, DSREADY));
-        mbar_arrive(bar_addr(sbase, VECEMPTY));
-      }
-      if (!ok) break;
-      // ---------------------------------------------------------- epilogue: dV, dK (with norm backward)
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DKDVDONE), uidx & 1, abort_flag))) break;
-      tc_fence_after();
-      const size_t orow = (((size_t)U.b * p.T + j) * p.H + U.h) * 128;
+          if (vsel == 0) {
+            vec[vq] = v0;
+            vec[64 + vq] = v1;
+          } else {
+            vec[128 + vq] = v0;
+          }
+          mbar_arrive(bar_addr(sbase, VECFULL + a));
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VECFULL + a), qc & 1, abort_flag))) {
+            ok = false;
+            break;
+          }
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, SFULL + a), qc & 1, abort_flag))) {
+            ok = false;
+            break;
+          }
+          if (qc > 0 &&
+              !__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DSFREE + a), (qc - 1) & 1, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // queries c (0..63) of this half visible to key j: c_lo <= c <= c_hi
+          const int c_lo = j - i0;
+          const int c_hi = min(j + p.w, p.T - 1) - i0;
+          const bool masked = (c_lo > 0) || (c_hi < 63);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t a[32];
-        tmem_ld32(tDV + 32 * c, a);
-        tmem_wait_ld();
-        uint32_t pk[16];
+          for (int c = 0; c < 2; ++c) {
+            uint32_t sv[32], dp[32];
+            tmem_ld32(tS + 32 * c, sv);
+            tmem_ld32(tDP + 32 * c, dp);
+            tmem_wait_ld();
+            const float4* l4 = reinterpret_cast<const float4*>(vec + 32 * c);
+            const float4* d4 = reinterpret_cast<const float4*>(vec + 64 + 32 * c);
+            const float4* r4 = reinterpret_cast<const float4*>(vec + 128 + 32 * c);
+            uint32_t pk[16], gk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1]));
-        if (j < p.T) {
-          uint4* dst = reinterpret_cast<uint4*>(p.dv + orow + 32 * c);
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const float4 L = l4[e4], Dl = d4[e4], R = r4[e4];
+              const float lv[4] = {L.x, L.y, L.z, L.w}, dl[4] = {Dl.x, Dl.y, Dl.z, Dl.w},
+                          rv[4] = {R.x, R.y, R.z, R.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+              for (int h2 = 0; h2 < 2; ++h2) {
+                const int e = 4 * e4 + 2 * h2;
+                // u = S rq_i C_j - lse2_i ;  P = 2^u
+                float t0, t1, u0, u1;
+                fmul2(t0, t1, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]), rv[2 * h2], rv[2 * h2 + 1]);
+                ffma2(u0, u1, t0, t1, Cj, Cj, -lv[2 * h2], -lv[2 * h2 + 1]);
+                float P0 = ex2(u0), P1 = ex2(u1);
+                if (masked) {
+                  const int cc = 32 * c + e;
+                  if (cc < c_lo || cc > c_hi) P0 = 0.f;
+                  if (cc + 1 < c_lo || cc + 1 > c_hi) P1 = 0.f;
+                }
+                // G = P (dP - delta_i) rq_i rk_j
+                float g0 = __uint_as_float(dp[e]), g1 = __uint_as_float(dp[e + 1]), f0, f1;
+                fadd2(g0, g1, -dl[2 * h2], -dl[2 * h2 + 1]);
+                fmul2(f0, f1, rv[2 * h2], rv[2 * h2 + 1], rk, rk);
+                fmul2(g0, g1, g0, g1, P0, P1);
+                fmul2(g0, g1, g0, g1, f0, f1);
+                pk[e >> 1] = pack_bf16(P0, P1);
+                gk[e >> 1] = pack_bf16(g0, g1);
+              }
+            }
+            tmem_st16(tS + 16 * c, pk);
+            // G^T row j, queries 32c..32c+31 of this half: 16-byte chunks 4c..4c+3
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              sts128(ga + sw128(row, 4 * c + q4),
+                     make_uint4(gk[4 * q4], gk[4 * q4 + 1], gk[4 * q4 + 2], gk[4 * q4 + 3]));
+          }
+          tmem_wait_st();
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(bar_addr(sbase, DSREADY + a));
+          mbar_arrive(bar_addr(sbase, VECEMPTY + a));
         }
+        if (!ok) break;
+        ++uidx;
       }
-      {
-        // dk = scale (acc - rk^2 k (acc . k) / D): first the dot product, then the output,
-        // each pass reading 32 accumulator columns at a time.
-        float dot[4] = {0.f, 0.f, 0.f, 0.f};
+    } else {
+      // ---------------------------------------------------------- dQ / epilogue warpgroup
+      const int row = threadIdx.x - 256;  // TMEM lane: feature d for dQ^T, key row for dV/dK
+      const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+      const uint32_t tDV = tbase + 256 + lane_off, tDK = tbase + 384 + lane_off;
+      uint32_t qc = 0;
+      int uidx = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int u = unit_index(cta, r, G);
+        if (u >= p.n_units) break;
+        const Unit U = decode(p, u);
+        for (int it = 0; it < U.N && ok; ++it, ++qc) {
+          const int qt = U.qlo + it;
+#pragma unroll 1
+          for (int a = 0; a < 2; ++a) {
+            if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DQFULL + a), qc & 1, abort_flag))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            uint32_t x[64];
+            tmem_ld32(tbase + 64 * a + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+            tmem_ld32(tbase + 64 * a + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(bar_addr(sbase, DQFREE + a));
+            const int i0 = qt * 128 + 64 * a;
+            const int nvalid = min(64, p.T - i0);
+            float* dst = p.dq_acc + (((size_t)U.b * p.T + i0) * p.H + U.h) * 128 + row;
+            const size_t stride = (size_t)p.H * 128;
+            if (nvalid == 64) {
+#pragma unroll
+              for (int c = 0; c < 64; ++c) red_add_f32(dst + c * stride, __uint_as_float(x[c]));
+            } else {
+#pragma unroll
+              for (int c = 0; c < 64; ++c)
+                if (c < nvalid) red_add_f32(dst + c * stride, __uint_as_float(x[c]));
+            }
+          }
+        }
+        if (!ok) break;
+        // ------------------------------------------------------------ dV, dK epilogue
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DKDVDONE), uidx & 1, abort_flag))) break;
+        tc_fence_after();
+        const int j = U.kt * 128 + row;
+        const size_t orow = (((size_t)U.b * p.T + j) * p.H + U.h) * 128;
+        const bool jv = j < p.T;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
-          uint32_t a[32];
-          tmem_ld32(tDK + 32 * c, a);
+          uint32_t x[32];
+          tmem_ld32(tDV + 32 * c, x);
           tmem_wait_ld();
+          uint32_t pk[16];
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int cc = 4 * c + q4;  // 16-byte chunk of the k row (8 elements)
-            const uint4 v = lds128(sbase + kK + (cc >> 3) * kHalf + sw128(row, cc & 7));
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]));
+          if (jv) {
+            uint4* d = reinterpret_cast<uint4*>(p.dv + orow + 32 * c);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              dot[e] = fmaf(__uint_as_float(a[8 * q4 + 2 * e]), bf16lo(w4[e]), dot[e]);
-              dot[e] = fmaf(__uint_as_float(a[8 * q4 + 2 * e + 1]), bf16hi(w4[e]), dot[e]);
-            }
+            for (int e = 0; e < 4; ++e) d[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
           }
         }
-        const float coef = rk * rk * ((dot[0] + dot[1]) + (dot[2] + dot[3])) * (1.0f / 128.0f);
+        // dk = scale (acc - rk^2 k (acc . k) / D), with k and rk from the raw key row
+        {
+          const uint4* krow = reinterpret_cast<const uint4*>(p.k + orow);
+          float ss = 0.f, dot = 0.f;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t a[32];
-          tmem_ld32(tDK + 32 * c, a);
-          tmem_wait_ld();
+          for (int c = 0; c < 4; ++c) {
+            uint32_t x[32];
+            tmem_ld32(tDK + 32 * c, x);
+            tmem_wait_ld();
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int cc = 4 * c + q4;
-            const uint4 v = lds128(sbase + kK + (cc >> 3) * kHalf + sw128(row, cc & 7));
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-            uint32_t o4[4];
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const uint4 v = jv ? __ldg(krow + 4 * c + q4) : make_uint4(0, 0, 0, 0);
+              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float g0 = p.scale * (__uint_as_float(a[8 * q4 + 2 * e]) - coef * bf16lo(w4[e]));
-              const float g1 = p.scale * (__uint_as_float(a[8 * q4 + 2 * e + 1]) - coef * bf16hi(w4[e]));
-              o4[e] = pack_bf16(g0, g1);
+              for (int e = 0; e < 4; ++e) {
+                const float k0 = bf16lo(w4[e]), k1 = bf16hi(w4[e]);
+                ss = fmaf(k0, k0, fmaf(k1, k1, ss));
+                dot = fmaf(__uint_as_float(x[8 * q4 + 2 * e]), k0, fmaf(__uint_as_float(x[8 * q4 + 2 * e + 1]), k1, dot));
+              }
             }
-            if (j < p.T)
-              *reinterpret_cast<uint4*>(p.dk + orow + 8 * cc) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+          }
+          const float coef = dot * (1.0f / 128.0f) / (ss * (1.0f / 128.0f) + p.eps);
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t x[32];
+            tmem_ld32(tDK + 32 * c, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const uint4 v = jv ? __ldg(krow + 4 * c + q4) : make_uint4(0, 0, 0, 0);
+              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+              uint32_t o4[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float g0 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e]) - coef * bf16lo(w4[e]));
+                const float g1 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e + 1]) - coef * bf16hi(w4[e]));
+                o4[e] = pack_bf16(g0, g1);
+              }
+              if (jv)
+                *reinterpret_cast<uint4*>(p.dk + orow + 32 * c + 8 * q4) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            }
           }
         }
         tc_fence_before();
         mbar_arrive(bar_addr(sbase, ACCFREE));
-      }
-      mbar_arrive(bar_addr(sbase, KVEMPTY));
-      ++uidx;
-    }
-  } else {
-    // ------------------------------------------------------------ dQ warpgroup (query rows)
-    const int row = threadIdx.x - 128;
-    const uint32_t tDQ = tbase + 128 + ((uint32_t)((warp & 3) * 32) << 16);
-    uint32_t qc = 0;
-    bool ok = true;
-    for (int r = 0; ok; ++r) {
-      const int u = unit_index(cta, r, G);
-      if (u >= p.n_units) break;
-      const Unit U = decode(p, u);
-      for (int it = 0; it < U.N; ++it, ++qc) {
-        const int i = (U.qlo + it) * 128 + row;
-        const float rqi = p.rq[(size_t)U.bh * p.T_pad + (U.qlo + it) * 128 + row];
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DQFULL), qc & 1, abort_flag))) { ok = false; break; }
-        tc_fence_after();
-        uint32_t a[128];
-        tmem_ld32(tDQ + 0, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
-        tmem_ld32(tDQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
-        tmem_ld32(tDQ + 64, *reinterpret_cast<uint32_t(*)[32]>(&a[64]));
-        tmem_ld32(tDQ + 96, *reinterpret_cast<uint32_t(*)[32]>(&a[96]));
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar_addr(sbase, DQFREE));
-        if (i < p.T) {
-          const float f = p.scale / rqi;
-          float* dst = p.dq_acc + (((size_t)U.b * p.T + i) * p.H + U.h) * 128;
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            red_add_v4(dst + 4 * c, __uint_as_float(a[4 * c]) * f, __uint_as_float(a[4 * c + 1]) * f,
-                       __uint_as_float(a[4 * c + 2]) * f, __uint_as_float(a[4 * c + 3]) * f);
-        }
+        ++uidx;
       }
     }
-  }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
