@@ -99,6 +99,37 @@ __device__ __forceinline__ void red_add_f32(float* gaddr, float v) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(gaddr), "f"(v) : "memory");
 }
 
+// One 32-query chunk of a key row: P = 2^(S rq_i C_j - lse2_i) (zero outside the
+// band when MASKED), G = P (dP - delta_i) rq_i rk_j, both packed to bf16 pairs.
+// vaddr: shared-memory address of this chunk's lse2 entries; delta follows at
+// +256 bytes and rq at +512 bytes.
+template <bool MASKED>
+__device__ __forceinline__ void grad_chunk(const uint32_t (&sv)[32], const uint32_t (&dp)[32], uint32_t vaddr,
+                                           float Cj, float rk, int c_lo, int c_hi, int cbase, uint32_t (&pk)[16],
+                                           uint32_t (&gk)[16]) {
+#pragma unroll
+  for (int e4 = 0; e4 < 8; ++e4) {
+    const float4 L = lds_f4(vaddr + 16 * e4);
+    const float4 Dl = lds_f4(vaddr + 256 + 16 * e4);
+    const float4 R = lds_f4(vaddr + 512 + 16 * e4);
+    const float lv[4] = {L.x, L.y, L.z, L.w}, rv[4] = {R.x, R.y, R.z, R.w}, dl[4] = {Dl.x, Dl.y, Dl.z, Dl.w};
+    float P[4], Gv[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = 4 * e4 + q;
+      const float t = __uint_as_float(sv[e]) * rv[q];
+      float p_ = ex2(fmaf(t, Cj, -lv[q]));
+      if (MASKED) p_ = (cbase + e < c_lo || cbase + e > c_hi) ? 0.f : p_;
+      P[q] = p_;
+      Gv[q] = (__uint_as_float(dp[e]) - dl[q]) * (p_ * rv[q]) * rk;
+    }
+    pk[2 * e4] = pack_bf16(P[0], P[1]);
+    pk[2 * e4 + 1] = pack_bf16(P[2], P[3]);
+    gk[2 * e4] = pack_bf16(Gv[0], Gv[1]);
+    gk[2 * e4 + 1] = pack_bf16(Gv[2], Gv[3]);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -281,7 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = threadIdx.x & 127;
       const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
       const uint32_t tS = tbase + 64 * a + lane_off, tDP = tbase + 128 + 64 * a + lane_off;
-      float* vec = reinterpret_cast<float*>(smem + kVec + a * kVecHalf);  // [0,64) lse2 [64,128) delta [128,192) rq
+      // per-half query vectors in shared memory: [0,64) lse2, [64,128) delta, [128,192) rq (floats)
+      const uint32_t vaddr = sbase + kVec + a * kVecHalf;
       const uint32_t ga = sbase + kG + a * kHalf;
       uint32_t qc = 0;
       int uidx = 0;
@@ -326,10 +358,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           if (vsel == 0) {
-            vec[vq] = v0;
-            vec[64 + vq] = v1;
+            sts_f32(vaddr + 4 * vq, v0);
+            sts_f32(vaddr + 256 + 4 * vq, v1);
           } else {
-            vec[128 + vq] = v0;
+            sts_f32(vaddr + 512 + 4 * vq, v0);
           }
           mbar_arrive(bar_addr(sbase, VECFULL + a));
           if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VECFULL + a), qc & 1, abort_flag))) {
@@ -356,38 +388,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(tS + 32 * c, sv);
             tmem_ld32(tDP + 32 * c, dp);
             tmem_wait_ld();
-            const float4* l4 = reinterpret_cast<const float4*>(vec + 32 * c);
-            const float4* d4 = reinterpret_cast<const float4*>(vec + 64 + 32 * c);
-            const float4* r4 = reinterpret_cast<const float4*>(vec + 128 + 32 * c);
             uint32_t pk[16], gk[16];
-#pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) {
-              const float4 L = l4[e4], Dl = d4[e4], R = r4[e4];
-              const float lv[4] = {L.x, L.y, L.z, L.w}, dl[4] = {Dl.x, Dl.y, Dl.z, Dl.w},
-                          rv[4] = {R.x, R.y, R.z, R.w};
-#pragma unroll
-              for (int h2 = 0; h2 < 2; ++h2) {
-                const int e = 4 * e4 + 2 * h2;
-                // u = S rq_i C_j - lse2_i ;  P = 2^u
-                float t0, t1, u0, u1;
-                fmul2(t0, t1, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]), rv[2 * h2], rv[2 * h2 + 1]);
-                ffma2(u0, u1, t0, t1, Cj, Cj, -lv[2 * h2], -lv[2 * h2 + 1]);
-                float P0 = ex2(u0), P1 = ex2(u1);
-                if (masked) {
-                  const int cc = 32 * c + e;
-                  if (cc < c_lo || cc > c_hi) P0 = 0.f;
-                  if (cc + 1 < c_lo || cc + 1 > c_hi) P1 = 0.f;
-                }
-                // G = P (dP - delta_i) rq_i rk_j
-                float g0 = __uint_as_float(dp[e]), g1 = __uint_as_float(dp[e + 1]), f0, f1;
-                fadd2(g0, g1, -dl[2 * h2], -dl[2 * h2 + 1]);
-                fmul2(f0, f1, rv[2 * h2], rv[2 * h2 + 1], rk, rk);
-                fmul2(g0, g1, g0, g1, P0, P1);
-                fmul2(g0, g1, g0, g1, f0, f1);
-                pk[e >> 1] = pack_bf16(P0, P1);
-                gk[e >> 1] = pack_bf16(g0, g1);
-              }
-            }
+            if (masked)
+              grad_chunk<true>(sv, dp, vaddr + 128 * c, Cj, rk, c_lo, c_hi, 32 * c, pk, gk);
+            else
+              grad_chunk<false>(sv, dp, vaddr + 128 * c, Cj, rk, c_lo, c_hi, 32 * c, pk, gk);
             tmem_st16(tS + 16 * c, pk);
             // G^T row j, queries 32c..32c+31 of this half: 16-byte chunks 4c..4c+3
 #pragma unroll

@@ -187,20 +187,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t id_qk = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t id_pv = idesc_bf16(128, 128, 0, 1);
+      // Descriptor bases; every operand below is a base plus a constant byte offset.
+      const uint64_t dQ_k = sdesc_sw128(sbase + kQ, 16, 1024), dK_k = sdesc_sw128(sbase + kK, 16, 1024);
+      const uint64_t dV_m = sdesc_sw128(sbase + kV, kHalf, 1024);
       auto issue_s = [&](int k, int st) {
-        const uint32_t qa = sbase + kQ + k * kTile, ka = sbase + kK + st * kTile;
+        const uint64_t qb = sdesc_add(dQ_k, k * kTile), kb = sdesc_add(dK_k, st * kTile);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          mma_ss(tbase + 128 * k, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), id_qk,
-                 kk > 0);
+          mma_ss(tbase + 128 * k, sdesc_add(qb, off), sdesc_add(kb, off), id_qk, kk > 0);
         }
       };
       auto issue_pv = [&](int k, int st, bool acc) {
-        const uint32_t va = sbase + kV + st * kTile;
+        const uint64_t vb = sdesc_add(dV_m, st * kTile);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tbase + 256 + 128 * k, tbase + 128 * k + kk * 8, sdesc_sw128(va + kk * 2048, kHalf, 1024), id_pv,
+          mma_ts(tbase + 256 + 128 * k, tbase + 128 * k + kk * 8, sdesc_add(vb, kk * 2048), id_pv,
                  (acc || kk > 0) ? 1u : 0u);
       };
       uint32_t kv = 0, pcount[2] = {0, 0}, ounits[2] = {0, 0};
@@ -340,12 +342,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
         tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
         tmem_wait_ld();
-        const float4* ck4 = reinterpret_cast<const float4*>(smem + kCK + stn * 512);
+        const uint32_t ck_addr = sbase + kCK + stn * 512;
         // x_j = S_j * ck_j (two at a time), running max three at a time
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
         for (int j4 = 0; j4 < 32; ++j4) {
-          const float4 c4 = ck4[j4];
+          const float4 c4 = lds_f4(ck_addr + 16 * j4);
           float x0, x1, x2, x3;
           fmul2(x0, x1, __uint_as_float(s[4 * j4]), __uint_as_float(s[4 * j4 + 1]), c4.x, c4.y);
           fmul2(x2, x3, __uint_as_float(s[4 * j4 + 2]), __uint_as_float(s[4 * j4 + 3]), c4.z, c4.w);
