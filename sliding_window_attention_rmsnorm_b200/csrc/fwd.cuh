@@ -16,7 +16,7 @@
 // CTA organisation (persistent, one CTA per SM, 384 threads):
 //   warps 0-3  softmax warpgroup 0: query tile 0 (rows r0..r0+127), one row per thread
 //   warps 4-7  softmax warpgroup 1: query tile 1 (rows r0+128..r0+255)
-//   warp 8     TMA producer: Q tiles, K and V tiles (2 stages each) and ck
+//   warp 8     TMA producer: Q tiles, K tiles (2 stages), V tiles and ck (3 stages)
 //   warp 9     MMA issuer: S_k = Q_k K^T into TMEM, O_k += P_k V with P_k read from TMEM
 //   warps 10-11 idle (their registers go to the softmax warpgroups)
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P_k (bf16
@@ -29,6 +29,8 @@
 // stages the normalised O tile in the warpgroup's Q buffer and writes it with
 // one TMA store (rows past T are clipped by the tensor map).
 #pragma once
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace ar {
@@ -50,13 +52,20 @@ constexpr int kThreads = 384;
 constexpr int kRegsLow = 104, kRegsHigh = 200, kLaunchRegs = 168;
 static_assert(256 * kRegsHigh + 128 * kRegsLow <= kLaunchRegs * kThreads, "register split exceeds the launch budget");
 constexpr uint32_t kTile = 32768, kHalf = 16384;
-constexpr uint32_t kQ = 0, kK = 2 * kTile, kV = 4 * kTile, kCK = 6 * kTile;
+// K tiles are double-buffered; V tiles (with their key factors ck) triple-buffered, because a V stage is
+// only released once both P V products of its tile are done and TMA loads take ~2 us under load.
+constexpr int kVStages = 3;
+constexpr uint32_t kQ = 0, kK = 2 * kTile, kV = 4 * kTile, kCK = 7 * kTile;
+// Of every 4 pairs of softmax exponentials, this many are computed on the FMA
+// pipe (exp2_fma2) and the rest on the MUFU unit.
+constexpr int kEmuPairsOf4 = 0;
 enum {
-  QFULL = 0, QEMPTY, KFULL, KEMPTY = KFULL + 2, VFULL = KEMPTY + 2, VEMPTY = VFULL + 2,
-  SFULL = VEMPTY + 2, PFULL = SFULL + 2, ODONE = PFULL + 2, OFREE = ODONE + 2, EPI = OFREE + 2,
+  QFULL = 0, QEMPTY, KFULL, KEMPTY = KFULL + 2, VFULL = KEMPTY + 2, VEMPTY = VFULL + kVStages,
+  SFULL = VEMPTY + kVStages, PFULL = SFULL + 2, ODONE = PFULL + 2, OFREE = ODONE + 2, EPI = OFREE + 2,
   FINAL = EPI + 2, NBAR
 };
-constexpr uint32_t kBar = kCK + 1024;
+constexpr uint32_t kBar = kCK + kVStages * 512;
+static_assert(kBar + 256 + 1024 <= 232448, "shared memory budget");
 constexpr uint32_t kTmemPtr = kBar + NBAR * 8;
 constexpr uint32_t kAbort = kTmemPtr + 4;
 constexpr uint32_t kSmemBytes = kAbort + 4 + 1024;  // + slack for 1024-byte alignment
@@ -141,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kv = 0;
       int uidx = 0;
       bool ok = true;
-      int last_k_par[2] = {-1, -1}, last_v_par[2] = {-1, -1}, last_q_par = -1;
+      int last_k_par[2] = {-1, -1}, last_v_par[kVStages] = {-1, -1, -1}, last_q_par = -1;
       for (int r = 0; ok; ++r) {
         const int u = unit_index(cta, r, G);
         if (u >= p.n_units) break;
@@ -163,24 +172,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d(sbase + kK + st * kTile + hf * kHalf, &tm_k, bar_addr(sbase, KFULL + st), hf * 64, U.h,
                         n * 128, U.b);
           last_k_par[st] = ph;
-          if (!mbar_wait(bar_addr(sbase, VEMPTY + st), ph ^ 1, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(bar_addr(sbase, VFULL + st), kTile + 512);
+          const int vs = kv % kVStages, vph = (kv / kVStages) & 1;
+          if (!mbar_wait(bar_addr(sbase, VEMPTY + vs), vph ^ 1, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(bar_addr(sbase, VFULL + vs), kTile + 512);
           for (int hf = 0; hf < 2; ++hf)
-            tma_load_4d(sbase + kV + st * kTile + hf * kHalf, &tm_v, bar_addr(sbase, VFULL + st), hf * 64, U.h,
+            tma_load_4d(sbase + kV + vs * kTile + hf * kHalf, &tm_v, bar_addr(sbase, VFULL + vs), hf * 64, U.h,
                         n * 128, U.b);
-          bulk_load(sbase + kCK + st * 512, p.ck + (size_t)U.bh * p.T_pad + n * 128, 512,
-                    bar_addr(sbase, VFULL + st));
-          last_v_par[st] = ph;
+          bulk_load(sbase + kCK + vs * 512, p.ck + (size_t)U.bh * p.T_pad + n * 128, 512,
+                    bar_addr(sbase, VFULL + vs));
+          last_v_par[vs] = vph;
         }
         ++uidx;
       }
       if (*abort_flag) {
         // Let copies still in flight land before the CTA's shared memory goes away.
         volatile int never = 0;
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < 2; ++s)
           if (last_k_par[s] >= 0) mbar_wait(bar_addr(sbase, KFULL + s), last_k_par[s], &never);
+        for (int s = 0; s < kVStages; ++s)
           if (last_v_par[s] >= 0) mbar_wait(bar_addr(sbase, VFULL + s), last_v_par[s], &never);
-        }
         if (last_q_par >= 0) mbar_wait(bar_addr(sbase, QFULL), last_q_par, &never);
       }
     } else if (warp == 9 && lane == 0) {
@@ -229,9 +239,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int it = 0; it < U.N && ok; ++it) {
           const int n = U.hi_u - it;
           const uint32_t kvn = kv + it, kvx = kvn + 1;
-          const int stn = kvn & 1, phn = (kvn >> 1) & 1, stx = kvx & 1, phx = (kvx >> 1) & 1;
+          const int vsn = kvn % kVStages, vphn = (kvn / kVStages) & 1, stx = kvx & 1, phx = (kvx >> 1) & 1;
           const bool has_next = it + 1 < U.N;
-          if (!mbar_wait(bar_addr(sbase, VFULL + stn), phn, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(bar_addr(sbase, VFULL + vsn), vphn, abort_flag)) { ok = false; break; }
           bool k_next_ready = false;
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
@@ -241,10 +251,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!mbar_wait(bar_addr(sbase, PFULL + k), pcount[k] & 1, abort_flag)) { ok = false; break; }
               ++pcount[k];
               tc_fence_after();
-              issue_pv(k, stn, !first_pv[k]);
+              issue_pv(k, vsn, !first_pv[k]);
               first_pv[k] = false;
             }
-            if (k == 1) mma_commit(bar_addr(sbase, VEMPTY + stn));
+            if (k == 1) mma_commit(bar_addr(sbase, VEMPTY + vsn));
             if (has_next && U.in(k, n - 1)) {
               if (!k_next_ready) {
                 if (!mbar_wait(bar_addr(sbase, KFULL + stx), phx, abort_flag)) { ok = false; break; }
@@ -325,13 +335,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool first = true;
       for (int n = hik; n >= lok; --n) {
         const uint32_t kvn = kv + (U.hi_u - n);
-        const int stn = kvn & 1, phn = (kvn >> 1) & 1;
+        const int vsn = kvn % kVStages, vphn = (kvn / kVStages) & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, SFULL + k), scount & 1, abort_flag))) {
           ok = false;
           break;
         }
         ++scount;
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VFULL + stn), phn, abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VFULL + vsn), vphn, abort_flag))) {
           ok = false;
           break;
         }
@@ -342,41 +352,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
         tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
         tmem_wait_ld();
-        const uint32_t ck_addr = sbase + kCK + stn * 512;
-        // x_j = S_j * ck_j (two at a time), running max three at a time
+        const uint32_t ck_addr = sbase + kCK + vsn * 512;
+        // x_j = S_j * ck_j (two at a time), masked to -inf outside the band on edge
+        // tiles, with the running max taken three at a time
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+        const int hi_c = i - n * 128;        // keys j <= hi_c are causal
+        const int lo_c = i - p.w - n * 128;  // keys j >= lo_c are inside the window
+        auto xpass = [&](auto masked_tag) {
+          constexpr bool kMasked = decltype(masked_tag)::value;
 #pragma unroll
-        for (int j4 = 0; j4 < 32; ++j4) {
-          const float4 c4 = lds_f4(ck_addr + 16 * j4);
-          float x0, x1, x2, x3;
-          fmul2(x0, x1, __uint_as_float(s[4 * j4]), __uint_as_float(s[4 * j4 + 1]), c4.x, c4.y);
-          fmul2(x2, x3, __uint_as_float(s[4 * j4 + 2]), __uint_as_float(s[4 * j4 + 3]), c4.z, c4.w);
-          s[4 * j4] = __float_as_uint(x0);
-          s[4 * j4 + 1] = __float_as_uint(x1);
-          s[4 * j4 + 2] = __float_as_uint(x2);
-          s[4 * j4 + 3] = __float_as_uint(x3);
-          if ((j4 & 1) == 0) {
-            mx0 = fmax3(mx0, x0, x1);
-            mx1 = fmax3(mx1, x2, x3);
-          } else {
-            mx2 = fmax3(mx2, x0, x1);
-            mx3 = fmax3(mx3, x2, x3);
-          }
-        }
-        // masking only on tiles that cross the diagonal or the window edge
-        if ((n * 128 + 127 > r0k) || (r0k + 127 - n * 128 > p.w)) {
-          const int hi_c = i - n * 128;        // keys j <= hi_c are causal
-          const int lo_c = i - p.w - n * 128;  // keys j >= lo_c are inside the window
-          mx0 = mx1 = mx2 = mx3 = -INFINITY;
+          for (int j4 = 0; j4 < 32; ++j4) {
+            const float4 c4 = lds_f4(ck_addr + 16 * j4);
+            float x[4];
+            fmul2(x[0], x[1], __uint_as_float(s[4 * j4]), __uint_as_float(s[4 * j4 + 1]), c4.x, c4.y);
+            fmul2(x[2], x[3], __uint_as_float(s[4 * j4 + 2]), __uint_as_float(s[4 * j4 + 3]), c4.z, c4.w);
+            if (kMasked) {
 #pragma unroll
-          for (int j = 0; j < 128; ++j) {
-            float x = __uint_as_float(s[j]);
-            x = (j > hi_c || j < lo_c) ? -INFINITY : x;
-            s[j] = __float_as_uint(x);
-            if ((j & 1) == 0) mx0 = fmaxf(mx0, x);
-            else mx1 = fmaxf(mx1, x);
+              for (int e = 0; e < 4; ++e) {
+                const int j = 4 * j4 + e;
+                x[e] = (j > hi_c || j < lo_c) ? -INFINITY : x[e];
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s[4 * j4 + e] = __float_as_uint(x[e]);
+            if ((j4 & 1) == 0) {
+              mx0 = fmax3(mx0, x[0], x[1]);
+              mx1 = fmax3(mx1, x[2], x[3]);
+            } else {
+              mx2 = fmax3(mx2, x[0], x[1]);
+              mx3 = fmax3(mx3, x[2], x[3]);
+            }
           }
-        }
+        };
+        if ((n * 128 + 127 > r0k) || (r0k + 127 - n * 128 > p.w))
+          xpass(std::integral_constant<bool, true>{});
+        else
+          xpass(std::integral_constant<bool, false>{});
         const float mrow = fmaxf(fmax3(mx0, mx1, mx2), mx3);
         const float mnew = fmaxf(m, mrow * rq);
         if (first) {
@@ -415,10 +426,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            float t0, t1;
+            float t0, t1, p0, p1;
             ffma2(t0, t1, __uint_as_float(s[32 * c + 2 * e]), __uint_as_float(s[32 * c + 2 * e + 1]), rq, rq, negm,
                   negm);
-            const float p0 = ex2(t0), p1 = ex2(t1);
+            if ((e & 3) < kEmuPairsOf4) {
+              exp2_fma2(t0, t1, p0, p1);  // FMA pipe
+            } else {
+              p0 = ex2(t0);  // MUFU
+              p1 = ex2(t1);
+            }
             fadd2(l0, l1, p0, p1);
             pk[e] = pack_bf16(p0, p1);
           }
