@@ -54,7 +54,8 @@ enum {
   AR_ERR_DEVICE = -6,      /* current device is not compute capability 10.0 (B200) */
   AR_ERR_CUDA = -7,        /* a CUDA runtime call failed */
   AR_ERR_TIMEOUT = -8,     /* a device-side wait gave up (reported by sync_status) */
-  AR_ERR_WORKSPACE = -9    /* workspace given but smaller than required */
+  AR_ERR_WORKSPACE = -9,   /* workspace given but smaller than required */
+  AR_ERR_TOO_LARGE = -10   /* problem exceeds ar_attn_fwd_noalloc's built-in scratch */
 };
 
 /* Bytes of scratch ar_attn_fwd needs: one fp32 per (b, h, t) rounded up to
@@ -120,6 +121,27 @@ int ar_attn_timing_enable(int on);
  * time in milliseconds (ms[AR_KERNEL_KINDS]) and the number of launches
  * (count[AR_KERNEL_KINDS]); either pointer may be NULL.  Clears the record. */
 int ar_attn_timing_read(double* ms, long long* count);
+
+/* Forward pass that allocates nothing, for callers that cannot call
+ * cudaMalloc: code running inside a CUDA-graph capture that must not allocate,
+ * plug-ins whose host application owns the device allocator, or real-time loops
+ * that forbid allocation after start-up.  It computes exactly what ar_attn_fwd
+ * computes (same arguments minus the workspace), using as scratch a fixed
+ * array compiled into the library instead of a caller or runtime allocation.
+ * There is no counterpart to this entry point on the reference pages.
+ *
+ * Limit: B * H * ceil(T / 128) * 128 <= AR_NOALLOC_MAX_KEYS (1,048,576 key
+ * rows, i.e. 4 MiB of per-key norm factors); larger problems return
+ * AR_ERR_TOO_LARGE without launching anything.
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before capturing a stream into a
+ * graph.  Every call on a device shares the one array and leaves its contents
+ * behind: calls that can overlap on the GPU (different streams, no ordering
+ * between them) race on it and must be serialised by the caller.  Every entry
+ * the kernels read is rewritten by the call itself, so no clearing is needed. */
+#define AR_NOALLOC_MAX_KEYS (1 << 20)
+int ar_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int T, int H, int D, int window, float eps, float scale, void* stream);
 
 #ifdef __cplusplus
 }

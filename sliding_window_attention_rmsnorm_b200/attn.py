@@ -19,6 +19,7 @@ AR_OK = 0
 STATUS = {
     0: "AR_OK", -1: "AR_ERR_NULL", -2: "AR_ERR_SHAPE", -3: "AR_ERR_UNSUPPORTED", -4: "AR_ERR_ALIGN",
     -5: "AR_ERR_ARG", -6: "AR_ERR_DEVICE", -7: "AR_ERR_CUDA", -8: "AR_ERR_TIMEOUT", -9: "AR_ERR_WORKSPACE",
+    -10: "AR_ERR_TOO_LARGE",
 }
 
 _lib = None
@@ -164,3 +165,31 @@ def timing_read():
     n = (ctypes.c_longlong * len(KERNELS))()
     _check(lib().ar_attn_timing_read(ms, n), "ar_attn_timing_read")
     return {k: (ms[i], n[i]) for i, k in enumerate(KERNELS)}
+
+
+NOALLOC_MAX_KEYS = 1 << 20
+
+
+def fwd_noalloc(q, k, v, window: int, eps: float = 1e-6, scale=None, out=None, lse=None):
+    """The forward through ar_attn_fwd_noalloc: no workspace is allocated.
+
+    For callers that must not allocate device memory (inside a graph capture,
+    under a host-owned allocator).  Scratch is the library's built-in array, so
+    B * H * ceil(T/128)*128 must not exceed NOALLOC_MAX_KEYS, and calls that
+    can overlap on the GPU must be serialised by the caller.  The outputs o and
+    lse may be passed in (out, lse) so that nothing at all is allocated here.
+    """
+    _check_inputs(q, k, v)
+    B, T, H, D = q.shape
+    if scale is None:
+        scale = default_scale(D)
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((B, H, T), dtype=torch.float32, device=q.device) if lse is None else lse
+    L = lib()
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    L.ar_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, vp]
+    L.ar_attn_fwd_noalloc.restype = i
+    st = L.ar_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, T, H, D, int(window),
+                               float(eps), float(scale), _stream())
+    _check(st, "ar_attn_fwd_noalloc")
+    return o, lse_t

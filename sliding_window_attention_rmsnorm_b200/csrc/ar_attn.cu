@@ -344,6 +344,7 @@ const char* ar_attn_strerror(int status) {
     case AR_ERR_CUDA: return "a CUDA runtime call failed";
     case AR_ERR_TIMEOUT: return "a device-side wait timed out; results of the affected call are invalid";
     case AR_ERR_WORKSPACE: return "workspace smaller than the required size";
+    case AR_ERR_TOO_LARGE: return "B * H * padded T exceeds the built-in scratch of ar_attn_fwd_noalloc";
     default: return "unknown status";
   }
 }
@@ -407,3 +408,72 @@ long long ar_attn_unmasked_pairs(int T, int window) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- allocation-free forward
+// Scratch for ar_attn_fwd_noalloc: the per-key norm factors of up to
+// AR_NOALLOC_MAX_KEYS key rows.  Compiled into the library, so it exists on
+// every device that loads it, for the life of the process.  In host code the
+// name is only a handle; its device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) float g_noalloc_ck[AR_NOALLOC_MAX_KEYS];
+
+namespace {
+float* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_ck on the current device, looked up once.
+int noalloc_scratch(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return AR_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return AR_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_ck) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return AR_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = static_cast<float*>(ptr);
+  }
+  *out = g_noalloc_ptr[dev];
+  return AR_OK;
+}
+}  // namespace
+
+extern "C" int ar_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T,
+                                   int H, int D, int window, float eps, float scale, void* stream) {
+  if (!q || !k || !v || !o || !lse) return AR_ERR_NULL;
+  int st = check_shape(B, T, H, D);
+  if (st != AR_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return AR_ERR_ALIGN;
+  if ((st = check_args(eps, scale)) != AR_OK) return st;
+  const int T_pad = (T + 127) / 128 * 128;
+  if ((long long)B * H * T_pad > (long long)AR_NOALLOC_MAX_KEYS) return AR_ERR_TOO_LARGE;
+  int sms = 0;
+  if ((st = device_setup(&sms)) != AR_OK) return st;
+  float* ck = nullptr;
+  if ((st = noalloc_scratch(&ck)) != AR_OK) return st;
+
+  CUtensorMap tq, tk, tv, to;
+  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, H) != AR_OK ||
+      make_map(&tv, v, B, T, H) != AR_OK || make_map(&to, o, B, T, H) != AR_OK)
+    return AR_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long rows = (long long)B * T * H;
+  ar::fwd_prep_kernel<<<prep_grid(rows, sms), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(k), ck, B, T, H, T_pad,
+                                                            eps, scale * 1.4426950408889634f);
+  ar::FwdParams p;
+  p.lse = lse;
+  p.ck = ck;
+  p.B = B;
+  p.T = T;
+  p.H = H;
+  p.T_pad = T_pad;
+  p.w = effective_window(window, T);
+  p.nqp = (T + 255) / 256;
+  p.n_units = B * H * p.nqp;
+  p.eps = eps;
+  const int grid = p.n_units < sms ? p.n_units : sms;
+  ar::fwd::fwd_kernel<<<grid, ar::fwd::kThreads, ar::fwd::kSmemBytes, s>>>(tq, tk, tv, to, p);
+  return cudaGetLastError() == cudaSuccess ? AR_OK : AR_ERR_CUDA;
+}
