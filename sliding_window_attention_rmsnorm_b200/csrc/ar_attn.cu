@@ -48,7 +48,9 @@ int device_setup(int* sms_out) {
       d.status = AR_ERR_CUDA;
     } else if (major != 10 || minor != 0) {
       d.status = AR_ERR_DEVICE;
-    } else if (cudaFuncSetAttribute(ar::fwd::fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    } else if (cudaFuncSetAttribute(ar::fwd::fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    ar::fwd::kSmemBytes) != cudaSuccess ||
+               cudaFuncSetAttribute(ar::fwd::fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     ar::fwd::kSmemBytes) != cudaSuccess ||
                cudaFuncSetAttribute(ar::bwd::bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     ar::bwd::kSmemBytes) != cudaSuccess) {
@@ -58,11 +60,13 @@ int device_setup(int* sms_out) {
       // The kernels move registers between warpgroups with setmaxnreg; the split
       // is sized for exactly 168 registers per thread at launch, so refuse any
       // other build rather than launch a kernel whose register raise cannot be met.
-      cudaFuncAttributes fa, ba;
-      if (cudaFuncGetAttributes(&fa, ar::fwd::fwd_kernel) != cudaSuccess ||
+      cudaFuncAttributes fa, fb, ba;
+      if (cudaFuncGetAttributes(&fa, ar::fwd::fwd_kernel<true>) != cudaSuccess ||
+          cudaFuncGetAttributes(&fb, ar::fwd::fwd_kernel<false>) != cudaSuccess ||
           cudaFuncGetAttributes(&ba, ar::bwd::bwd_kernel) != cudaSuccess)
         d.status = AR_ERR_CUDA;
-      else if (fa.numRegs != ar::fwd::kLaunchRegs || ba.numRegs != ar::bwd::kLaunchRegs)
+      else if (fa.numRegs != ar::fwd::kLaunchRegs || fb.numRegs != ar::fwd::kLaunchRegs ||
+               ba.numRegs != ar::bwd::kLaunchRegs)
         d.status = AR_ERR_CUDA;
     }
     if (!g_encode && d.status == AR_OK) {
@@ -117,6 +121,16 @@ int make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? AR_OK : AR_ERR_CUDA;
+}
+
+// The forward with the fixed softmax offset when the logit bound allows it
+// (see fwd.cuh), else the running-max forward.
+void launch_fwd(int grid, cudaStream_t s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                const CUtensorMap& to, const ar::FwdParams& p) {
+  if (p.bound <= ar::fwd::kFixedBoundMax)
+    ar::fwd::fwd_kernel<true><<<grid, ar::fwd::kThreads, ar::fwd::kSmemBytes, s>>>(tq, tk, tv, to, p);
+  else
+    ar::fwd::fwd_kernel<false><<<grid, ar::fwd::kThreads, ar::fwd::kSmemBytes, s>>>(tq, tk, tv, to, p);
 }
 
 size_t vec_bytes(int B, int T, int H) {
@@ -234,10 +248,11 @@ int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
   p.nqp = (T + 255) / 256;
   p.n_units = B * H * p.nqp;
   p.eps = eps;
+  p.bound = scale * 128.0f * 1.4426950408889634f;
   const int grid = p.n_units < sms ? p.n_units : sms;
   {
     KernelTimer t(AR_KERNEL_FWD, s);
-    ar::fwd::fwd_kernel<<<grid, ar::fwd::kThreads, ar::fwd::kSmemBytes, s>>>(tq, tk, tv, to, p);
+    launch_fwd(grid, s, tq, tk, tv, to, p);
     t.stop();
   }
   cudaError_t e = cudaGetLastError();
@@ -473,7 +488,8 @@ extern "C" int ar_attn_fwd_noalloc(const void* q, const void* k, const void* v, 
   p.nqp = (T + 255) / 256;
   p.n_units = B * H * p.nqp;
   p.eps = eps;
+  p.bound = scale * 128.0f * 1.4426950408889634f;
   const int grid = p.n_units < sms ? p.n_units : sms;
-  ar::fwd::fwd_kernel<<<grid, ar::fwd::kThreads, ar::fwd::kSmemBytes, s>>>(tq, tk, tv, to, p);
+  launch_fwd(grid, s, tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? AR_OK : AR_ERR_CUDA;
 }

@@ -24,10 +24,22 @@
 // S0 S1 | PV0 S0' PV1 S1' | ... lets one warpgroup's softmax run while the
 // tensor core works for the other.
 // Only key tiles that intersect the band of a query tile are visited, in
-// descending order from the diagonal tile.  Output rescaling is lazy: the
-// running max is raised only when it grows by more than 2^8.  The epilogue
-// stages the normalised O tile in the warpgroup's Q buffer and writes it with
-// one TMA store (rows past T are clipped by the tensor map).
+// descending order from the diagonal tile.
+//
+// Softmax offset.  The norm bounds every logit: |qhat . khat| <= D, because
+// |qhat|^2 = sum q^2 / (mean q^2 + eps) <= D, and likewise for khat; so
+// |s_ij log2 e| <= scale D log2 e =: bound.  When bound <= kFixedBoundMax (the
+// default scale 1/sqrt(128) gives 16.3), p_ij = 2^(s_ij log2 e - bound) lies in
+// [2^-2 bound, 1] for every row, with no underflow in fp32 or bf16, and the
+// kernel uses that fixed offset instead of a running row max: one streaming
+// pass per tile, no max reduction and no rescaling of O.  Otherwise
+// (kFixed = false) it keeps the running max, raised lazily only when it grows
+// by more than 2^8.  With the fixed offset no exponential is exactly 1, so O is
+// normalised by the sum of the bf16-rounded p that the P V product used (lse
+// still takes the unrounded sum); o is then a convex combination of v rows
+// with weights that sum to 1 up to fp32 rounding.
+// The epilogue stages the normalised O tile in the warpgroup's Q buffer and
+// writes it with one TMA store (rows past T are clipped by the tensor map).
 #pragma once
 #include <type_traits>
 
@@ -43,6 +55,7 @@ struct FwdParams {
   int nqp;           // query-tile pairs per head = ceil(T / 256)
   int n_units;       // B * H * nqp
   float eps;
+  float bound;       // scale * D * log2(e): the largest |logit| in log2 units
 };
 
 namespace fwd {
@@ -59,6 +72,9 @@ constexpr uint32_t kQ = 0, kK = 2 * kTile, kV = 4 * kTile, kCK = 7 * kTile;
 // Of every 4 pairs of softmax exponentials, this many are computed on the FMA
 // pipe (exp2_fma2) and the rest on the MUFU unit.
 constexpr int kEmuPairsOf4 = 0;
+// Largest logit bound (log2 units) for which the fixed softmax offset is used:
+// p >= 2^-64 stays a normal number in fp32 and bf16.
+constexpr float kFixedBoundMax = 32.0f;
 enum {
   QFULL = 0, QEMPTY, KFULL, KEMPTY = KFULL + 2, VFULL = KEMPTY + 2, VEMPTY = VFULL + kVStages,
   SFULL = VEMPTY + kVStages, PFULL = SFULL + 2, ODONE = PFULL + 2, OFREE = ODONE + 2, EPI = OFREE + 2,
@@ -107,6 +123,7 @@ __device__ __forceinline__ Unit decode(const FwdParams& p, int u) {
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t sbase, int i) { return sbase + kBar + 8u * i; }
 
+template <bool kFixed>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -331,7 +348,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         rq = rsqrtf((ss[0] + ss[1] + ss[2] + ss[3]) * (1.0f / 128.0f) + p.eps);
       }
-      float m = -INFINITY, l0 = 0.f, l1 = 0.f;
+      // l: row sum of the exponentials (gives lse); lr: row sum of the same values
+      // rounded to bf16 as the P V product sees them (normalises O in the
+      // fixed-offset path, so that o is an exact convex combination of v rows)
+      float m = -INFINITY, l0 = 0.f, l1 = 0.f, lr0 = 0.f, lr1 = 0.f;
       bool first = true;
       for (int n = hik; n >= lok; --n) {
         const uint32_t kvn = kv + (U.hi_u - n);
@@ -353,11 +373,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
         tmem_wait_ld();
         const uint32_t ck_addr = sbase + kCK + vsn * 512;
+        const int hi_c = i - n * 128;        // keys j <= hi_c are causal
+        const int lo_c = i - p.w - n * 128;  // keys j >= lo_c are inside the window
+        const bool edge = (n * 128 + 127 > r0k) || (r0k + 127 - n * 128 > p.w);
+        if constexpr (kFixed) {
+          // p_j = 2^(S_j ck_j rq - bound), in one pass, packed to bf16 pairs into
+          // the S columns of TMEM; -inf outside the band on edge tiles
+          const float negb = -p.bound;
+          auto ppass = [&](auto masked_tag) {
+            constexpr bool kMasked = decltype(masked_tag)::value;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int j4 = 0; j4 < 8; ++j4) {
+                const int jb = 32 * c + 4 * j4;
+                const float4 c4 = lds_f4(ck_addr + 4 * jb);
+                float x[4];
+                fmul2(x[0], x[1], __uint_as_float(s[jb]), __uint_as_float(s[jb + 1]), c4.x, c4.y);
+                fmul2(x[2], x[3], __uint_as_float(s[jb + 2]), __uint_as_float(s[jb + 3]), c4.z, c4.w);
+                if (kMasked) {
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) x[e] = (jb + e > hi_c || jb + e < lo_c) ? -INFINITY : x[e];
+                }
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                  float t0, t1, p0, p1;
+                  ffma2(t0, t1, x[2 * h2], x[2 * h2 + 1], rq, rq, negb, negb);
+                  if (((2 * j4 + h2) & 3) < kEmuPairsOf4) {
+                    exp2_fma2(t0, t1, p0, p1);  // FMA pipe
+                  } else {
+                    p0 = ex2(t0);  // MUFU
+                    p1 = ex2(t1);
+                  }
+                  fadd2(l0, l1, p0, p1);
+                  const uint32_t pp = pack_bf16(p0, p1);
+                  fadd2(lr0, lr1, bf16lo(pp), bf16hi(pp));
+                  pk[2 * j4 + h2] = pp;
+                }
+              }
+              tmem_st16(tS + 16 * c, pk);
+            }
+          };
+          if (edge)
+            ppass(std::integral_constant<bool, true>{});
+          else
+            ppass(std::integral_constant<bool, false>{});
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar_addr(sbase, PFULL + k));
+          continue;
+        }
         // x_j = S_j * ck_j (two at a time), masked to -inf outside the band on edge
         // tiles, with the running max taken three at a time
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-        const int hi_c = i - n * 128;        // keys j <= hi_c are causal
-        const int lo_c = i - p.w - n * 128;  // keys j >= lo_c are inside the window
         auto xpass = [&](auto masked_tag) {
           constexpr bool kMasked = decltype(masked_tag)::value;
 #pragma unroll
@@ -384,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         };
-        if ((n * 128 + 127 > r0k) || (r0k + 127 - n * 128 > p.w))
+        if (edge)
           xpass(std::integral_constant<bool, true>{});
         else
           xpass(std::integral_constant<bool, false>{});
@@ -450,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++ecount;
       tc_fence_after();
       const float l = l0 + l1;
-      const float inv = 1.0f / l;
+      const float inv = 1.0f / (kFixed ? lr0 + lr1 : l);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t ov[32];
@@ -475,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar_addr(sbase, OFREE + k));
       fence_proxy_async_smem();
       mbar_arrive(bar_addr(sbase, EPI + k));
-      if (i < p.T) p.lse[(size_t)U.bh * p.T + i] = (m + log2f(l)) * kLn2;
+      if (i < p.T) p.lse[(size_t)U.bh * p.T + i] = ((kFixed ? p.bound : m) + log2f(l)) * kLn2;
       if (row == 0) {
         // one thread stores the tile once every row is staged, then frees the Q buffer
         if (mbar_wait(bar_addr(sbase, EPI + k), (ecount - 1) & 1, abort_flag)) {

@@ -123,6 +123,27 @@ def test_other_eps_and_scale():
         compare(run_gpu(x, 100, eps, scale), run_oracle(x, 100, eps, scale), H, tag="eps=%g" % eps, edge=True)
 
 
+def test_running_max_forward():
+    """A scale whose logit bound (scale * D * log2 e = 36.9 at scale 0.2) is too
+    wide for the fixed softmax offset takes the running-max forward; random
+    and peaked keys, sliding and full causal.  Forward outputs only: the
+    backward does not depend on which forward path ran."""
+    B, T, H = 1, 320, 2
+    x = synth.layer_inputs(12, 0, B, T, H, 128)
+    for w, peaked in ((150, False), (-1, False), (-1, True)):
+        if peaked:
+            x["k"] = synth.peaked_keys(x["q"], 9998)
+        q, k, v = (x[r].cuda() for r in ("q", "k", "v"))
+        o, lse = attn.fwd(q, k, v, w, EPS, 0.2)
+        attn.sync_status()
+        ro, rl = orc.attn_fwd(x["q"], x["k"], x["v"], w, EPS, 0.2)
+        o = o.float().cpu().numpy().astype(np.float64)
+        err = np.abs(o - ro)
+        assert (err - (MAX_ABS + ULP_SLACK * np.abs(ro))).max() <= 0, (w, peaked, err.max())
+        assert np.linalg.norm(o - ro) / np.linalg.norm(ro) <= REL_L2, (w, peaked)
+        assert np.abs(lse.cpu().numpy() - rl).max() <= LSE_ABS, (w, peaked)
+
+
 # ------------------------------------------------------------------ full-size workloads, sampled heads
 @pytest.mark.parametrize("window", [1024, 2048])
 def test_full_size_layer_sampled_heads(window):
