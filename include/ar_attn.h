@@ -30,10 +30,11 @@
  *     abort crosses the ABI.  Argument errors are detected before any work is
  *     enqueued.  A device-side wait that gives up (AR_ERR_TIMEOUT) is reported
  *     by ar_attn_sync_status().
- *   - Workspace: if `workspace` is NULL the library allocates it stream-ordered
- *     (cudaMallocAsync / cudaFreeAsync on `stream`); otherwise it must hold at
- *     least the bytes returned by the matching *_workspace_bytes() call and be
- *     256-byte aligned.  It is scratch: its contents on entry do not matter.
+ *   - Workspace (ar_attn_bwd; the forward needs none): if `workspace` is NULL
+ *     the library allocates it stream-ordered (cudaMallocAsync / cudaFreeAsync
+ *     on `stream`); otherwise it must hold at least the bytes returned by
+ *     ar_attn_bwd_workspace_bytes() and be 256-byte aligned.  It is scratch:
+ *     its contents on entry do not matter.
  */
 #ifndef AR_ATTN_H
 #define AR_ATTN_H
@@ -58,13 +59,14 @@ enum {
   AR_ERR_TOO_LARGE = -10   /* problem exceeds ar_attn_fwd_noalloc's built-in scratch */
 };
 
-/* Bytes of scratch ar_attn_fwd needs: one fp32 per (b, h, t) rounded up to
- * whole 128-token tiles (the per-key norm factors).  0 on invalid sizes. */
+/* Bytes of scratch ar_attn_fwd needs: always 0.  The fused forward kernel
+ * derives the per-key norm factors from each K tile it loads, so it needs no
+ * scratch; the workspace arguments of ar_attn_fwd are accepted and ignored. */
 size_t ar_attn_fwd_workspace_bytes(int B, int T, int H, int D);
 
 /* Forward pass.  Inputs q, k, v; outputs o [B,T,H,D] bf16 and lse [B,H,T] fp32
- * (lse is what ar_attn_bwd needs).  Launches a per-key norm pre-pass and the
- * fused attention kernel on `stream`. */
+ * (lse is what ar_attn_bwd needs).  One fused kernel on `stream`; allocates
+ * nothing.  `workspace` and `workspace_bytes` are ignored (may be NULL / 0). */
 int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                 int B, int T, int H, int D, int window, float eps, float scale,
                 void* workspace, size_t workspace_bytes, void* stream);
@@ -125,9 +127,12 @@ int ar_attn_timing_read(double* ms, long long* count);
 /* Forward pass that allocates nothing, for callers that cannot call
  * cudaMalloc: code running inside a CUDA-graph capture that must not allocate,
  * plug-ins whose host application owns the device allocator, or real-time loops
- * that forbid allocation after start-up.  It computes exactly what ar_attn_fwd
- * computes (same arguments minus the workspace), using as scratch a fixed
- * array compiled into the library instead of a caller or runtime allocation.
+ * that forbid allocation after start-up.  It computes what ar_attn_fwd computes
+ * (same arguments minus the workspace) in two launches: a pre-pass writes the
+ * per-key norm factors into a fixed array compiled into the library, and the
+ * forward kernel reads them from there.  (ar_attn_fwd itself now derives the
+ * factors inside its kernel and allocates nothing either; this entry point
+ * keeps the two-launch form and its contract.)
  * There is no counterpart to this entry point on the reference pages.
  *
  * Limit: B * H * ceil(T / 128) * 128 <= AR_NOALLOC_MAX_KEYS (1,048,576 key

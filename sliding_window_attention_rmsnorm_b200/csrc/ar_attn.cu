@@ -33,6 +33,15 @@ std::mutex g_mu;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 // Checks the current device once: compute capability 10.0, kernel attributes.
+using FwdKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, ar::FwdParams);
+cudaError_t fwd_attr(FwdKernel f) {
+  return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, ar::fwd::kSmemBytes);
+}
+bool fwd_regs_ok(FwdKernel f) {
+  cudaFuncAttributes a;
+  return cudaFuncGetAttributes(&a, f) == cudaSuccess && a.numRegs == ar::fwd::kLaunchRegs;
+}
+
 int device_setup(int* sms_out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return AR_ERR_CUDA;
@@ -48,10 +57,10 @@ int device_setup(int* sms_out) {
       d.status = AR_ERR_CUDA;
     } else if (major != 10 || minor != 0) {
       d.status = AR_ERR_DEVICE;
-    } else if (cudaFuncSetAttribute(ar::fwd::fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    ar::fwd::kSmemBytes) != cudaSuccess ||
-               cudaFuncSetAttribute(ar::fwd::fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    ar::fwd::kSmemBytes) != cudaSuccess ||
+    } else if (fwd_attr(ar::fwd::fwd_kernel<true, false>) != cudaSuccess ||
+               fwd_attr(ar::fwd::fwd_kernel<false, false>) != cudaSuccess ||
+               fwd_attr(ar::fwd::fwd_kernel<true, true>) != cudaSuccess ||
+               fwd_attr(ar::fwd::fwd_kernel<false, true>) != cudaSuccess ||
                cudaFuncSetAttribute(ar::bwd::bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     ar::bwd::kSmemBytes) != cudaSuccess) {
       d.status = AR_ERR_CUDA;
@@ -60,13 +69,11 @@ int device_setup(int* sms_out) {
       // The kernels move registers between warpgroups with setmaxnreg; the split
       // is sized for exactly 168 registers per thread at launch, so refuse any
       // other build rather than launch a kernel whose register raise cannot be met.
-      cudaFuncAttributes fa, fb, ba;
-      if (cudaFuncGetAttributes(&fa, ar::fwd::fwd_kernel<true>) != cudaSuccess ||
-          cudaFuncGetAttributes(&fb, ar::fwd::fwd_kernel<false>) != cudaSuccess ||
-          cudaFuncGetAttributes(&ba, ar::bwd::bwd_kernel) != cudaSuccess)
+      if (!fwd_regs_ok(ar::fwd::fwd_kernel<true, false>) || !fwd_regs_ok(ar::fwd::fwd_kernel<false, false>) ||
+          !fwd_regs_ok(ar::fwd::fwd_kernel<true, true>) || !fwd_regs_ok(ar::fwd::fwd_kernel<false, true>))
         d.status = AR_ERR_CUDA;
-      else if (fa.numRegs != ar::fwd::kLaunchRegs || fb.numRegs != ar::fwd::kLaunchRegs ||
-               ba.numRegs != ar::bwd::kLaunchRegs)
+      cudaFuncAttributes ba;
+      if (cudaFuncGetAttributes(&ba, ar::bwd::bwd_kernel) != cudaSuccess || ba.numRegs != ar::bwd::kLaunchRegs)
         d.status = AR_ERR_CUDA;
     }
     if (!g_encode && d.status == AR_OK) {
@@ -123,14 +130,38 @@ int make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
   return r == CUDA_SUCCESS ? AR_OK : AR_ERR_CUDA;
 }
 
+ar::FwdParams fwd_params(float* lse, const float* ck, int B, int T, int H, int window, float eps, float scale) {
+  ar::FwdParams p;
+  p.lse = lse;
+  p.ck = ck;
+  p.B = B;
+  p.T = T;
+  p.H = H;
+  p.T_pad = (T + 127) / 128 * 128;
+  p.w = effective_window(window, T);
+  p.nqp = (T + 255) / 256;
+  p.n_units = B * H * p.nqp;
+  p.eps = eps;
+  p.bound = scale * 128.0f * 1.4426950408889634f;
+  p.cscale = scale * 1.4426950408889634f;
+  return p;
+}
+
 // The forward with the fixed softmax offset when the logit bound allows it
-// (see fwd.cuh), else the running-max forward.
+// (see fwd.cuh), else the running-max forward; key factors computed in the
+// kernel, or (ck_global) read from p.ck.
 void launch_fwd(int grid, cudaStream_t s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                const CUtensorMap& to, const ar::FwdParams& p) {
-  if (p.bound <= ar::fwd::kFixedBoundMax)
-    ar::fwd::fwd_kernel<true><<<grid, ar::fwd::kThreads, ar::fwd::kSmemBytes, s>>>(tq, tk, tv, to, p);
+                const CUtensorMap& to, const ar::FwdParams& p, bool ck_global) {
+  using namespace ar::fwd;
+  const bool fixed = p.bound <= kFixedBoundMax;
+  if (fixed && !ck_global)
+    fwd_kernel<true, false><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, to, p);
+  else if (!fixed && !ck_global)
+    fwd_kernel<false, false><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, to, p);
+  else if (fixed)
+    fwd_kernel<true, true><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, to, p);
   else
-    ar::fwd::fwd_kernel<false><<<grid, ar::fwd::kThreads, ar::fwd::kSmemBytes, s>>>(tq, tk, tv, to, p);
+    fwd_kernel<false, true><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, to, p);
 }
 
 size_t vec_bytes(int B, int T, int H) {
@@ -196,8 +227,8 @@ int prep_grid(long long rows, int sms) {
 extern "C" {
 
 size_t ar_attn_fwd_workspace_bytes(int B, int T, int H, int D) {
-  if (check_shape(B, T, H, D) != AR_OK) return 0;
-  return vec_bytes(B, T, H);
+  (void)B, (void)T, (void)H, (void)D;
+  return 0;  // the forward kernel derives the per-key norm factors itself
 }
 
 size_t ar_attn_bwd_workspace_bytes(int B, int T, int H, int D) {
@@ -213,9 +244,7 @@ int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return AR_ERR_ALIGN;
   if ((st = check_args(eps, scale)) != AR_OK) return st;
-  const size_t need = ar_attn_fwd_workspace_bytes(B, T, H, D);
-  if (workspace && workspace_bytes < need) return AR_ERR_WORKSPACE;
-  if (workspace && !aligned(workspace, 256)) return AR_ERR_ALIGN;
+  (void)workspace, (void)workspace_bytes;  // no scratch needed: see ar_attn_fwd_workspace_bytes
   int sms = 0;
   if ((st = device_setup(&sms)) != AR_OK) return st;
 
@@ -224,40 +253,14 @@ int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
       make_map(&tv, v, B, T, H) != AR_OK || make_map(&to, o, B, T, H) != AR_OK)
     return AR_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  void* ws = workspace;
-  if (!ws && cudaMallocAsync(&ws, need, s) != cudaSuccess) return AR_ERR_CUDA;
-
-  const int T_pad = (T + 127) / 128 * 128;
-  float* ck = static_cast<float*>(ws);
-  const long long rows = (long long)B * T * H;
-  const float cscale = scale * 1.4426950408889634f;
-  {
-    KernelTimer t(AR_KERNEL_FWD_PREP, s);
-    ar::fwd_prep_kernel<<<prep_grid(rows, sms), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(k), ck, B, T, H,
-                                                              T_pad, eps, cscale);
-    t.stop();
-  }
-  ar::FwdParams p;
-  p.lse = lse;
-  p.ck = ck;
-  p.B = B;
-  p.T = T;
-  p.H = H;
-  p.T_pad = T_pad;
-  p.w = effective_window(window, T);
-  p.nqp = (T + 255) / 256;
-  p.n_units = B * H * p.nqp;
-  p.eps = eps;
-  p.bound = scale * 128.0f * 1.4426950408889634f;
+  const ar::FwdParams p = fwd_params(lse, nullptr, B, T, H, window, eps, scale);
   const int grid = p.n_units < sms ? p.n_units : sms;
   {
     KernelTimer t(AR_KERNEL_FWD, s);
-    launch_fwd(grid, s, tq, tk, tv, to, p);
+    launch_fwd(grid, s, tq, tk, tv, to, p, false);
     t.stop();
   }
-  cudaError_t e = cudaGetLastError();
-  if (!workspace) cudaFreeAsync(ws, s);
-  return e == cudaSuccess ? AR_OK : AR_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? AR_OK : AR_ERR_CUDA;
 }
 
 int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
@@ -477,19 +480,8 @@ extern "C" int ar_attn_fwd_noalloc(const void* q, const void* k, const void* v, 
   const long long rows = (long long)B * T * H;
   ar::fwd_prep_kernel<<<prep_grid(rows, sms), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(k), ck, B, T, H, T_pad,
                                                             eps, scale * 1.4426950408889634f);
-  ar::FwdParams p;
-  p.lse = lse;
-  p.ck = ck;
-  p.B = B;
-  p.T = T;
-  p.H = H;
-  p.T_pad = T_pad;
-  p.w = effective_window(window, T);
-  p.nqp = (T + 255) / 256;
-  p.n_units = B * H * p.nqp;
-  p.eps = eps;
-  p.bound = scale * 128.0f * 1.4426950408889634f;
+  const ar::FwdParams p = fwd_params(lse, ck, B, T, H, window, eps, scale);
   const int grid = p.n_units < sms ? p.n_units : sms;
-  launch_fwd(grid, s, tq, tk, tv, to, p);
+  launch_fwd(grid, s, tq, tk, tv, to, p, true);
   return cudaGetLastError() == cudaSuccess ? AR_OK : AR_ERR_CUDA;
 }

@@ -30,7 +30,21 @@ __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
 }
 
 // Rows are visited in memory order (b, t, h); row r is token t = (r / H) % T of
-// head (b, h).
+// head (b, h).  The split uses 32-bit division whenever the row count allows it
+// (a 64-bit division costs several times the issue slots of the row's load).
+__device__ __forceinline__ void split_row(long long r, int T, int H, int& b, int& t, int& h) {
+  if (r < 0x7fffffffLL && (long long)T * H < 0x7fffffffLL) {
+    const unsigned ur = (unsigned)r, bt = ur / (unsigned)H;
+    h = (int)(ur - bt * (unsigned)H);
+    b = (int)(bt / (unsigned)T);
+    t = (int)(bt - (unsigned)b * (unsigned)T);
+  } else {
+    const long long bt = r / H;
+    h = (int)(r - bt * H);
+    b = (int)(bt / T);
+    t = (int)(bt - (long long)b * T);
+  }
+}
 __global__ void fwd_prep_kernel(const __nv_bfloat16* __restrict__ k, float* __restrict__ ck, int B, int T, int H,
                                 int T_pad, float eps, float cscale) {
   const long long rows = (long long)B * T * H;
@@ -45,9 +59,8 @@ __global__ void fwd_prep_kernel(const __nv_bfloat16* __restrict__ k, float* __re
     for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
     ss = half_warp_sum(ss);
     if (sub == 0) {
-      const int h = (int)(r % H);
-      const long long bt = r / H;
-      const int t = (int)(bt % T), b = (int)(bt / T);
+      int b, t, h;
+      split_row(r, T, H, b, t, h);
       ck[((long long)b * H + h) * T_pad + t] = rsqrtf(ss * (1.0f / 128.0f) + eps) * cscale;
     }
   }
@@ -85,9 +98,8 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (sub == 0) {
-      const int h = (int)(r % H);
-      const long long bt = r / H;
-      const int t = (int)(bt % T), b = (int)(bt / T);
+      int b, t, h;
+      split_row(r, T, H, b, t, h);
       const long long bh = (long long)b * H + h;
       delta[bh * T_pad + t] = dl;
       rq[bh * T_pad + t] = rsqrtf(ss * (1.0f / 128.0f) + eps);

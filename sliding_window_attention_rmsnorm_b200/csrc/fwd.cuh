@@ -16,9 +16,12 @@
 // CTA organisation (persistent, one CTA per SM, 384 threads):
 //   warps 0-3  softmax warpgroup 0: query tile 0 (rows r0..r0+127), one row per thread
 //   warps 4-7  softmax warpgroup 1: query tile 1 (rows r0+128..r0+255)
-//   warp 8     TMA producer: Q tiles, K tiles (2 stages), V tiles and ck (3 stages)
+//   warp 8     TMA producer: Q tiles, K tiles (2 stages), V tiles (3 stages)
 //   warp 9     MMA issuer: S_k = Q_k K^T into TMEM, O_k += P_k V with P_k read from TMEM
-//   warps 10-11 idle (their registers go to the softmax warpgroups)
+//   warps 10-11 key factors: ck_j = rk_j * scale * log2(e) of each K tile, from the
+//              tile in shared memory, into a 3-slot ring read by the softmax
+//              (kCkGlobal: read instead from a [B*H, T_pad] vector in global memory,
+//              loaded with the V tile; warps 10-11 then idle)
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P_k (bf16
 // pairs) overwrites the first 64 columns of S_k.  The MMA issue order
 // S0 S1 | PV0 S0' PV1 S1' | ... lets one warpgroup's softmax run while the
@@ -49,13 +52,14 @@ namespace ar {
 
 struct FwdParams {
   float* lse;        // [B, H, T]
-  const float* ck;   // [B*H, T_pad]: rk_j * scale * log2(e), 0 on padding
+  const float* ck;   // kCkGlobal only: [B*H, T_pad] rk_j * scale * log2(e), 0 on padding
   int B, T, H, T_pad;
   int w;             // left window (w >= T means full causal)
   int nqp;           // query-tile pairs per head = ceil(T / 256)
   int n_units;       // B * H * nqp
   float eps;
   float bound;       // scale * D * log2(e): the largest |logit| in log2 units
+  float cscale;      // scale * log2(e)
 };
 
 namespace fwd {
@@ -78,8 +82,9 @@ constexpr float kFixedBoundMax = 32.0f;
 enum {
   QFULL = 0, QEMPTY, KFULL, KEMPTY = KFULL + 2, VFULL = KEMPTY + 2, VEMPTY = VFULL + kVStages,
   SFULL = VEMPTY + kVStages, PFULL = SFULL + 2, ODONE = PFULL + 2, OFREE = ODONE + 2, EPI = OFREE + 2,
-  FINAL = EPI + 2, NBAR
+  CKFULL = EPI + 2, FINAL = CKFULL + kVStages, NBAR
 };
+constexpr int kCkThreads = 64;  // warps 10-11
 constexpr uint32_t kBar = kCK + kVStages * 512;
 static_assert(kBar + 256 + 1024 <= 232448, "shared memory budget");
 constexpr uint32_t kTmemPtr = kBar + NBAR * 8;
@@ -123,7 +128,7 @@ __device__ __forceinline__ Unit decode(const FwdParams& p, int u) {
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t sbase, int i) { return sbase + kBar + 8u * i; }
 
-template <bool kFixed>
+template <bool kFixed, bool kCkGlobal>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -140,6 +145,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t cnt = 1;
       if (i == PFULL || i == PFULL + 1 || i == OFREE || i == OFREE + 1 || i == EPI || i == EPI + 1) cnt = 128;
       if (i == QEMPTY) cnt = 2;  // one arrival per softmax warpgroup and unit
+      if (!kCkGlobal && (i == KEMPTY || i == KEMPTY + 1)) cnt = 1 + kCkThreads;  // MMA commit + key-factor warps
+      if (i >= CKFULL && i < CKFULL + kVStages) cnt = kCkThreads;
       mbar_init(bar_addr(sbase, i), cnt);
     }
     *abort_flag = 0;
@@ -191,12 +198,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           last_k_par[st] = ph;
           const int vs = kv % kVStages, vph = (kv / kVStages) & 1;
           if (!mbar_wait(bar_addr(sbase, VEMPTY + vs), vph ^ 1, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(bar_addr(sbase, VFULL + vs), kTile + 512);
+          mbar_expect_tx(bar_addr(sbase, VFULL + vs), kTile + (kCkGlobal ? 512 : 0));
           for (int hf = 0; hf < 2; ++hf)
             tma_load_4d(sbase + kV + vs * kTile + hf * kHalf, &tm_v, bar_addr(sbase, VFULL + vs), hf * 64, U.h,
                         n * 128, U.b);
-          bulk_load(sbase + kCK + vs * 512, p.ck + (size_t)U.bh * p.T_pad + n * 128, 512,
-                    bar_addr(sbase, VFULL + vs));
+          if (kCkGlobal)
+            bulk_load(sbase + kCK + vs * 512, p.ck + (size_t)U.bh * p.T_pad + n * 128, 512,
+                      bar_addr(sbase, VFULL + vs));
           last_v_par[vs] = vph;
         }
         ++uidx;
@@ -209,6 +217,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kVStages; ++s)
           if (last_v_par[s] >= 0) mbar_wait(bar_addr(sbase, VFULL + s), last_v_par[s], &never);
         if (last_q_par >= 0) mbar_wait(bar_addr(sbase, QFULL), last_q_par, &never);
+      }
+    } else if (!kCkGlobal && warp >= 10) {
+      // ---------------------------------------------------------- key factors
+      // Tile kv's factors go to ring slot kv % 3.  The slot is free: the K load
+      // of tile kv waited for the MMAs of tile kv - 2 (KEMPTY), which were issued
+      // after both softmax warpgroups finished tile kv - 3.
+      const int tid = threadIdx.x - 320;
+      uint32_t kv = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int u = unit_index(cta, r, G);
+        if (u >= p.n_units) break;
+        const Unit U = decode(p, u);
+        for (int it = 0; it < U.N; ++it, ++kv) {
+          const int n = U.hi_u - it;
+          const int st = kv & 1, ph = (kv >> 1) & 1;
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, KFULL + st), ph, abort_flag))) {
+            ok = false;
+            break;
+          }
+          const uint32_t kt = sbase + kK + st * kTile;
+          const uint32_t slot = sbase + kCK + (kv % kVStages) * 512;
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int row = tid + 64 * h2;
+            float ss[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const uint4 v = lds128(kt + hf * kHalf + sw128(row, c));
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float a = bf16lo(w4[e]), b2 = bf16hi(w4[e]);
+                  ss[e] = fmaf(a, a, ss[e]);
+                  ss[e] = fmaf(b2, b2, ss[e]);
+                }
+              }
+            const float ck = (n * 128 + row < p.T)
+                                 ? rsqrtf((ss[0] + ss[1] + ss[2] + ss[3]) * (1.0f / 128.0f) + p.eps) * p.cscale
+                                 : 0.f;
+            sts_f32(slot + 4 * row, ck);
+          }
+          mbar_arrive(bar_addr(sbase, KEMPTY + st));  // done reading the K tile
+          mbar_arrive(bar_addr(sbase, CKFULL + kv % kVStages));
+        }
       }
     } else if (warp == 9 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
@@ -356,15 +411,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int n = hik; n >= lok; --n) {
         const uint32_t kvn = kv + (U.hi_u - n);
         const int vsn = kvn % kVStages, vphn = (kvn / kVStages) & 1;
+        // key factors of this tile: in the ring (CKFULL) or loaded with V (VFULL).
+        // They are normally ready before S, so this wait comes first and the one
+        // on S is the last before the tile's work starts.
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(bar_addr(sbase, (kCkGlobal ? VFULL : CKFULL) + vsn), vphn, abort_flag))) {
+          ok = false;
+          break;
+        }
         if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, SFULL + k), scount & 1, abort_flag))) {
           ok = false;
           break;
         }
         ++scount;
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VFULL + vsn), vphn, abort_flag))) {
-          ok = false;
-          break;
-        }
         tc_fence_after();
         uint32_t s[128];
         tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
