@@ -101,7 +101,8 @@ __device__ __forceinline__ void red_add_f32(float* gaddr, float v) {
 
 // One 32-query chunk of a key row: P = 2^(S rq_i C_j - lse2_i) (zero outside the
 // band when MASKED), G = P (dP - delta_i) rq_i rk_j, both packed to bf16 pairs.
-// vaddr: shared-memory address of this chunk's lse2 entries; delta follows at
+// Two queries at a time in packed fp32x2 arithmetic.
+// vaddr: shared-memory address of this chunk's -lse2 entries; delta follows at
 // +256 bytes and rq at +512 bytes.
 template <bool MASKED>
 __device__ __forceinline__ void grad_chunk(const uint32_t (&sv)[32], const uint32_t (&dp)[32], uint32_t vaddr,
@@ -109,24 +110,28 @@ __device__ __forceinline__ void grad_chunk(const uint32_t (&sv)[32], const uint3
                                            uint32_t (&gk)[16]) {
 #pragma unroll
   for (int e4 = 0; e4 < 8; ++e4) {
-    const float4 L = lds_f4(vaddr + 16 * e4);
+    const float4 L = lds_f4(vaddr + 16 * e4);  // -lse2
     const float4 Dl = lds_f4(vaddr + 256 + 16 * e4);
     const float4 R = lds_f4(vaddr + 512 + 16 * e4);
-    const float lv[4] = {L.x, L.y, L.z, L.w}, rv[4] = {R.x, R.y, R.z, R.w}, dl[4] = {Dl.x, Dl.y, Dl.z, Dl.w};
-    float P[4], Gv[4];
+    const float nl[4] = {L.x, L.y, L.z, L.w}, dl[4] = {Dl.x, Dl.y, Dl.z, Dl.w}, rv[4] = {R.x, R.y, R.z, R.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int e = 4 * e4 + q;
-      const float t = __uint_as_float(sv[e]) * rv[q];
-      float p_ = ex2(fmaf(t, Cj, -lv[q]));
-      if (MASKED) p_ = (cbase + e < c_lo || cbase + e > c_hi) ? 0.f : p_;
-      P[q] = p_;
-      Gv[q] = (__uint_as_float(dp[e]) - dl[q]) * (p_ * rv[q]) * rk;
+    for (int h = 0; h < 2; ++h) {
+      const int e = 4 * e4 + 2 * h;
+      float rc0, rc1, t0, t1, x0, x1, rr0, rr1;
+      fmul2(rc0, rc1, rv[2 * h], rv[2 * h + 1], Cj, Cj);  // rq_i C_j
+      ffma2(t0, t1, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]), rc0, rc1, nl[2 * h], nl[2 * h + 1]);
+      float p0 = ex2(t0), p1 = ex2(t1);
+      if (MASKED) {
+        p0 = (cbase + e < c_lo || cbase + e > c_hi) ? 0.f : p0;
+        p1 = (cbase + e + 1 < c_lo || cbase + e + 1 > c_hi) ? 0.f : p1;
+      }
+      fsub2(x0, x1, __uint_as_float(dp[e]), __uint_as_float(dp[e + 1]), dl[2 * h], dl[2 * h + 1]);
+      fmul2(rr0, rr1, rv[2 * h], rv[2 * h + 1], rk, rk);  // rq_i rk_j
+      fmul2(x0, x1, x0, x1, p0, p1);
+      fmul2(x0, x1, x0, x1, rr0, rr1);
+      pk[e4 * 2 + h] = pack_bf16(p0, p1);
+      gk[e4 * 2 + h] = pack_bf16(x0, x1);
     }
-    pk[2 * e4] = pack_bf16(P[0], P[1]);
-    pk[2 * e4 + 1] = pack_bf16(P[2], P[3]);
-    gk[2 * e4] = pack_bf16(Gv[0], Gv[1]);
-    gk[2 * e4 + 1] = pack_bf16(Gv[2], Gv[3]);
   }
 }
 
@@ -312,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = threadIdx.x & 127;
       const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
       const uint32_t tS = tbase + 64 * a + lane_off, tDP = tbase + 128 + 64 * a + lane_off;
-      // per-half query vectors in shared memory: [0,64) lse2, [64,128) delta, [128,192) rq (floats)
+      // per-half query vectors in shared memory: [0,64) -lse2, [64,128) delta, [128,192) rq (floats)
       const uint32_t vaddr = sbase + kVec + a * kVecHalf;
       const uint32_t ga = sbase + kG + a * kHalf;
       uint32_t qc = 0;
@@ -358,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           if (vsel == 0) {
-            sts_f32(vaddr + 4 * vq, v0);
+            sts_f32(vaddr + 4 * vq, -v0);  // grad_chunk adds -lse2
             sts_f32(vaddr + 256 + 4 * vq, v1);
           } else {
             sts_f32(vaddr + 512 + 4 * vq, v0);

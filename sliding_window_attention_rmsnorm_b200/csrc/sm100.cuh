@@ -270,6 +270,12 @@ __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, 
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2pack(a0, a1)), "l"(f2pack(b0, b1)), "l"(f2pack(c0, c1)));
   f2unpack(d, d0, d1);
 }
+// (d0, d1) = (a0 - b0, a1 - b1)
+__device__ __forceinline__ void fsub2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  uint64_t d;
+  asm("sub.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2pack(a0, a1)), "l"(f2pack(b0, b1)));
+  f2unpack(d, d0, d1);
+}
 // (d0, d1) += (a0, a1)
 __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1) {
   uint64_t d;
