@@ -64,11 +64,22 @@ def parse():
     return ap.parse_args()
 
 
-def windows_for(wl):
+def windows_for(wl, rule):
+    """Per-layer windows of the workload; rule(n_layer, T, pattern) is the
+    library's window rule on the product path and the oracle's in its legs."""
     if "windows" in wl:
         return list(wl["windows"])
-    from oracle.stack import layer_windows  # pure-Python rule, used only for FLOP counting here
-    return layer_windows(wl["n_layer"], wl["T"], wl["pattern"])
+    return rule(wl["n_layer"], wl["T"], wl["pattern"])
+
+
+def lib_windows(wl):
+    from sliding_window_attention_rmsnorm_b200.stack import layer_windows
+    return windows_for(wl, layer_windows)
+
+
+def oracle_windows(wl):
+    from oracle.stack import layer_windows
+    return windows_for(wl, layer_windows)
 
 
 def pairs(T, w):
@@ -77,9 +88,9 @@ def pairs(T, w):
     return n1 * (n1 + 1) // 2 + (T - n1) * (w + 1)
 
 
-def step_flops(wl):
+def step_flops(wl, windows):
     """(forward, backward) counted FLOPs of one step of the workload."""
-    f = sum(wl["B"] * wl["H"] * pairs(wl["T"], w) * FWD_FLOPS_PER_PAIR for w in windows_for(wl))
+    f = sum(wl["B"] * wl["H"] * pairs(wl["T"], w) * FWD_FLOPS_PER_PAIR for w in windows)
     return f, BWD_FACTOR * f
 
 
@@ -185,7 +196,7 @@ def oracle_sample(wl, seconds, seed_layer_offset=0):
     """Run the fp64 oracle fwd+bwd on whole heads of the workload's layers,
     cycling through layers, for about `seconds`; returns (flops, secs, desc, threads)."""
     from oracle import oracle as orc
-    ws = windows_for(wl)
+    ws = oracle_windows(wl)
     B, T, H = wl["B"], wl["T"], wl["H"]
     flops, heads_done, t_total, n = 0.0, [], 0.0, 0
     while t_total < seconds or n == 0:
@@ -243,7 +254,8 @@ def run_ours(args, wl, rank, world, dist):
     host = [synth.layer_inputs(wl["config"], l, B, T, H, D) for l in range(L)]
     layers = [{r: t.to("cuda", non_blocking=False) for r, t in x.items()} for x in host]
     st = stack.Stack(layers, wl.get("pattern", "SSSL"), windows=wl.get("windows"))
-    fwd_f, bwd_f = step_flops(wl)
+    windows = lib_windows(wl)
+    fwd_f, bwd_f = step_flops(wl, windows)
 
     def barrier():
         if dist is not None:
@@ -309,9 +321,14 @@ def run_ours(args, wl, rank, world, dist):
             kernels[k]["tflops"] = per_kind_flops[k] * kern[k][1] / (kern[k][0] * 1e-3) / 1e12
     # memory-bound helpers: algorithmic bytes per launch
     tok = B * T * H
+    # the dq kernel reads one 32 KB G tile per (query tile, key tile) pair of the band
+    # (mean over the stack's layers) plus q, and writes dq; its K tile reads hit L2
+    nq = -(-T // 128)
+    g_pairs = sum(B * H * sum(min(qt + 1, min(nq, (min(w, T) + 127) // 128 + 1)) for qt in range(nq))
+                  for w in windows) / L
     algo_bytes = {"fwd_prep": tok * D * 2 + tok * 4,
-                  "bwd_prep": 3 * tok * D * 2 + tok * 4 * 4 + tok * D * 4,
-                  "dq_post": tok * D * 4 + tok * D * 2 * 2}
+                  "bwd_prep": 3 * tok * D * 2 + tok * 4 * 4,
+                  "dq": g_pairs * 32768 + tok * D * 2 * 2}
     for k, by in algo_bytes.items():
         if kern[k][1]:
             kernels[k]["gbs"] = by * kern[k][1] / (kern[k][0] * 1e-3) / 1e9
@@ -361,7 +378,7 @@ def run_ours(args, wl, rank, world, dist):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl["name"], "global_batch": B * world, "seq_len": T, "heads": H,
-                       "layers": L, "windows": windows_for(wl), "parallelism": "replicas x%d" % world,
+                       "layers": L, "windows": windows, "parallelism": "replicas x%d" % world,
                        "l2": "inputs larger than L2 (%.0f MB of q,k,v,dO per step)" % (4 * L * tok * D * 2 / 1e6)},
             "pct_of_bf16_peak": {"sustained": value / world / peaks["bf16_sustained"],
                                  "burst": value / world / peaks["bf16_burst"], "source": peaks["source"]},

@@ -71,15 +71,22 @@ int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
                 int B, int T, int H, int D, int window, float eps, float scale,
                 void* workspace, size_t workspace_bytes, void* stream);
 
-/* Bytes of scratch ar_attn_bwd needs: an fp32 [B,T,H,D] dq accumulator plus
- * three fp32 per-(b, h, t) vectors.  0 on invalid sizes. */
+/* Bytes of scratch ar_attn_bwd needs: three fp32 per-(b, h, t) vectors (rounded
+ * up to whole 128-token tiles) plus a buffer of bf16 128x128 tiles G^T, one per
+ * (query tile, key tile) pair of the causal band of a group of heads: for
+ * nq = ceil(T/128), nq(nq+1)/2 tiles of 32 KB per head, for as many heads as
+ * fit in 1 GiB (at least one, at most B*H); larger problems are processed in
+ * head groups.  Sized for full causal, so it serves every window.  0 on invalid
+ * sizes. */
 size_t ar_attn_bwd_workspace_bytes(int B, int T, int H, int D);
 
 /* Backward pass.  Inputs q, k, v, the forward's o and lse, and the upstream
  * gradient dO; outputs dq, dk, dv [B,T,H,D] bf16 (overwritten, not added to).
  * window, eps and scale must be the forward's.  Launches, on `stream`: the
- * pre-pass (delta = rowsum(dO * o), 1/rms(q), accumulator reset), the fused
- * backward kernel (dk, dv, dq accumulation), and the dq RMSNorm post-pass. */
+ * pre-pass (delta = rowsum(dO * o), 1/rms(q), lse * log2 e), then per head
+ * group the fused backward kernel (dk, dv, and the bf16 tiles G = dS rq rk
+ * into the workspace) and the dq kernel (dq = G K and the q-side RMSNorm
+ * backward). */
 int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                 const float* lse, void* dq, void* dk, void* dv,
                 int B, int T, int H, int D, int window, float eps, float scale,
@@ -107,9 +114,9 @@ long long ar_attn_unmasked_pairs(int T, int window);
 enum {
   AR_KERNEL_FWD_PREP = 0, /* per-key norm factors (memory-bound) */
   AR_KERNEL_FWD = 1,      /* fused forward attention (tensor-core bound) */
-  AR_KERNEL_BWD_PREP = 2, /* delta, 1/rms(q), accumulator reset (memory-bound) */
-  AR_KERNEL_BWD = 3,      /* fused backward attention (tensor-core bound) */
-  AR_KERNEL_DQ_POST = 4,  /* dq RMSNorm backward (memory-bound) */
+  AR_KERNEL_BWD_PREP = 2, /* delta, 1/rms(q), lse * log2(e) (memory-bound) */
+  AR_KERNEL_BWD = 3,      /* fused backward attention: dk, dv, G tiles (tensor-core bound) */
+  AR_KERNEL_DQ = 4,       /* dq = G K with the q-side RMSNorm backward (reads the G tiles) */
   AR_KERNEL_KINDS = 5
 };
 

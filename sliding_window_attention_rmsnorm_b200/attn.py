@@ -151,7 +151,7 @@ def unmasked_pairs(T: int, window: int) -> int:
     return int(lib().ar_attn_unmasked_pairs(int(T), int(window)))
 
 
-KERNELS = ("fwd_prep", "fwd", "bwd_prep", "bwd", "dq_post")
+KERNELS = ("fwd_prep", "fwd", "bwd_prep", "bwd", "dq")
 
 
 def timing_enable(on: bool = True):

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cctype>
 #include <cmath>
 #include <cstdint>
@@ -15,6 +16,7 @@
 
 #include "aux.cuh"
 #include "bwd.cuh"
+#include "dq.cuh"
 #include "fwd.cuh"
 #include "sm100.cuh"
 
@@ -62,7 +64,9 @@ int device_setup(int* sms_out) {
                fwd_attr(ar::fwd::fwd_kernel<true, true>) != cudaSuccess ||
                fwd_attr(ar::fwd::fwd_kernel<false, true>) != cudaSuccess ||
                cudaFuncSetAttribute(ar::bwd::bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    ar::bwd::kSmemBytes) != cudaSuccess) {
+                                    ar::bwd::kSmemBytes) != cudaSuccess ||
+               cudaFuncSetAttribute(ar::dqk::dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    ar::dqk::kSmemBytes) != cudaSuccess) {
       d.status = AR_ERR_CUDA;
     }
     if (d.status == AR_OK) {
@@ -169,6 +173,42 @@ size_t vec_bytes(int B, int T, int H) {
   return round_up((size_t)B * H * T_pad * sizeof(float), 256);
 }
 
+// The G buffer of the backward: one 128x128 bf16 tile (32 KB) per (query tile,
+// key tile) pair of the band, per head.  nb = key tiles in a query tile's band.
+constexpr size_t kGTile = 32768;
+constexpr size_t kGBufferCap = size_t(1) << 30;  // heads are processed in groups whose G tiles fit in this
+long long g_pairs_head(int T, int nb) {
+  const long long nq = (T + 127) / 128;
+  return nq <= nb ? nq * (nq + 1) / 2 : (long long)nb * (nb + 1) / 2 + (nq - nb) * nb;
+}
+size_t g_head_bytes(int T, int nb) { return (size_t)g_pairs_head(T, nb) * kGTile; }
+// Heads whose G tiles the workspace holds at once, sized for the widest band (full causal).
+size_t g_heads_cap(int B, int T, int H) {
+  const size_t per = g_head_bytes(T, (T + 127) / 128);
+  size_t n = kGBufferCap / per;
+  if (n < 1) n = 1;
+  const size_t bh = (size_t)B * H;
+  return n < bh ? n : bh;
+}
+int band_tiles(int w, int T) {
+  const int nq = (T + 127) / 128;
+  const long long nb = ((long long)w + 127) / 128 + 1;
+  return nb < nq ? (int)nb : nq;
+}
+
+// [rows, 64] bf16 viewed as 2-D; boxes of 64 x 128 land as one 128-byte-swizzled
+// half of a G^T tile.
+int make_g_map(CUtensorMap* m, void* base, long long rows) {
+  cuuint64_t dims[2] = {64, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? AR_OK : AR_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- kernel timing
 struct TimingRec {
   int kind;
@@ -233,7 +273,7 @@ size_t ar_attn_fwd_workspace_bytes(int B, int T, int H, int D) {
 
 size_t ar_attn_bwd_workspace_bytes(int B, int T, int H, int D) {
   if (check_shape(B, T, H, D) != AR_OK) return 0;
-  return round_up((size_t)B * T * H * kD * sizeof(float), 256) + 3 * vec_bytes(B, T, H);
+  return 3 * vec_bytes(B, T, H) + g_heads_cap(B, T, H) * g_head_bytes(T, (T + 127) / 128);
 }
 
 int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T, int H, int D,
@@ -289,49 +329,83 @@ int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, cons
 
   const int T_pad = (T + 127) / 128 * 128;
   char* w8 = static_cast<char*>(ws);
-  float* dq_acc = reinterpret_cast<float*>(w8);
-  const size_t acc_bytes = round_up((size_t)B * T * H * kD * sizeof(float), 256);
   const size_t vb = vec_bytes(B, T, H);
-  float* lse2 = reinterpret_cast<float*>(w8 + acc_bytes);
-  float* delta = reinterpret_cast<float*>(w8 + acc_bytes + vb);
-  float* rq = reinterpret_cast<float*>(w8 + acc_bytes + 2 * vb);
+  float* lse2 = reinterpret_cast<float*>(w8);
+  float* delta = reinterpret_cast<float*>(w8 + vb);
+  float* rq = reinterpret_cast<float*>(w8 + 2 * vb);
+  char* gbuf = w8 + 3 * vb;
   const long long rows = (long long)B * T * H;
 
   {
     KernelTimer t(AR_KERNEL_BWD_PREP, s);
     ar::bwd_prep_kernel<<<prep_grid(rows, sms), 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(o),
-        static_cast<const __nv_bfloat16*>(dO), lse, lse2, delta, rq, dq_acc, B, T, H, T_pad, eps);
+        static_cast<const __nv_bfloat16*>(dO), lse, lse2, delta, rq, B, T, H, T_pad, eps);
     t.stop();
   }
-  ar::BwdParams p;
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
-  p.dq_acc = dq_acc;
-  p.k = static_cast<const __nv_bfloat16*>(k);
-  p.lse2 = lse2;
-  p.delta = delta;
-  p.rq = rq;
-  p.B = B;
-  p.T = T;
-  p.H = H;
-  p.T_pad = T_pad;
-  p.w = effective_window(window, T);
-  p.nk = (T + 127) / 128;
-  p.n_units = B * H * p.nk;
-  p.eps = eps;
-  p.scale = scale;
-  const int grid = p.n_units < sms ? p.n_units : sms;
-  {
-    KernelTimer t(AR_KERNEL_BWD, s);
-    ar::bwd::bwd_kernel<<<grid, ar::bwd::kThreads, ar::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
-    t.stop();
+  const int w = effective_window(window, T);
+  const int nk = (T + 127) / 128;
+  const int nb = band_tiles(w, T);
+  const long long ph = g_pairs_head(T, nb);
+  // heads per launch: as many as the G buffer holds for this window
+  const long long cap_tiles = (long long)g_heads_cap(B, T, H) * g_pairs_head(T, nk);
+  const int BH = B * H;
+  const int hpl_max = (int)std::min<long long>(BH, std::max<long long>(1, cap_tiles / ph));
+  const int n_groups = (BH + hpl_max - 1) / hpl_max;
+  const int hpl = (BH + n_groups - 1) / n_groups;  // equal groups
+  CUtensorMap tg;
+  if (make_g_map(&tg, gbuf, 2 * (long long)hpl * ph * 128) != AR_OK) {
+    if (!workspace) cudaFreeAsync(ws, s);
+    return AR_ERR_CUDA;
   }
-  {
-    KernelTimer t(AR_KERNEL_DQ_POST, s);
-    ar::dq_post_kernel<<<prep_grid(rows, sms), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q), dq_acc,
-                                                             static_cast<__nv_bfloat16*>(dq), B, T, H, eps, scale);
-    t.stop();
+  for (int bh0 = 0; bh0 < BH; bh0 += hpl) {
+    const int n_bh = std::min(hpl, BH - bh0);
+    ar::BwdParams p;
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.k = static_cast<const __nv_bfloat16*>(k);
+    p.lse2 = lse2;
+    p.delta = delta;
+    p.rq = rq;
+    p.B = B;
+    p.T = T;
+    p.H = H;
+    p.T_pad = T_pad;
+    p.w = w;
+    p.nk = nk;
+    p.n_units = n_bh * nk;
+    p.bh0 = bh0;
+    p.n_bh = n_bh;
+    p.nb = nb;
+    p.pairs_head = (int)ph;
+    p.eps = eps;
+    p.scale = scale;
+    {
+      KernelTimer t(AR_KERNEL_BWD, s);
+      ar::bwd::bwd_kernel<<<std::min(p.n_units, sms), ar::bwd::kThreads, ar::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo,
+                                                                                                 tg, p);
+      t.stop();
+    }
+    ar::DqParams d;
+    d.q = static_cast<const __nv_bfloat16*>(q);
+    d.dq = static_cast<__nv_bfloat16*>(dq);
+    d.B = B;
+    d.T = T;
+    d.H = H;
+    d.w = w;
+    d.nq = nk;
+    d.n_units = n_bh * nk;
+    d.bh0 = bh0;
+    d.n_bh = n_bh;
+    d.nb = nb;
+    d.pairs_head = (int)ph;
+    d.eps = eps;
+    d.scale = scale;
+    {
+      KernelTimer t(AR_KERNEL_DQ, s);
+      ar::dqk::dq_kernel<<<std::min(d.n_units, sms), ar::dqk::kThreads, ar::dqk::kSmemBytes, s>>>(tg, tk, d);
+      t.stop();
+    }
   }
   cudaError_t e = cudaGetLastError();
   if (!workspace) cudaFreeAsync(ws, s);

@@ -4,9 +4,7 @@
 //   fwd_prep  : ck[bh, t] = rk_t * scale * log2(e), rk_t = 1/sqrt(mean_d k_td^2 + eps)
 //   bwd_prep  : delta[bh, t] = sum_d dO_td o_td  (FlashAttention's backward pre-pass),
 //               rq[bh, t]    = 1/sqrt(mean_d q_td^2 + eps),
-//               lse2[bh, t]  = lse[bh, t] * log2(e), and dq_acc[t] = 0
-//   dq_post   : dq = rq (dqhat - qhat (dqhat . qhat) / D), qhat = rq q  (RMSNorm backward),
-//               from the accumulator rq dqhat / scale of the backward kernel
+//               lse2[bh, t]  = lse[bh, t] * log2(e)
 // The [B*H, T_pad] vectors are zero on the padding t >= T so that every tile
 // of 128 entries can be copied whole.
 #pragma once
@@ -75,8 +73,8 @@ __global__ void fwd_prep_kernel(const __nv_bfloat16* __restrict__ k, float* __re
 
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ o,
                                 const __nv_bfloat16* __restrict__ dO, const float* __restrict__ lse,
-                                float* __restrict__ lse2, float* __restrict__ delta, float* __restrict__ rq,
-                                float* __restrict__ dq_acc, int B, int T, int H, int T_pad, float eps) {
+                                float* __restrict__ lse2, float* __restrict__ delta, float* __restrict__ rq, int B,
+                                int T, int H, int T_pad, float eps) {
   const long long rows = (long long)B * T * H;
   const int sub = threadIdx.x & 15;
   const long long gstride = (long long)gridDim.x * (blockDim.x / 16);
@@ -94,9 +92,6 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_
     }
     ss = half_warp_sum(ss);
     dl = half_warp_sum(dl);
-    float4* z = reinterpret_cast<float4*>(dq_acc + r * 128) + 2 * sub;
-    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (sub == 0) {
       int b, t, h;
       split_row(r, T, H, b, t, h);
@@ -113,37 +108,6 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_
     delta[bh * T_pad + t] = 0.f;
     rq[bh * T_pad + t] = 0.f;
     lse2[bh * T_pad + t] = 0.f;
-  }
-}
-
-// dq from the fp32 accumulator acc_i = sum_j G_ij k_j = rq_i dqhat_i / scale:
-//   dq = rq (dqhat - qhat (dqhat . qhat) / D) = scale (acc - rq^2 q (acc . q) / D)
-__global__ void dq_post_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ dq_acc,
-                               __nv_bfloat16* __restrict__ dq, int B, int T, int H, float eps, float scale) {
-  const long long rows = (long long)B * T * H;
-  const int sub = threadIdx.x & 15;
-  const long long gstride = (long long)gridDim.x * (blockDim.x / 16);
-  for (long long r = (long long)blockIdx.x * (blockDim.x / 16) + threadIdx.x / 16; r < rows; r += gstride) {
-    float fq[8];
-    unpack8(__ldg(reinterpret_cast<const uint4*>(q + r * 128) + sub), fq);
-    const float4* g4 = reinterpret_cast<const float4*>(dq_acc + r * 128) + 2 * sub;
-    const float4 ga = __ldcs(g4), gb = __ldcs(g4 + 1);
-    const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-    float ss = 0.f, gq = 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      ss = fmaf(fq[e], fq[e], ss);
-      gq = fmaf(g[e], fq[e], gq);
-    }
-    ss = half_warp_sum(ss);
-    gq = half_warp_sum(gq);
-    const float c = gq * (1.0f / 128.0f) / (ss * (1.0f / 128.0f) + eps);
-    uint4 out;
-    out.x = pack_bf16(scale * (g[0] - c * fq[0]), scale * (g[1] - c * fq[1]));
-    out.y = pack_bf16(scale * (g[2] - c * fq[2]), scale * (g[3] - c * fq[3]));
-    out.z = pack_bf16(scale * (g[4] - c * fq[4]), scale * (g[5] - c * fq[5]));
-    out.w = pack_bf16(scale * (g[6] - c * fq[6]), scale * (g[7] - c * fq[7]));
-    reinterpret_cast<uint4*>(dq + r * 128)[sub] = out;
   }
 }
 

@@ -8,28 +8,30 @@
 //   dkhat_j = scale sum_i dS_ij qhat_i,  dqhat_i = scale sum_j dS_ij khat_j
 // The RMSNorm enters as the rank-1 factor rq_i rk_j: the tensor core works on
 // raw bf16 q and k, and one bf16 matrix G_ij = dS_ij rq_i rk_j feeds both
-// gradient products, dK_acc = G^T Q = rk_j dkhat_j / scale and
-// dQ_acc = G K = rq_i dqhat_i / scale.  The key-side RMSNorm backward
-// (dk = rk (dkhat - khat (dkhat.khat)/D)) runs in this kernel's epilogue;
-// dQ_acc is accumulated in fp32 in global memory and finished (the factor
-// scale / rq_i and the query-side norm backward) by the dq post-pass.
+// gradient products, dK_acc = G^T Q = rk_j dkhat_j / scale here and
+// dQ_acc = G K = rq_i dqhat_i / scale in the dq kernel (dq.cuh).  The key-side
+// RMSNorm backward (dk = rk (dkhat - khat (dkhat.khat)/D)) runs in this
+// kernel's epilogue.  Each 128x128 tile of G^T is written to a global buffer
+// (one slot per (query tile, key tile) pair of the band) for the dq kernel,
+// so no TMEM columns are spent on dQ and no query tile waits for a dQ read-out.
 //
 // Each 128-query tile is handled as two 64-query halves a = 0, 1, one per
 // compute warpgroup, and the MMAs are software-pipelined so that the tensor
 // core computes half a of the next tile while the warpgroups finish this one:
 //   grad(0,i) dP_0(i+1) S_0(i+1) | grad(1,i) dP_1(i+1) S_1(i+1) | grad(0,i+1) ...
-// with grad(a,i) = dV += P_a^T dO_a, dK += G_a^T Q_a, dQ_a^T = K^T G_a^T.
-// dQ is produced transposed (TMEM lane = feature d, column = query), so its
-// fp32 reductions into global memory are coalesced across a warp.
+// with grad(a,i) = dV += P_a^T dO_a, dK += G_a^T Q_a.  S_a(i+1) overwrites the
+// columns holding P_a^T(i); the tensor core runs one thread's MMAs in order, so
+// the dV product has read them first.
 //
 // CTA organisation (persistent, one CTA per SM, 512 threads):
 //   warps 0-3   compute warpgroup 0: query half 0; one key row per thread
 //   warps 4-7   compute warpgroup 1: query half 1
-//   warps 8-11  dQ/epilogue warpgroup: dQ^T read-out and reduction; dK, dV epilogue
+//   warps 8-11  epilogue warpgroup: dK, dV of each key tile
 //   warp 12     TMA producer: K, V per unit; Q, dO per query tile (2 stages)
-//   warp 13     MMA issuer;  warps 14-15 idle
-// TMEM (512 columns): S_0 | S_1 (64 each; P_a^T overwrites the first 32, then
-// dQ_a^T the whole slot) | dP_0 | dP_1 (64 each) | dV (128) | dK (128).
+//   warp 13     MMA issuer
+//   warp 14     TMA store of each G^T half to the global G buffer;  warp 15 idle
+// TMEM (512 columns): S_0 | S_1 (64 each; P_a^T overwrites the first 32) |
+// dP_0 | dP_1 (64 each) | dV (128) | dK (128).
 // Shared memory: K, V, Q[2], dO[2], G^T (all 128x128 bf16, 128-byte swizzled,
 // G^T half a = query columns 64a..64a+63), plus per-half query vectors.
 #pragma once
@@ -40,7 +42,6 @@ namespace ar {
 struct BwdParams {
   __nv_bfloat16* dk;       // [B, T, H, 128]
   __nv_bfloat16* dv;       // [B, T, H, 128]
-  float* dq_acc;           // [B, T, H, 128] fp32 sum_j G_ij k_j (zeroed by the pre-pass)
   const __nv_bfloat16* k;  // [B, T, H, 128] raw keys, for the dk epilogue
   const float* lse2;       // [B*H, T_pad] lse * log2(e), 0 on padding
   const float* delta;      // [B*H, T_pad] rowsum(dO * o), 0 on padding
@@ -48,9 +49,21 @@ struct BwdParams {
   int B, T, H, T_pad;
   int w;        // left window (w >= T means full causal)
   int nk;       // key tiles per head = ceil(T / 128)
-  int n_units;  // B * H * nk
+  int n_units;  // n_bh * nk
+  int bh0, n_bh;   // heads bh0 .. bh0 + n_bh - 1 (b * H + h) are processed by this launch
+  int nb;          // key tiles in one query tile's band: min(nk, floor((w + 127) / 128) + 1)
+  int pairs_head;  // G tiles per head: sum over query tiles of min(qt + 1, nb)
   float eps, scale;
 };
+
+// Slot of the G tile of (query tile qt, key tile kt) of the launch's head
+// number hl (0 .. n_bh - 1) in the G buffer: query tiles in order, each followed
+// by its band's key tiles, newest first.
+__device__ __forceinline__ long long g_pair(int hl, int qt, int kt, int nb, int pairs_head) {
+  const long long before = qt <= nb ? (long long)qt * (qt + 1) / 2
+                                    : (long long)nb * (nb + 1) / 2 + (long long)(qt - nb) * nb;
+  return (long long)hl * pairs_head + before + (qt - kt);
+}
 
 namespace bwd {
 constexpr int kThreads = 512;
@@ -60,8 +73,7 @@ constexpr uint32_t kTile = 32768, kHalf = 16384;
 constexpr uint32_t kK = 0, kV = kTile, kQ = 2 * kTile, kDO = 4 * kTile, kG = 6 * kTile, kVec = 7 * kTile;
 enum {
   KVFULL = 0, KVEMPTY, QFULL, QEMPTY = QFULL + 2, SFULL = QEMPTY + 2, DSREADY = SFULL + 2, DSFREE = DSREADY + 2,
-  DQFULL = DSFREE + 2, DQFREE = DQFULL + 2, VECFULL = DQFREE + 2, VECEMPTY = VECFULL + 2, DKDVDONE = VECEMPTY + 2,
-  ACCFREE, FINAL, NBAR
+  VECFULL = DSFREE + 2, VECEMPTY = VECFULL + 2, DKDVDONE = VECEMPTY + 2, ACCFREE, FINAL, NBAR
 };
 constexpr uint32_t kVecHalf = 3 * 64 * 4;  // lse2, delta, rq for 64 queries
 constexpr uint32_t kBar = kVec + 2 * kVecHalf;
@@ -71,7 +83,7 @@ constexpr uint32_t kSmemBytes = kAbort + 4 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Unit {
-  int bh, b, h, kt, qlo, N;
+  int hl, bh, b, h, kt, qlo, N;
 };
 
 __device__ __forceinline__ int unit_index(int cta, int round, int G) {
@@ -81,9 +93,9 @@ __device__ __forceinline__ int unit_index(int cta, int round, int G) {
 // Units are (head, key tile), low key tiles first (they see the most queries).
 __device__ __forceinline__ Unit decode(const BwdParams& p, int u) {
   Unit U;
-  const int BH = p.B * p.H;
-  U.kt = u / BH;
-  U.bh = u % BH;
+  U.kt = u / p.n_bh;
+  U.hl = u % p.n_bh;
+  U.bh = p.bh0 + U.hl;
   U.b = U.bh / p.H;
   U.h = U.bh % p.H;
   U.qlo = U.kt;
@@ -94,10 +106,6 @@ __device__ __forceinline__ Unit decode(const BwdParams& p, int u) {
 }
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t sbase, int i) { return sbase + kBar + 8u * i; }
-
-__device__ __forceinline__ void red_add_f32(float* gaddr, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(gaddr), "f"(v) : "memory");
-}
 
 // One 32-query chunk of a key row: P = 2^(S rq_i C_j - lse2_i) (zero outside the
 // band when MASKED), G = P (dP - delta_i) rq_i rk_j, both packed to bf16 pairs.
@@ -138,7 +146,7 @@ __device__ __forceinline__ void grad_chunk(const uint32_t (&sv)[32], const uint3
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-               const BwdParams p) {
+               const __grid_constant__ CUtensorMap tm_g, const BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -149,9 +157,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBAR; ++i) {
       uint32_t cnt = 1;
-      if (i == DSREADY || i == DSREADY + 1 || i == DQFREE || i == DQFREE + 1 || i == VECFULL || i == VECFULL + 1 ||
-          i == VECEMPTY || i == VECEMPTY + 1 || i == ACCFREE)
+      if (i == DSREADY || i == DSREADY + 1 || i == VECFULL || i == VECFULL + 1 || i == VECEMPTY ||
+          i == VECEMPTY + 1 || i == ACCFREE)
         cnt = 128;
+      if (i == DSFREE || i == DSFREE + 1) cnt = 2;  // the MMA commit + the G^T store's read
       if (i == KVEMPTY) cnt = 1 + 256;  // the MMA commit + every compute thread once rk is read
       mbar_init(bar_addr(sbase, i), cnt);
     }
@@ -167,6 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_do);
+    prefetch_tmap(&tm_g);
   }
   tc_fence_before();
   __syncthreads();
@@ -213,11 +223,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 2; ++s)
           if (last_q_par[s] >= 0) mbar_wait(bar_addr(sbase, QFULL + s), last_q_par[s], &never);
       }
+    } else if (warp == 14 && lane == 0) {
+      // ---------------------------------------------------------- G^T stores
+      // Each half of G^T, once its compute warpgroup has written it (DSREADY), is
+      // stored to its slot of the global G buffer; the shared-memory half is
+      // released (the second DSFREE arrival) once the store has read it.
+      uint32_t qc = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int u = unit_index(cta, r, G);
+        if (u >= p.n_units) break;
+        const Unit U = decode(p, u);
+        for (int it = 0; it < U.N && ok; ++it, ++qc) {
+          const long long pair = g_pair(U.hl, U.qlo + it, U.kt, p.nb, p.pairs_head);
+          for (int a = 0; a < 2; ++a) {
+            if (!mbar_wait(bar_addr(sbase, DSREADY + a), qc & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tma_store_2d(&tm_g, sbase + kG + a * kHalf, 0, (int)((2 * pair + a) * 128));
+            bulk_commit();
+            bulk_wait_read();
+            mbar_arrive(bar_addr(sbase, DSFREE + a));
+          }
+        }
+      }
+      bulk_wait_all();  // every G tile has reached global memory
     } else if (warp == 13 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t id_s = idesc_bf16(128, 64, 0, 0);     // S^T, dP^T: both K-major, N = 64 queries
       constexpr uint32_t id_acc = idesc_bf16(128, 128, 0, 1);  // dV, dK: A K-major, B MN-major
-      constexpr uint32_t id_dq = idesc_bf16(128, 64, 1, 1);    // dQ^T: both MN-major
       const uint32_t tDV = tbase + 256, tDK = tbase + 384;
       auto issue_s = [&](int a, int st) {  // S_a^T = K Q_a^T
         const uint32_t qa = sbase + kQ + st * kTile + a * 64 * 128;
@@ -249,10 +284,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < 4; ++kk)  // dK += G_a^T Q_a
           mma_ss(tDK, sdesc_sw128(ga + kk * 32, 16, 1024), sdesc_sw128(qrow + kk * 2048, kHalf, 1024), id_acc,
                  (first && kk == 0) ? 0u : 1u);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // dQ_a^T = K^T G_a^T  (16 keys per step), into slot S_a
-          mma_ss(tbase + 64 * a, sdesc_sw128(sbase + kK + kk * 2048, kHalf, 1024),
-                 sdesc_sw128(ga + kk * 2048, kHalf, 1024), id_dq, kk > 0);
       };
       uint32_t qc = 0;
       int uidx = 0;
@@ -267,7 +298,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(bar_addr(sbase, QFULL + st), ph, abort_flag)) break;
 #pragma unroll
           for (int a = 0; a < 2; ++a) {
-            if (qc > 0 && !mbar_wait(bar_addr(sbase, DQFREE + a), (qc - 1) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             issue_s(a, st);
             issue_dp(a, st);
@@ -286,15 +316,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 !mbar_wait(bar_addr(sbase, ACCFREE), (uidx - 1) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             issue_grad(a, st, it == 0 && a == 0);
-            mma_commit(bar_addr(sbase, DQFULL + a));
             mma_commit(bar_addr(sbase, DSFREE + a));
             if (a == 1) mma_commit(bar_addr(sbase, QEMPTY + st));
             if (has_next) {
               if (a == 0 && !mbar_wait(bar_addr(sbase, QFULL + st1), ph1, abort_flag)) { ok = false; break; }
               tc_fence_after();
               issue_dp(a, st1);
-              if (!mbar_wait(bar_addr(sbase, DQFREE + a), q & 1, abort_flag)) { ok = false; break; }
-              tc_fence_after();
               issue_s(a, st1);
               mma_commit(bar_addr(sbase, SFULL + a));
             }
@@ -415,53 +442,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++uidx;
       }
     } else {
-      // ---------------------------------------------------------- dQ / epilogue warpgroup
-      const int row = threadIdx.x - 256;  // TMEM lane: feature d for dQ^T, key row for dV/dK
+      // ---------------------------------------------------------- dK, dV epilogue warpgroup
+      const int row = threadIdx.x - 256;  // TMEM lane: key row
       const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
       const uint32_t tDV = tbase + 256 + lane_off, tDK = tbase + 384 + lane_off;
-      uint32_t qc = 0;
       int uidx = 0;
-      bool ok = true;
-      for (int r = 0; ok; ++r) {
+      for (int r = 0;; ++r) {
         const int u = unit_index(cta, r, G);
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
-        for (int it = 0; it < U.N && ok; ++it, ++qc) {
-          const int qt = U.qlo + it;
-#pragma unroll 1
-          for (int a = 0; a < 2; ++a) {
-            if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DQFULL + a), qc & 1, abort_flag))) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            uint32_t x[64];
-            tmem_ld32(tbase + 64 * a + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
-            tmem_ld32(tbase + 64 * a + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(bar_addr(sbase, DQFREE + a));
-            const int i0 = qt * 128 + 64 * a;
-            const int nvalid = min(64, p.T - i0);
-            float* dst = p.dq_acc + (((size_t)U.b * p.T + i0) * p.H + U.h) * 128 + row;
-            const size_t stride = (size_t)p.H * 128;
-            if (nvalid == 64) {
-#pragma unroll
-              for (int c = 0; c < 64; ++c) red_add_f32(dst + c * stride, __uint_as_float(x[c]));
-            } else {
-#pragma unroll
-              for (int c = 0; c < 64; ++c)
-                if (c < nvalid) red_add_f32(dst + c * stride, __uint_as_float(x[c]));
-            }
-          }
-        }
-        if (!ok) break;
         // ------------------------------------------------------------ dV, dK epilogue
+        const int j = U.kt * 128 + row;
+        const size_t orow = (((size_t)U.b * p.T + (j < p.T ? j : 0)) * p.H + U.h) * 128;
+        const bool jv = j < p.T;
+        // the raw key row for the k-side norm backward
+        const uint4* krow = reinterpret_cast<const uint4*>(p.k + orow);
+        if (jv) {  // pull the row towards L2 while the products finish
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(krow));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(krow + 8));
+        }
         if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DKDVDONE), uidx & 1, abort_flag))) break;
         tc_fence_after();
-        const int j = U.kt * 128 + row;
-        const size_t orow = (((size_t)U.b * p.T + j) * p.H + U.h) * 128;
-        const bool jv = j < p.T;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t x[32];
@@ -478,9 +479,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // dk = scale (acc - rk^2 k (acc . k) / D), with k and rk from the raw key row
         {
-          const uint4* krow = reinterpret_cast<const uint4*>(p.k + orow);
           float ss = 0.f, dot = 0.f;
-#pragma unroll 1
+#pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t x[32];
             tmem_ld32(tDK + 32 * c, x);
@@ -498,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           const float coef = dot * (1.0f / 128.0f) / (ss * (1.0f / 128.0f) + p.eps);
-#pragma unroll 1
+#pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t x[32];
             tmem_ld32(tDK + 32 * c, x);

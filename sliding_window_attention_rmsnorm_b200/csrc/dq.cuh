@@ -1,0 +1,250 @@
+// Query gradient of the fused QK-RMSNorm attention backward, sm_100a.
+//
+// dq = rq (dqhat - qhat (dqhat . qhat) / D), qhat = rq q: the RMSNorm backward
+// (the same formula as for k) applied to dqhat_i = scale sum_j dS_ij khat_j,
+// the attention gradient of the query (FlashAttention backward; norm(q) before
+// the attention product as in the "autoresearch" README (gitee), section 7.3).
+//
+// The backward main kernel stores, for every (query tile, key tile) pair of the
+// band, the bf16 tile G^T with G_ij = dS_ij rq_i rk_j.  Here one CTA owns one
+// 128-query tile at a time and accumulates, in TMEM,
+//   acc_i = sum_j G_ij k_j = rq_i dqhat_i / scale      (raw bf16 k rows)
+// over the tile's band, then finishes dq_i = scale (acc_i - c_i q_i) with
+// c_i = (acc_i . q_i) / D / (mean q_i^2 + eps) and writes it as bf16.
+//
+// CTA organisation (persistent, one CTA per SM, 192 threads):
+//   warps 0-3  epilogue warpgroup: one query row per thread
+//   warp 4     TMA producer: G tile (two 64-query halves) + K tile per stage
+//   warp 5     MMA issuer
+// TMEM: two 128-column accumulators, so one tile's epilogue overlaps the next
+// tile's products.  The product is acc (M = 128 queries, N = 128 features,
+// K = 16 keys per step) with A = G read from the G^T tile (queries contiguous:
+// MN-major) and B = the K tile (features contiguous: MN-major).
+#pragma once
+#include "sm100.cuh"
+
+namespace ar {
+
+struct DqParams {
+  const __nv_bfloat16* q;  // [B, T, H, 128]
+  __nv_bfloat16* dq;       // [B, T, H, 128]
+  int B, T, H;
+  int w;           // left window (w >= T means full causal)
+  int nq;          // query tiles per head
+  int n_units;     // n_bh * nq
+  int bh0, n_bh;   // heads processed by this launch (as in the backward kernel)
+  int nb;          // key tiles in one query tile's band (as in the backward kernel)
+  int pairs_head;  // G tiles per head
+  float eps, scale;
+};
+
+namespace dqk {
+constexpr int kThreads = 192;
+constexpr uint32_t kTile = 32768, kHalf = 16384;
+constexpr int kStages = 3;
+constexpr uint32_t kStage = 2 * kTile;  // G tile + K tile
+enum { FULL = 0, EMPTY = FULL + kStages, ACCFULL = EMPTY + kStages, ACCFREE = ACCFULL + 2, FINAL = ACCFREE + 2, NBAR };
+constexpr uint32_t kBar = kStages * kStage;
+constexpr uint32_t kTmemPtr = kBar + NBAR * 8;
+constexpr uint32_t kAbort = kTmemPtr + 4;
+constexpr uint32_t kSmemBytes = kAbort + 4 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+struct Unit {
+  int hl, bh, b, h, qt, klo, N;
+};
+
+__device__ __forceinline__ int unit_index(int cta, int round, int G) {
+  return round * G + ((round & 1) ? (G - 1 - cta) : cta);
+}
+
+// Units are (head, query tile), later query tiles (longer bands) first.
+__device__ __forceinline__ Unit decode(const DqParams& p, int u) {
+  Unit U;
+  U.qt = p.nq - 1 - u / p.n_bh;
+  U.hl = u % p.n_bh;
+  U.bh = p.bh0 + U.hl;
+  U.b = U.bh / p.H;
+  U.h = U.bh % p.H;
+  U.klo = max(0, U.qt * 128 - p.w) / 128;
+  U.N = U.qt - U.klo + 1;
+  return U;
+}
+
+// Same slot layout as g_pair in the backward kernel.
+__device__ __forceinline__ long long g_slot(const DqParams& p, int hl, int qt, int kt) {
+  const long long before = qt <= p.nb ? (long long)qt * (qt + 1) / 2
+                                      : (long long)p.nb * (p.nb + 1) / 2 + (long long)(qt - p.nb) * p.nb;
+  return (long long)hl * p.pairs_head + before + (qt - kt);
+}
+
+__device__ __forceinline__ uint32_t bar_addr(uint32_t sbase, int i) { return sbase + kBar + 8u * i; }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    dq_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_k, const DqParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kAbort);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int G = gridDim.x, cta = blockIdx.x;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar_addr(sbase, i), (i == ACCFREE || i == ACCFREE + 1) ? 128 : 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(sbase + kTmemPtr, 256);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&tm_g);
+    prefetch_tmap(&tm_k);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + kTmemPtr);
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- TMA producer
+      uint32_t c = 0;
+      bool ok = true;
+      int last_par[kStages] = {-1, -1, -1};
+      for (int r = 0; ok; ++r) {
+        const int u = unit_index(cta, r, G);
+        if (u >= p.n_units) break;
+        const Unit U = decode(p, u);
+        for (int it = 0; it < U.N; ++it, ++c) {
+          const int kt = U.qt - it;
+          const int s = c % kStages, ph = (c / kStages) & 1;
+          if (!mbar_wait(bar_addr(sbase, EMPTY + s), ph ^ 1, abort_flag)) { ok = false; break; }
+          const uint32_t st = sbase + s * kStage;
+          const long long slot = g_slot(p, U.hl, U.qt, kt);
+          mbar_expect_tx(bar_addr(sbase, FULL + s), kStage);
+          for (int hf = 0; hf < 2; ++hf) {
+            tma_load_2d(st + hf * kHalf, &tm_g, bar_addr(sbase, FULL + s), 0, (int)((2 * slot + hf) * 128));
+            tma_load_4d(st + kTile + hf * kHalf, &tm_k, bar_addr(sbase, FULL + s), hf * 64, U.h, kt * 128, U.b);
+          }
+          last_par[s] = ph;
+        }
+      }
+      if (*abort_flag) {
+        volatile int never = 0;
+        for (int s = 0; s < kStages; ++s)
+          if (last_par[s] >= 0) mbar_wait(bar_addr(sbase, FULL + s), last_par[s], &never);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t id = idesc_bf16(128, 128, 1, 1);  // A (G) and B (K) both MN-major
+      const uint64_t dA = sdesc_sw128(sbase, kHalf, 1024), dB = sdesc_sw128(sbase + kTile, kHalf, 1024);
+      uint32_t c = 0;
+      int uidx = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int u = unit_index(cta, r, G);
+        if (u >= p.n_units) break;
+        const Unit U = decode(p, u);
+        const int ab = uidx & 1;
+        if (uidx >= 2 && !mbar_wait(bar_addr(sbase, ACCFREE + ab), ((uidx >> 1) - 1) & 1, abort_flag)) break;
+        for (int it = 0; it < U.N; ++it, ++c) {
+          const int s = c % kStages, ph = (c / kStages) & 1;
+          if (!mbar_wait(bar_addr(sbase, FULL + s), ph, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tbase + 128 * ab, sdesc_add(dA, s * kStage + kk * 2048), sdesc_add(dB, s * kStage + kk * 2048), id,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar_addr(sbase, EMPTY + s));
+        }
+        if (!ok) break;
+        mma_commit(bar_addr(sbase, ACCFULL + ab));
+        ++uidx;
+      }
+      mma_commit(bar_addr(sbase, FINAL));
+      volatile int never = 0;
+      mbar_wait(bar_addr(sbase, FINAL), 0, &never);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int row = threadIdx.x;  // TMEM lane = query row of the tile
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    int uidx = 0;
+    for (int r = 0;; ++r) {
+      const int u = unit_index(cta, r, G);
+      if (u >= p.n_units) break;
+      const Unit U = decode(p, u);
+      const int ab = uidx & 1;
+      const int i = U.qt * 128 + row;
+      const bool iv = i < p.T;
+      const size_t orow = (((size_t)U.b * p.T + (iv ? i : 0)) * p.H + U.h) * 128;
+      // the whole q row, loaded before the wait for the accumulator so that its
+      // latency overlaps the tile's products
+      uint4 qv[16];
+      {
+        const uint4* qrow = reinterpret_cast<const uint4*>(p.q + orow);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) qv[c] = iv ? __ldg(qrow + c) : make_uint4(0, 0, 0, 0);
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, ACCFULL + ab), (uidx >> 1) & 1, abort_flag))) break;
+      tc_fence_after();
+      const uint32_t tA = tbase + 128 * ab + lane_off;
+      // pass 1: (acc . q) and sum q^2
+      float ss = 0.f, dot = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t x[32];
+        tmem_ld32(tA + 32 * cc, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint4 v = qv[4 * cc + q4];
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float q0 = bf16lo(w4[e]), q1 = bf16hi(w4[e]);
+            ss = fmaf(q0, q0, fmaf(q1, q1, ss));
+            dot = fmaf(__uint_as_float(x[8 * q4 + 2 * e]), q0, fmaf(__uint_as_float(x[8 * q4 + 2 * e + 1]), q1, dot));
+          }
+        }
+      }
+      const float coef = dot * (1.0f / 128.0f) / (ss * (1.0f / 128.0f) + p.eps);
+      // pass 2: dq = scale (acc - coef q)
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t x[32];
+        tmem_ld32(tA + 32 * cc, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint4 v = qv[4 * cc + q4];
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+          uint32_t o4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float g0 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e]) - coef * bf16lo(w4[e]));
+            const float g1 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e + 1]) - coef * bf16hi(w4[e]));
+            o4[e] = pack_bf16(g0, g1);
+          }
+          if (iv) *reinterpret_cast<uint4*>(p.dq + orow + 32 * cc + 8 * q4) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_addr(sbase, ACCFREE + ab));
+      ++uidx;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 256);
+  }
+}
+
+}  // namespace dqk
+}  // namespace ar

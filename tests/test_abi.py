@@ -72,9 +72,14 @@ def test_workspace_sizes(L):
     # the forward kernel derives the per-key norm factors itself: no scratch
     assert attn.fwd_workspace_bytes(B, T, H, D) == 0
     assert attn.fwd_workspace_bytes(1, 200, 1, 128) == 0
-    assert attn.bwd_workspace_bytes(B, T, H, D) == B * T * H * D * 4 + 3 * B * H * T * 4
-    # ragged T rounds the per-token vectors up to whole 128-token tiles
-    assert attn.bwd_workspace_bytes(1, 200, 1, 128) == 200 * 128 * 4 + 3 * 256 * 4
+    # three per-token fp32 vectors + one 32 KB G tile per (query tile, key tile)
+    # pair of the full causal band, nq (nq + 1) / 2 per head (nq = 16 here)
+    assert attn.bwd_workspace_bytes(B, T, H, D) == 3 * B * H * T * 4 + B * H * 136 * 32768
+    # ragged T rounds the per-token vectors up to whole 128-token tiles (nq = 2: 3 tiles)
+    assert attn.bwd_workspace_bytes(1, 200, 1, 128) == 3 * 256 * 4 + 3 * 32768
+    # heads are grouped so that the G tiles fit in 1 GiB: T = 8192 gives 2080 tiles per
+    # head (68 MB), 15 heads per group
+    assert attn.bwd_workspace_bytes(4, 8192, 8, 128) == 3 * 32 * 8192 * 4 + 15 * 2080 * 32768
     assert attn.bwd_workspace_bytes(0, 200, 1, 128) == 0
     assert attn.bwd_workspace_bytes(1, 200, 1, 64) == 0
 
