@@ -304,6 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(bar_addr(sbase, SFULL + a));
           }
           if (!ok) break;
+          // K and V are read only by the S and dP products: once the last of
+          // them is issued, the next unit's tiles may start loading
+          if (U.N == 1) mma_commit(bar_addr(sbase, KVEMPTY));
         }
         for (int it = 0; it < U.N && ok; ++it) {
           const uint32_t q = qc + it, q1 = q + 1;
@@ -324,12 +327,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               issue_dp(a, st1);
               issue_s(a, st1);
               mma_commit(bar_addr(sbase, SFULL + a));
+              if (a == 1 && it + 2 == U.N) mma_commit(bar_addr(sbase, KVEMPTY));
             }
           }
         }
         if (!ok) break;
         mma_commit(bar_addr(sbase, DKDVDONE));
-        mma_commit(bar_addr(sbase, KVEMPTY));
         qc += U.N;
         ++uidx;
       }
@@ -451,34 +454,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = unit_index(cta, r, G);
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
-        // ------------------------------------------------------------ dV, dK epilogue
+        // ------------------------------------------------------------ dK, dV epilogue
         const int j = U.kt * 128 + row;
         const size_t orow = (((size_t)U.b * p.T + (j < p.T ? j : 0)) * p.H + U.h) * 128;
         const bool jv = j < p.T;
-        // the raw key row for the k-side norm backward
-        const uint4* krow = reinterpret_cast<const uint4*>(p.k + orow);
-        if (jv) {  // pull the row towards L2 while the products finish
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(krow));
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(krow + 8));
-        }
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DKDVDONE), uidx & 1, abort_flag))) break;
-        tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t x[32];
-          tmem_ld32(tDV + 32 * c, x);
-          tmem_wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]));
-          if (jv) {
-            uint4* d = reinterpret_cast<uint4*>(p.dv + orow + 32 * c);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) d[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-          }
-        }
-        // dk = scale (acc - rk^2 k (acc . k) / D), with k and rk from the raw key row
+        // dk = scale (acc - rk^2 k (acc . k) / D), with k and rk from the raw key
+        // row, pulled towards L2 before the wait so that its latency overlaps the
+        // unit's last products
         {
+          const uint4* krow = reinterpret_cast<const uint4*>(p.k + orow);
+          if (jv) {
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(krow));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(krow + 8));
+          }
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DKDVDONE), uidx & 1, abort_flag))) break;
+          tc_fence_after();
           float ss = 0.f, dot = 0.f;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -517,6 +507,20 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (jv)
                 *reinterpret_cast<uint4*>(p.dk + orow + 32 * c + 8 * q4) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
             }
+          }
+        }
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t x[32];
+          tmem_ld32(tDV + 32 * c, x);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]));
+          if (jv) {
+            uint4* d = reinterpret_cast<uint4*>(p.dv + orow + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
           }
         }
         tc_fence_before();

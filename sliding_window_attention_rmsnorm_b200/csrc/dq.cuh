@@ -12,10 +12,12 @@
 // over the tile's band, then finishes dq_i = scale (acc_i - c_i q_i) with
 // c_i = (acc_i . q_i) / D / (mean q_i^2 + eps) and writes it as bf16.
 //
-// CTA organisation (persistent, one CTA per SM, 192 threads):
+// CTA organisation (persistent, one CTA per SM, 224 threads):
 //   warps 0-3  epilogue warpgroup: one query row per thread
-//   warp 4     TMA producer: G tile (two 64-query halves) + K tile per stage
+//   warp 4     TMA producer of the G tiles (two 64-query halves each; 4 stages:
+//              they come from DRAM, so they get the deeper ring)
 //   warp 5     MMA issuer
+//   warp 6     TMA producer of the K tiles (3 stages; mostly L2 hits)
 // TMEM: two 128-column accumulators, so one tile's epilogue overlaps the next
 // tile's products.  The product is acc (M = 128 queries, N = 128 features,
 // K = 16 keys per step) with A = G read from the G^T tile (queries contiguous:
@@ -39,12 +41,15 @@ struct DqParams {
 };
 
 namespace dqk {
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr uint32_t kTile = 32768, kHalf = 16384;
-constexpr int kStages = 3;
-constexpr uint32_t kStage = 2 * kTile;  // G tile + K tile
-enum { FULL = 0, EMPTY = FULL + kStages, ACCFULL = EMPTY + kStages, ACCFREE = ACCFULL + 2, FINAL = ACCFREE + 2, NBAR };
-constexpr uint32_t kBar = kStages * kStage;
+constexpr int kGStages = 4, kKStages = 3;
+constexpr uint32_t kG = 0, kK = kGStages * kTile;
+enum {
+  GFULL = 0, GEMPTY = GFULL + kGStages, KFULL = GEMPTY + kGStages, KEMPTY = KFULL + kKStages,
+  ACCFULL = KEMPTY + kKStages, ACCFREE = ACCFULL + 2, FINAL = ACCFREE + 2, NBAR
+};
+constexpr uint32_t kBar = kK + kKStages * kTile;
 constexpr uint32_t kTmemPtr = kBar + NBAR * 8;
 constexpr uint32_t kAbort = kTmemPtr + 4;
 constexpr uint32_t kSmemBytes = kAbort + 4 + 1024;
@@ -98,7 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(sbase + kTmemPtr, 256);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if ((warp == 4 || warp == 6) && lane == 0) {
     prefetch_tmap(&tm_g);
     prefetch_tmap(&tm_k);
   }
@@ -107,41 +112,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + kTmemPtr);
 
-  if (warp == 4) {
+  if (warp == 4 || warp == 6) {
     if (lane == 0) {
-      // ---------------------------------------------------------- TMA producer
+      // ---------------------------------------------------------- TMA producers: G (warp 4), K (warp 6)
+      const bool is_g = warp == 4;
+      const int nst = is_g ? kGStages : kKStages;
+      const int full = is_g ? GFULL : KFULL, empty = is_g ? GEMPTY : KEMPTY;
       uint32_t c = 0;
       bool ok = true;
-      int last_par[kStages] = {-1, -1, -1};
+      int last_par[kGStages] = {-1, -1, -1, -1};
       for (int r = 0; ok; ++r) {
         const int u = unit_index(cta, r, G);
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
         for (int it = 0; it < U.N; ++it, ++c) {
           const int kt = U.qt - it;
-          const int s = c % kStages, ph = (c / kStages) & 1;
-          if (!mbar_wait(bar_addr(sbase, EMPTY + s), ph ^ 1, abort_flag)) { ok = false; break; }
-          const uint32_t st = sbase + s * kStage;
-          const long long slot = g_slot(p, U.hl, U.qt, kt);
-          mbar_expect_tx(bar_addr(sbase, FULL + s), kStage);
-          for (int hf = 0; hf < 2; ++hf) {
-            tma_load_2d(st + hf * kHalf, &tm_g, bar_addr(sbase, FULL + s), 0, (int)((2 * slot + hf) * 128));
-            tma_load_4d(st + kTile + hf * kHalf, &tm_k, bar_addr(sbase, FULL + s), hf * 64, U.h, kt * 128, U.b);
+          const int s = c % nst, ph = (c / nst) & 1;
+          if (!mbar_wait(bar_addr(sbase, empty + s), ph ^ 1, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(bar_addr(sbase, full + s), kTile);
+          if (is_g) {
+            const long long slot = g_slot(p, U.hl, U.qt, kt);
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_2d(sbase + kG + s * kTile + hf * kHalf, &tm_g, bar_addr(sbase, full + s), 0,
+                          (int)((2 * slot + hf) * 128));
+          } else {
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_4d(sbase + kK + s * kTile + hf * kHalf, &tm_k, bar_addr(sbase, full + s), hf * 64, U.h,
+                          kt * 128, U.b);
           }
           last_par[s] = ph;
         }
       }
       if (*abort_flag) {
         volatile int never = 0;
-        for (int s = 0; s < kStages; ++s)
-          if (last_par[s] >= 0) mbar_wait(bar_addr(sbase, FULL + s), last_par[s], &never);
+        for (int s = 0; s < nst; ++s)
+          if (last_par[s] >= 0) mbar_wait(bar_addr(sbase, full + s), last_par[s], &never);
       }
     }
   } else if (warp == 5) {
     if (lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t id = idesc_bf16(128, 128, 1, 1);  // A (G) and B (K) both MN-major
-      const uint64_t dA = sdesc_sw128(sbase, kHalf, 1024), dB = sdesc_sw128(sbase + kTile, kHalf, 1024);
+      const uint64_t dA = sdesc_sw128(sbase + kG, kHalf, 1024), dB = sdesc_sw128(sbase + kK, kHalf, 1024);
       uint32_t c = 0;
       int uidx = 0;
       bool ok = true;
@@ -152,14 +164,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ab = uidx & 1;
         if (uidx >= 2 && !mbar_wait(bar_addr(sbase, ACCFREE + ab), ((uidx >> 1) - 1) & 1, abort_flag)) break;
         for (int it = 0; it < U.N; ++it, ++c) {
-          const int s = c % kStages, ph = (c / kStages) & 1;
-          if (!mbar_wait(bar_addr(sbase, FULL + s), ph, abort_flag)) { ok = false; break; }
+          const int gs = c % kGStages, gph = (c / kGStages) & 1;
+          const int ks = c % kKStages, kph = (c / kKStages) & 1;
+          if (!mbar_wait(bar_addr(sbase, GFULL + gs), gph, abort_flag) ||
+              !mbar_wait(bar_addr(sbase, KFULL + ks), kph, abort_flag)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tbase + 128 * ab, sdesc_add(dA, s * kStage + kk * 2048), sdesc_add(dB, s * kStage + kk * 2048), id,
+            mma_ss(tbase + 128 * ab, sdesc_add(dA, gs * kTile + kk * 2048), sdesc_add(dB, ks * kTile + kk * 2048), id,
                    (it > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(bar_addr(sbase, EMPTY + s));
+          mma_commit(bar_addr(sbase, GEMPTY + gs));
+          mma_commit(bar_addr(sbase, KEMPTY + ks));
         }
         if (!ok) break;
         mma_commit(bar_addr(sbase, ACCFULL + ab));
