@@ -6,20 +6,23 @@
 // the attention product as in the "autoresearch" README (gitee), section 7.3).
 //
 // The backward main kernel stores, for every (query tile, key tile) pair of the
-// band, the bf16 tile G^T with G_ij = dS_ij rq_i rk_j.  Here one CTA owns one
-// 128-query tile at a time and accumulates, in TMEM,
+// band, the bf16 tile G^T with G_ij = dS_ij rq_i rk_j.  Here one CTA owns two
+// consecutive 128-query tiles at a time (a unit) and accumulates, in TMEM,
 //   acc_i = sum_j G_ij k_j = rq_i dqhat_i / scale      (raw bf16 k rows)
-// over the tile's band, then finishes dq_i = scale (acc_i - c_i q_i) with
-// c_i = (acc_i . q_i) / D / (mean q_i^2 + eps) and writes it as bf16.
+// over each tile's band, then finishes dq_i = scale (acc_i - c_i q_i) with
+// c_i = (acc_i . q_i) / D / (mean q_i^2 + eps) and writes it as bf16.  The two
+// tiles' bands overlap in all but one key tile, so each K tile is loaded once
+// for both: the kernel streams 32 KB per G tile plus 32 KB per K tile, which
+// is what bounds it (the SM's TMA ingest, about 64 bytes per clock).
 //
 // CTA organisation (persistent, one CTA per SM, 224 threads):
-//   warps 0-3  epilogue warpgroup: one query row per thread
-//   warp 4     TMA producer of the G tiles (two 64-query halves each; 4 stages:
-//              they come from DRAM, so they get the deeper ring)
+//   warps 0-3  epilogue warpgroup: one query row per thread, tile 0 then tile 1
+//   warp 4     TMA producer of the G tiles (two 64-query halves each; 4 stages)
 //   warp 5     MMA issuer
-//   warp 6     TMA producer of the K tiles (3 stages; mostly L2 hits)
-// TMEM: two 128-column accumulators, so one tile's epilogue overlaps the next
-// tile's products.  The product is acc (M = 128 queries, N = 128 features,
+//   warp 6     TMA producer of the K tiles (3 stages)
+// TMEM (512 columns): accumulators for the unit's two tiles, double-buffered
+// (column 256 * buffer + 128 * tile), so one unit's epilogue overlaps the next
+// unit's products.  The product is acc (M = 128 queries, N = 128 features,
 // K = 16 keys per step) with A = G read from the G^T tile (queries contiguous:
 // MN-major) and B = the K tile (features contiguous: MN-major).
 #pragma once
@@ -33,7 +36,7 @@ struct DqParams {
   int B, T, H;
   int w;           // left window (w >= T means full causal)
   int nq;          // query tiles per head
-  int n_units;     // n_bh * nq
+  int n_units;     // n_bh * ceil(nq / 2)
   int bh0, n_bh;   // heads processed by this launch (as in the backward kernel)
   int nb;          // key tiles in one query tile's band (as in the backward kernel)
   int pairs_head;  // G tiles per head
@@ -55,24 +58,36 @@ constexpr uint32_t kAbort = kTmemPtr + 4;
 constexpr uint32_t kSmemBytes = kAbort + 4 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
+// A unit: query tiles q0 = 2 qp and q1 = q0 + 1 (q1 only if has1) of one head;
+// key tiles kt = khi down to klo, where tile t uses kt in [lo[t], hi[t]].
 struct Unit {
-  int hl, bh, b, h, qt, klo, N;
+  int hl, bh, b, h, q0, has1, khi, klo, lo[2], hi[2];
+  __device__ bool in(int t, int kt) const { return (t == 0 || has1) && kt >= lo[t] && kt <= hi[t]; }
 };
 
 __device__ __forceinline__ int unit_index(int cta, int round, int G) {
   return round * G + ((round & 1) ? (G - 1 - cta) : cta);
 }
 
-// Units are (head, query tile), later query tiles (longer bands) first.
+// Units are (head, pair of query tiles), later pairs (longer bands) first.
 __device__ __forceinline__ Unit decode(const DqParams& p, int u) {
   Unit U;
-  U.qt = p.nq - 1 - u / p.n_bh;
+  const int npairs = (p.nq + 1) / 2;
+  const int qp = npairs - 1 - u / p.n_bh;
   U.hl = u % p.n_bh;
   U.bh = p.bh0 + U.hl;
   U.b = U.bh / p.H;
   U.h = U.bh % p.H;
-  U.klo = max(0, U.qt * 128 - p.w) / 128;
-  U.N = U.qt - U.klo + 1;
+  U.q0 = 2 * qp;
+  U.has1 = U.q0 + 1 < p.nq;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qt = U.q0 + t;
+    U.lo[t] = max(0, qt * 128 - p.w) / 128;
+    U.hi[t] = qt;
+  }
+  U.klo = U.lo[0];
+  U.khi = U.has1 ? U.hi[1] : U.hi[0];
   return U;
 }
 
@@ -100,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (warp == 5) {
-    tmem_alloc(sbase + kTmemPtr, 256);
+    tmem_alloc(sbase + kTmemPtr, 512);
     tmem_relinquish();
   }
   if ((warp == 4 || warp == 6) && lane == 0) {
@@ -115,6 +130,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 4 || warp == 6) {
     if (lane == 0) {
       // ---------------------------------------------------------- TMA producers: G (warp 4), K (warp 6)
+      // Both walk the unit's key tiles newest first; the G producer loads, per key
+      // tile, the G tile of each query tile whose band holds it (tile 0 first).
       const bool is_g = warp == 4;
       const int nst = is_g ? kGStages : kKStages;
       const int full = is_g ? GFULL : KFULL, empty = is_g ? GEMPTY : KEMPTY;
@@ -125,22 +142,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = unit_index(cta, r, G);
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
-        for (int it = 0; it < U.N; ++it, ++c) {
-          const int kt = U.qt - it;
-          const int s = c % nst, ph = (c / nst) & 1;
-          if (!mbar_wait(bar_addr(sbase, empty + s), ph ^ 1, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(bar_addr(sbase, full + s), kTile);
-          if (is_g) {
-            const long long slot = g_slot(p, U.hl, U.qt, kt);
-            for (int hf = 0; hf < 2; ++hf)
-              tma_load_2d(sbase + kG + s * kTile + hf * kHalf, &tm_g, bar_addr(sbase, full + s), 0,
-                          (int)((2 * slot + hf) * 128));
-          } else {
-            for (int hf = 0; hf < 2; ++hf)
-              tma_load_4d(sbase + kK + s * kTile + hf * kHalf, &tm_k, bar_addr(sbase, full + s), hf * 64, U.h,
-                          kt * 128, U.b);
+        for (int kt = U.khi; kt >= U.klo && ok; --kt) {
+          for (int t = 0; t < (is_g ? 2 : 1); ++t) {
+            if (is_g && !U.in(t, kt)) continue;
+            const int s = c % nst, ph = (c / nst) & 1;
+            if (!mbar_wait(bar_addr(sbase, empty + s), ph ^ 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(bar_addr(sbase, full + s), kTile);
+            if (is_g) {
+              const long long slot = g_slot(p, U.hl, U.q0 + t, kt);
+              for (int hf = 0; hf < 2; ++hf)
+                tma_load_2d(sbase + kG + s * kTile + hf * kHalf, &tm_g, bar_addr(sbase, full + s), 0,
+                            (int)((2 * slot + hf) * 128));
+            } else {
+              for (int hf = 0; hf < 2; ++hf)
+                tma_load_4d(sbase + kK + s * kTile + hf * kHalf, &tm_k, bar_addr(sbase, full + s), hf * 64, U.h,
+                            kt * 128, U.b);
+            }
+            last_par[s] = ph;
+            ++c;
           }
-          last_par[s] = ph;
         }
       }
       if (*abort_flag) {
@@ -154,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t id = idesc_bf16(128, 128, 1, 1);  // A (G) and B (K) both MN-major
       const uint64_t dA = sdesc_sw128(sbase + kG, kHalf, 1024), dB = sdesc_sw128(sbase + kK, kHalf, 1024);
-      uint32_t c = 0;
+      uint32_t cg = 0, ck = 0;
       int uidx = 0;
       bool ok = true;
       for (int r = 0; ok; ++r) {
@@ -163,20 +186,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Unit U = decode(p, u);
         const int ab = uidx & 1;
         if (uidx >= 2 && !mbar_wait(bar_addr(sbase, ACCFREE + ab), ((uidx >> 1) - 1) & 1, abort_flag)) break;
-        for (int it = 0; it < U.N; ++it, ++c) {
-          const int gs = c % kGStages, gph = (c / kGStages) & 1;
-          const int ks = c % kKStages, kph = (c / kKStages) & 1;
-          if (!mbar_wait(bar_addr(sbase, GFULL + gs), gph, abort_flag) ||
-              !mbar_wait(bar_addr(sbase, KFULL + ks), kph, abort_flag)) {
+        for (int kt = U.khi; kt >= U.klo && ok; --kt, ++ck) {
+          const int ks = ck % kKStages, kph = (ck / kKStages) & 1;
+          if (!mbar_wait(bar_addr(sbase, KFULL + ks), kph, abort_flag)) {
             ok = false;
             break;
           }
-          tc_fence_after();
+          for (int t = 0; t < 2; ++t) {
+            if (!U.in(t, kt)) continue;
+            const int gs = cg % kGStages, gph = (cg / kGStages) & 1;
+            if (!mbar_wait(bar_addr(sbase, GFULL + gs), gph, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const bool first = kt == U.hi[t];
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tbase + 128 * ab, sdesc_add(dA, gs * kTile + kk * 2048), sdesc_add(dB, ks * kTile + kk * 2048), id,
-                   (it > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(bar_addr(sbase, GEMPTY + gs));
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tbase + 256 * ab + 128 * t, sdesc_add(dA, gs * kTile + kk * 2048),
+                     sdesc_add(dB, ks * kTile + kk * 2048), id, (!first || kk > 0) ? 1u : 0u);
+            mma_commit(bar_addr(sbase, GEMPTY + gs));
+            ++cg;
+          }
           mma_commit(bar_addr(sbase, KEMPTY + ks));
         }
         if (!ok) break;
@@ -189,68 +220,77 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int row = threadIdx.x;  // TMEM lane = query row of the tile
+    const int row = threadIdx.x;  // TMEM lane = query row of a tile
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     int uidx = 0;
-    for (int r = 0;; ++r) {
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
       const int u = unit_index(cta, r, G);
       if (u >= p.n_units) break;
       const Unit U = decode(p, u);
       const int ab = uidx & 1;
-      const int i = U.qt * 128 + row;
-      const bool iv = i < p.T;
-      const size_t orow = (((size_t)U.b * p.T + (iv ? i : 0)) * p.H + U.h) * 128;
-      // the whole q row, loaded before the wait for the accumulator so that its
-      // latency overlaps the tile's products
-      uint4 qv[16];
-      {
-        const uint4* qrow = reinterpret_cast<const uint4*>(p.q + orow);
+      for (int t = 0; t < 1 + U.has1; ++t) {
+        const int i = (U.q0 + t) * 128 + row;
+        const bool iv = i < p.T;
+        const size_t orow = (((size_t)U.b * p.T + (iv ? i : 0)) * p.H + U.h) * 128;
+        // the whole q row, loaded before the wait for the accumulator so that its
+        // latency overlaps the products
+        uint4 qv[16];
+        {
+          const uint4* qrow = reinterpret_cast<const uint4*>(p.q + orow);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) qv[c] = iv ? __ldg(qrow + c) : make_uint4(0, 0, 0, 0);
-      }
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, ACCFULL + ab), (uidx >> 1) & 1, abort_flag))) break;
-      tc_fence_after();
-      const uint32_t tA = tbase + 128 * ab + lane_off;
-      // pass 1: (acc . q) and sum q^2
-      float ss = 0.f, dot = 0.f;
+          for (int c = 0; c < 16; ++c) qv[c] = iv ? __ldg(qrow + c) : make_uint4(0, 0, 0, 0);
+        }
+        if (t == 0 &&
+            !__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, ACCFULL + ab), (uidx >> 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tA = tbase + 256 * ab + 128 * t + lane_off;
+        // pass 1: (acc . q) and sum q^2
+        float ss = 0.f, dot = 0.f;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t x[32];
-        tmem_ld32(tA + 32 * cc, x);
-        tmem_wait_ld();
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t x[32];
+          tmem_ld32(tA + 32 * cc, x);
+          tmem_wait_ld();
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const uint4 v = qv[4 * cc + q4];
-          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint4 v = qv[4 * cc + q4];
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float q0 = bf16lo(w4[e]), q1 = bf16hi(w4[e]);
-            ss = fmaf(q0, q0, fmaf(q1, q1, ss));
-            dot = fmaf(__uint_as_float(x[8 * q4 + 2 * e]), q0, fmaf(__uint_as_float(x[8 * q4 + 2 * e + 1]), q1, dot));
+            for (int e = 0; e < 4; ++e) {
+              const float q0 = bf16lo(w4[e]), q1 = bf16hi(w4[e]);
+              ss = fmaf(q0, q0, fmaf(q1, q1, ss));
+              dot = fmaf(__uint_as_float(x[8 * q4 + 2 * e]), q0, fmaf(__uint_as_float(x[8 * q4 + 2 * e + 1]), q1, dot));
+            }
+          }
+        }
+        const float coef = dot * (1.0f / 128.0f) / (ss * (1.0f / 128.0f) + p.eps);
+        // pass 2: dq = scale (acc - coef q)
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t x[32];
+          tmem_ld32(tA + 32 * cc, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint4 v = qv[4 * cc + q4];
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float g0 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e]) - coef * bf16lo(w4[e]));
+              const float g1 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e + 1]) - coef * bf16hi(w4[e]));
+              o4[e] = pack_bf16(g0, g1);
+            }
+            if (iv)
+              *reinterpret_cast<uint4*>(p.dq + orow + 32 * cc + 8 * q4) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
           }
         }
       }
-      const float coef = dot * (1.0f / 128.0f) / (ss * (1.0f / 128.0f) + p.eps);
-      // pass 2: dq = scale (acc - coef q)
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t x[32];
-        tmem_ld32(tA + 32 * cc, x);
-        tmem_wait_ld();
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const uint4 v = qv[4 * cc + q4];
-          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-          uint32_t o4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float g0 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e]) - coef * bf16lo(w4[e]));
-            const float g1 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e + 1]) - coef * bf16hi(w4[e]));
-            o4[e] = pack_bf16(g0, g1);
-          }
-          if (iv) *reinterpret_cast<uint4*>(p.dq + orow + 32 * cc + 8 * q4) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-        }
-      }
+      if (!ok) break;
       tc_fence_before();
       mbar_arrive(bar_addr(sbase, ACCFREE + ab));
       ++uidx;
@@ -260,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 5) {
     tc_fence_after();
-    tmem_dealloc(tbase, 256);
+    tmem_dealloc(tbase, 512);
   }
 }
 
