@@ -107,12 +107,12 @@ def measured_peaks():
 # (profiles/attn_kernels_layer_s.md: S layer, B=8 T=2048 H=4), valid only while the
 # kernel's sources are byte-identical to the ones captured.
 CAPTURED_TRAFFIC = {
-    "bwd": {"bytes": 126138368,
-            "sources": {"bwd.cuh": "4acf64b6b2d65373d8428bcf9dd9f73a9073f2620868c7b26120fa4470f017a5",
-                        "sm100.cuh": "5f9e4443f303b7c498fe0eba328f4572a2f34cf75b3726dce0b45c2c691843c8"}},
-    "fwd": {"bytes": 53138176,
-            "sources": {"fwd.cuh": "231f252c63049c19c70cf9d7af681b31244b5da298e42a4cdbed1f9d365e3456",
-                        "sm100.cuh": "5f9e4443f303b7c498fe0eba328f4572a2f34cf75b3726dce0b45c2c691843c8"}},
+    "bwd": {"bytes": 174437632,
+            "sources": {"bwd.cuh": "b98fc7bf9948fa328b45ad2eb9ff9249068b628cec76aa3456dfb33f6549994e",
+                        "sm100.cuh": "e8840c99391be84966b29d31a4e191b1191a0954bc2c199f8e03b6be6a2367b7"}},
+    "fwd": {"bytes": 52859904,
+            "sources": {"fwd.cuh": "78368305976e50f22ee65fe41bb9d099b5cfa324272e07d1dc7d2690e458d1ab",
+                        "sm100.cuh": "e8840c99391be84966b29d31a4e191b1191a0954bc2c199f8e03b6be6a2367b7"}},
 }
 
 
