@@ -56,7 +56,8 @@ enum {
   AR_ERR_CUDA = -7,        /* a CUDA runtime call failed */
   AR_ERR_TIMEOUT = -8,     /* a device-side wait gave up (reported by sync_status) */
   AR_ERR_WORKSPACE = -9,   /* workspace given but smaller than required */
-  AR_ERR_TOO_LARGE = -10   /* problem exceeds ar_attn_fwd_noalloc's built-in scratch */
+  AR_ERR_TOO_LARGE = -10,  /* problem exceeds ar_attn_fwd_noalloc's built-in scratch */
+  AR_ERR_LAYOUT = -11      /* a kernel found its shared memory misaligned and did not run (sync_status) */
 };
 
 /* Bytes of scratch ar_attn_fwd needs: always 0.  The fused forward kernel

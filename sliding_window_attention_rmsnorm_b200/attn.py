@@ -20,6 +20,7 @@ STATUS = {
     0: "AR_OK", -1: "AR_ERR_NULL", -2: "AR_ERR_SHAPE", -3: "AR_ERR_UNSUPPORTED", -4: "AR_ERR_ALIGN",
     -5: "AR_ERR_ARG", -6: "AR_ERR_DEVICE", -7: "AR_ERR_CUDA", -8: "AR_ERR_TIMEOUT", -9: "AR_ERR_WORKSPACE",
     -10: "AR_ERR_TOO_LARGE",
+    -11: "AR_ERR_LAYOUT",
 }
 
 _lib = None

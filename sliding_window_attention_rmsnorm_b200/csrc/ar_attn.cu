@@ -35,7 +35,7 @@ std::mutex g_mu;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 // Checks the current device once: compute capability 10.0, kernel attributes.
-using FwdKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, ar::FwdParams);
+using FwdKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, ar::FwdParams);
 cudaError_t fwd_attr(FwdKernel f) {
   return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, ar::fwd::kSmemBytes);
 }
@@ -134,8 +134,10 @@ int make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
   return r == CUDA_SUCCESS ? AR_OK : AR_ERR_CUDA;
 }
 
-ar::FwdParams fwd_params(float* lse, const float* ck, int B, int T, int H, int window, float eps, float scale) {
+ar::FwdParams fwd_params(void* o, float* lse, const float* ck, int B, int T, int H, int window, float eps,
+                         float scale) {
   ar::FwdParams p;
+  p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.ck = ck;
   p.B = B;
@@ -155,17 +157,17 @@ ar::FwdParams fwd_params(float* lse, const float* ck, int B, int T, int H, int w
 // (see fwd.cuh), else the running-max forward; key factors computed in the
 // kernel, or (ck_global) read from p.ck.
 void launch_fwd(int grid, cudaStream_t s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                const CUtensorMap& to, const ar::FwdParams& p, bool ck_global) {
+                const ar::FwdParams& p, bool ck_global) {
   using namespace ar::fwd;
   const bool fixed = p.bound <= kFixedBoundMax;
   if (fixed && !ck_global)
-    fwd_kernel<true, false><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, to, p);
+    fwd_kernel<true, false><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
   else if (!fixed && !ck_global)
-    fwd_kernel<false, false><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, to, p);
+    fwd_kernel<false, false><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
   else if (fixed)
-    fwd_kernel<true, true><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, to, p);
+    fwd_kernel<true, true><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
   else
-    fwd_kernel<false, true><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, to, p);
+    fwd_kernel<false, true><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
 }
 
 size_t vec_bytes(int B, int T, int H) {
@@ -288,16 +290,15 @@ int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
   int sms = 0;
   if ((st = device_setup(&sms)) != AR_OK) return st;
 
-  CUtensorMap tq, tk, tv, to;
-  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, H) != AR_OK ||
-      make_map(&tv, v, B, T, H) != AR_OK || make_map(&to, o, B, T, H) != AR_OK)
+  CUtensorMap tq, tk, tv;
+  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, H) != AR_OK || make_map(&tv, v, B, T, H) != AR_OK)
     return AR_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const ar::FwdParams p = fwd_params(lse, nullptr, B, T, H, window, eps, scale);
+  const ar::FwdParams p = fwd_params(o, lse, nullptr, B, T, H, window, eps, scale);
   const int grid = p.n_units < sms ? p.n_units : sms;
   {
     KernelTimer t(AR_KERNEL_FWD, s);
-    launch_fwd(grid, s, tq, tk, tv, to, p, false);
+    launch_fwd(grid, s, tq, tk, tv, p, false);
     t.stop();
   }
   return cudaGetLastError() == cudaSuccess ? AR_OK : AR_ERR_CUDA;
@@ -419,7 +420,7 @@ int ar_attn_sync_status(void* stream) {
   if (flag != 0) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(ar::g_status, &zero, sizeof(int)) != cudaSuccess) return AR_ERR_CUDA;
-    return AR_ERR_TIMEOUT;
+    return (flag & ar::DEV_LAYOUT) ? AR_ERR_LAYOUT : AR_ERR_TIMEOUT;
   }
   return AR_OK;
 }
@@ -437,6 +438,7 @@ const char* ar_attn_strerror(int status) {
     case AR_ERR_TIMEOUT: return "a device-side wait timed out; results of the affected call are invalid";
     case AR_ERR_WORKSPACE: return "workspace smaller than the required size";
     case AR_ERR_TOO_LARGE: return "B * H * padded T exceeds the built-in scratch of ar_attn_fwd_noalloc";
+    case AR_ERR_LAYOUT: return "a kernel's shared memory was not 1024-byte aligned; it did not run";
     default: return "unknown status";
   }
 }
@@ -546,16 +548,15 @@ extern "C" int ar_attn_fwd_noalloc(const void* q, const void* k, const void* v, 
   float* ck = nullptr;
   if ((st = noalloc_scratch(&ck)) != AR_OK) return st;
 
-  CUtensorMap tq, tk, tv, to;
-  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, H) != AR_OK ||
-      make_map(&tv, v, B, T, H) != AR_OK || make_map(&to, o, B, T, H) != AR_OK)
+  CUtensorMap tq, tk, tv;
+  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, H) != AR_OK || make_map(&tv, v, B, T, H) != AR_OK)
     return AR_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long long rows = (long long)B * T * H;
   ar::fwd_prep_kernel<<<prep_grid(rows, sms), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(k), ck, B, T, H, T_pad,
                                                             eps, scale * 1.4426950408889634f);
-  const ar::FwdParams p = fwd_params(lse, ck, B, T, H, window, eps, scale);
+  const ar::FwdParams p = fwd_params(o, lse, ck, B, T, H, window, eps, scale);
   const int grid = p.n_units < sms ? p.n_units : sms;
-  launch_fwd(grid, s, tq, tk, tv, to, p, true);
+  launch_fwd(grid, s, tq, tk, tv, p, true);
   return cudaGetLastError() == cudaSuccess ? AR_OK : AR_ERR_CUDA;
 }

@@ -16,12 +16,12 @@
 // CTA organisation (persistent, one CTA per SM, 384 threads):
 //   warps 0-3  softmax warpgroup 0: query tile 0 (rows r0..r0+127), one row per thread
 //   warps 4-7  softmax warpgroup 1: query tile 1 (rows r0+128..r0+255)
-//   warp 8     TMA producer: Q tiles, K tiles (2 stages), V tiles (3 stages)
+//   warp 8     TMA producer: Q tiles, K tiles (3 stages), V tiles (2 stages)
 //   warp 9     MMA issuer: S_k = Q_k K^T into TMEM, O_k += P_k V with P_k read from TMEM
 //   warps 10-11 key factors: ck_j = rk_j * scale * log2(e) of each K tile, from the
-//              tile in shared memory, into a 3-slot ring read by the softmax
+//              tile in shared memory, into a 4-slot ring read by the softmax
 //              (kCkGlobal: read instead from a [B*H, T_pad] vector in global memory,
-//              loaded with the V tile; warps 10-11 then idle)
+//              loaded with the V tile into a slot per V stage; warps 10-11 then idle)
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P_k (bf16
 // pairs) overwrites the first 64 columns of S_k.  The MMA issue order
 // S0 S1 | PV0 S0' PV1 S1' | ... lets one warpgroup's softmax run while the
@@ -41,8 +41,10 @@
 // normalised by the sum of the bf16-rounded p that the P V product used (lse
 // still takes the unrounded sum); o is then a convex combination of v rows
 // with weights that sum to 1 up to fp32 rounding.
-// The epilogue stages the normalised O tile in the warpgroup's Q buffer and
-// writes it with one TMA store (rows past T are clipped by the tensor map).
+// The epilogue writes each thread's normalised O row straight from registers
+// to global memory, so a unit's Q buffers are free as soon as its last S
+// product has run: the next unit's Q tiles load under the last tile's softmax
+// and the epilogue.
 #pragma once
 #include <type_traits>
 
@@ -51,6 +53,7 @@
 namespace ar {
 
 struct FwdParams {
+  __nv_bfloat16* o;  // [B, T, H, 128]
   float* lse;        // [B, H, T]
   const float* ck;   // kCkGlobal only: [B*H, T_pad] rk_j * scale * log2(e), 0 on padding
   int B, T, H, T_pad;
@@ -69,10 +72,15 @@ constexpr int kThreads = 384;
 constexpr int kRegsLow = 104, kRegsHigh = 200, kLaunchRegs = 168;
 static_assert(256 * kRegsHigh + 128 * kRegsLow <= kLaunchRegs * kThreads, "register split exceeds the launch budget");
 constexpr uint32_t kTile = 32768, kHalf = 16384;
-// K tiles are double-buffered; V tiles (with their key factors ck) triple-buffered, because a V stage is
-// only released once both P V products of its tile are done and TMA loads take ~2 us under load.
-constexpr int kVStages = 3;
-constexpr uint32_t kQ = 0, kK = 2 * kTile, kV = 4 * kTile, kCK = 7 * kTile;
+// Stage counts: a K tile is needed first (S = Q K^T) and its loads, which take
+// ~5000 cycles under load, were what held the pipeline with two stages; V tiles
+// are needed one softmax later and two stages keep them ahead.
+constexpr int kKStages = 3, kVStages = 2;
+// Key-factor ring: the slot of tile n is free once tile n's K load has been
+// issued, because that load waited for the MMAs of tile n - kKStages, which were
+// issued after both softmax warpgroups finished tile n - kKStages - 1.
+constexpr int kCkSlots = kKStages + 1;
+constexpr uint32_t kQ = 0, kK = 2 * kTile, kV = kK + kKStages * kTile, kCK = kV + kVStages * kTile;
 // Of every 4 pairs of softmax exponentials, this many are computed on the FMA
 // pipe (exp2_fma2) and the rest on the MUFU unit.
 constexpr int kEmuPairsOf4 = 0;
@@ -80,16 +88,19 @@ constexpr int kEmuPairsOf4 = 0;
 // p >= 2^-64 stays a normal number in fp32 and bf16.
 constexpr float kFixedBoundMax = 32.0f;
 enum {
-  QFULL = 0, QEMPTY, KFULL, KEMPTY = KFULL + 2, VFULL = KEMPTY + 2, VEMPTY = VFULL + kVStages,
-  SFULL = VEMPTY + kVStages, PFULL = SFULL + 2, ODONE = PFULL + 2, OFREE = ODONE + 2, EPI = OFREE + 2,
-  CKFULL = EPI + 2, FINAL = CKFULL + kVStages, NBAR
+  QFULL = 0, QEMPTY, KFULL, KEMPTY = KFULL + kKStages, VFULL = KEMPTY + kKStages, VEMPTY = VFULL + kVStages,
+  SFULL = VEMPTY + kVStages, PFULL = SFULL + 2, ODONE = PFULL + 2, OFREE = ODONE + 2,
+  CKFULL = OFREE + 2, FINAL = CKFULL + kCkSlots, NBAR
 };
 constexpr int kCkThreads = 64;  // warps 10-11
-constexpr uint32_t kBar = kCK + kVStages * 512;
-static_assert(kBar + 256 + 1024 <= 232448, "shared memory budget");
+constexpr uint32_t kBar = kCK + kCkSlots * 512;
 constexpr uint32_t kTmemPtr = kBar + NBAR * 8;
 constexpr uint32_t kAbort = kTmemPtr + 4;
-constexpr uint32_t kSmemBytes = kAbort + 4 + 1024;  // + slack for 1024-byte alignment
+// No alignment slack: the dynamic shared memory of a kernel without static
+// shared memory starts 1024-byte aligned; the kernel checks and refuses to run
+// (DEV_LAYOUT) otherwise.
+constexpr uint32_t kSmemBytes = kAbort + 4;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Unit {
   int bh, b, h;
@@ -131,11 +142,14 @@ __device__ __forceinline__ uint32_t bar_addr(uint32_t sbase, int i) { return sba
 template <bool kFixed, bool kCkGlobal>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-               const FwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {  // uniform over the CTA: every thread returns before any barrier
+    if (threadIdx.x == 0) atomicOr(&g_status, DEV_LAYOUT);
+    return;
+  }
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kAbort);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int G = gridDim.x, cta = blockIdx.x;
@@ -143,10 +157,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBAR; ++i) {
       uint32_t cnt = 1;
-      if (i == PFULL || i == PFULL + 1 || i == OFREE || i == OFREE + 1 || i == EPI || i == EPI + 1) cnt = 128;
-      if (i == QEMPTY) cnt = 2;  // one arrival per softmax warpgroup and unit
-      if (!kCkGlobal && (i == KEMPTY || i == KEMPTY + 1)) cnt = 1 + kCkThreads;  // MMA commit + key-factor warps
-      if (i >= CKFULL && i < CKFULL + kVStages) cnt = kCkThreads;
+      if (i == PFULL || i == PFULL + 1 || i == OFREE || i == OFREE + 1) cnt = 128;
+      if (!kCkGlobal && i >= KEMPTY && i < KEMPTY + kKStages) cnt = 1 + kCkThreads;  // MMA commit + key-factor warps
+      if (i >= CKFULL && i < CKFULL + kCkSlots) cnt = kCkThreads;
       mbar_init(bar_addr(sbase, i), cnt);
     }
     *abort_flag = 0;
@@ -160,7 +173,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
-    prefetch_tmap(&tm_o);
   }
   tc_fence_before();
   __syncthreads();
@@ -174,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kv = 0;
       int uidx = 0;
       bool ok = true;
-      int last_k_par[2] = {-1, -1}, last_v_par[kVStages] = {-1, -1, -1}, last_q_par = -1;
+      int last_k_par[kKStages] = {-1, -1, -1}, last_v_par[kVStages] = {-1, -1}, last_q_par = -1;
       for (int r = 0; ok; ++r) {
         const int u = unit_index(cta, r, G);
         if (u >= p.n_units) break;
@@ -189,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         last_q_par = uidx & 1;
         for (int it = 0; it < U.N; ++it, ++kv) {
           const int n = U.hi_u - it;
-          const int st = kv & 1, ph = (kv >> 1) & 1;
+          const int st = kv % kKStages, ph = (kv / kKStages) & 1;
           if (!mbar_wait(bar_addr(sbase, KEMPTY + st), ph ^ 1, abort_flag)) { ok = false; break; }
           mbar_expect_tx(bar_addr(sbase, KFULL + st), kTile);
           for (int hf = 0; hf < 2; ++hf)
@@ -212,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*abort_flag) {
         // Let copies still in flight land before the CTA's shared memory goes away.
         volatile int never = 0;
-        for (int s = 0; s < 2; ++s)
+        for (int s = 0; s < kKStages; ++s)
           if (last_k_par[s] >= 0) mbar_wait(bar_addr(sbase, KFULL + s), last_k_par[s], &never);
         for (int s = 0; s < kVStages; ++s)
           if (last_v_par[s] >= 0) mbar_wait(bar_addr(sbase, VFULL + s), last_v_par[s], &never);
@@ -220,9 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (!kCkGlobal && warp >= 10) {
       // ---------------------------------------------------------- key factors
-      // Tile kv's factors go to ring slot kv % 3.  The slot is free: the K load
-      // of tile kv waited for the MMAs of tile kv - 2 (KEMPTY), which were issued
-      // after both softmax warpgroups finished tile kv - 3.
+      // Tile kv's factors go to ring slot kv % kCkSlots (free: see kCkSlots).
       const int tid = threadIdx.x - 320;
       uint32_t kv = 0;
       bool ok = true;
@@ -232,13 +242,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Unit U = decode(p, u);
         for (int it = 0; it < U.N; ++it, ++kv) {
           const int n = U.hi_u - it;
-          const int st = kv & 1, ph = (kv >> 1) & 1;
+          const int st = kv % kKStages, ph = (kv / kKStages) & 1;
           if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, KFULL + st), ph, abort_flag))) {
             ok = false;
             break;
           }
           const uint32_t kt = sbase + kK + st * kTile;
-          const uint32_t slot = sbase + kCK + (kv % kVStages) * 512;
+          const uint32_t slot = sbase + kCK + (kv % kCkSlots) * 512;
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
             const int row = tid + 64 * h2;
@@ -262,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             sts_f32(slot + 4 * row, ck);
           }
           mbar_arrive(bar_addr(sbase, KEMPTY + st));  // done reading the K tile
-          mbar_arrive(bar_addr(sbase, CKFULL + kv % kVStages));
+          mbar_arrive(bar_addr(sbase, CKFULL + kv % kCkSlots));
         }
       }
     } else if (warp == 9 && lane == 0) {
@@ -296,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Unit U = decode(p, u);
         if (!mbar_wait(bar_addr(sbase, QFULL), uidx & 1, abort_flag)) break;
         {
-          const int st = kv & 1, ph = (kv >> 1) & 1;
+          const int st = kv % kKStages, ph = (kv / kKStages) & 1;
           if (!mbar_wait(bar_addr(sbase, KFULL + st), ph, abort_flag)) break;
           tc_fence_after();
 #pragma unroll
@@ -306,12 +316,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_commit(bar_addr(sbase, SFULL + k));
             }
           mma_commit(bar_addr(sbase, KEMPTY + st));
+          // Q tiles are read only by the S products: after a unit's last one the
+          // producer may load the next unit's Q
+          if (U.N == 1) mma_commit(bar_addr(sbase, QEMPTY));
         }
         bool first_pv[2] = {true, true};
         for (int it = 0; it < U.N && ok; ++it) {
           const int n = U.hi_u - it;
           const uint32_t kvn = kv + it, kvx = kvn + 1;
-          const int vsn = kvn % kVStages, vphn = (kvn / kVStages) & 1, stx = kvx & 1, phx = (kvx >> 1) & 1;
+          const int vsn = kvn % kVStages, vphn = (kvn / kVStages) & 1;
+          const int stx = kvx % kKStages, phx = (kvx / kKStages) & 1;
           const bool has_next = it + 1 < U.N;
           if (!mbar_wait(bar_addr(sbase, VFULL + vsn), vphn, abort_flag)) { ok = false; break; }
           bool k_next_ready = false;
@@ -338,6 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (ok && has_next) mma_commit(bar_addr(sbase, KEMPTY + stx));
+          if (ok && it + 2 == U.N) mma_commit(bar_addr(sbase, QEMPTY));
         }
         if (!ok) break;
 #pragma unroll
@@ -377,7 +392,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int lok = k ? U.lo[1] : U.lo[0];
       const int hik = k ? U.hi[1] : U.hi[0];
       if (!validk) {
-        if (row == 0) mbar_arrive(bar_addr(sbase, QEMPTY));  // nothing of ours in the Q buffers
         kv += U.N;
         ++uidx;
         continue;
@@ -410,10 +424,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool first = true;
       for (int n = hik; n >= lok; --n) {
         const uint32_t kvn = kv + (U.hi_u - n);
-        const int vsn = kvn % kVStages, vphn = (kvn / kVStages) & 1;
         // key factors of this tile: in the ring (CKFULL) or loaded with V (VFULL).
         // They are normally ready before S, so this wait comes first and the one
         // on S is the last before the tile's work starts.
+        constexpr int kSlots = kCkGlobal ? kVStages : kCkSlots;
+        const int vsn = kvn % kSlots, vphn = (kvn / kSlots) & 1;
         if (!__all_sync(0xffffffffu,
                         mbar_wait(bar_addr(sbase, (kCkGlobal ? VFULL : CKFULL) + vsn), vphn, abort_flag))) {
           ok = false;
@@ -579,6 +594,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float l = l0 + l1;
       const float inv = 1.0f / (kFixed ? lr0 + lr1 : l);
+      const bool iv = i < p.T;
+      __nv_bfloat16* orow = p.o + (((size_t)U.b * p.T + (iv ? i : 0)) * p.H + U.h) * 128;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t ov[32];
@@ -591,33 +608,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           fmul2(a0, a1, __uint_as_float(ov[2 * e]), __uint_as_float(ov[2 * e + 1]), inv, inv);
           pk[e] = pack_bf16(a0, a1);
         }
-        // columns 32c..32c+31 = 16-byte chunks 4c..4c+3 of the row, in the Q buffer's layout
+        if (iv) {
+          uint4* d = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int chunk = 4 * c + e;
-          sts128(qa + (chunk >> 3) * kHalf + sw128(row, chunk & 7),
-                 make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]));
+          for (int e = 0; e < 4; ++e) d[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
       }
       tc_fence_before();
       mbar_arrive(bar_addr(sbase, OFREE + k));
-      fence_proxy_async_smem();
-      mbar_arrive(bar_addr(sbase, EPI + k));
-      if (i < p.T) p.lse[(size_t)U.bh * p.T + i] = ((kFixed ? p.bound : m) + log2f(l)) * kLn2;
-      if (row == 0) {
-        // one thread stores the tile once every row is staged, then frees the Q buffer
-        if (mbar_wait(bar_addr(sbase, EPI + k), (ecount - 1) & 1, abort_flag)) {
-          tma_store_4d(&tm_o, qa, 0, U.h, r0k, U.b);
-          tma_store_4d(&tm_o, qa + kHalf, 64, U.h, r0k, U.b);
-          bulk_commit();
-          bulk_wait_read();
-        }
-        mbar_arrive(bar_addr(sbase, QEMPTY));
-      }
+      if (iv) p.lse[(size_t)U.bh * p.T + i] = ((kFixed ? p.bound : m) + log2f(l)) * kLn2;
       kv += U.N;
       ++uidx;
     }
-    if (row == 0) bulk_wait_all();  // the last output tile has reached global memory
   }
   tc_fence_before();
   __syncthreads();

@@ -12,7 +12,7 @@ namespace ar {
 // ------------------------------------------------------------------ status
 // Device-side status word: kernels OR error bits into it, the host reads and
 // clears it in ar_attn_sync_status().
-enum : int { DEV_TIMEOUT = 1 };
+enum : int { DEV_TIMEOUT = 1, DEV_LAYOUT = 2 };
 __device__ int g_status = 0;
 
 // A wait gives up after this many nanoseconds of %globaltimer.
