@@ -73,13 +73,17 @@ constexpr uint32_t kTile = 32768, kHalf = 16384;
 constexpr uint32_t kK = 0, kV = kTile, kQ = 2 * kTile, kDO = 4 * kTile, kG = 6 * kTile, kVec = 7 * kTile;
 enum {
   KVFULL = 0, KVEMPTY, QFULL, QEMPTY = QFULL + 2, SFULL = QEMPTY + 2, DSREADY = SFULL + 2, DSFREE = DSREADY + 2,
-  VECFULL = DSFREE + 2, VECEMPTY = VECFULL + 2, DKDVDONE = VECEMPTY + 2, ACCFREE, FINAL, NBAR
+  VECFULL = DSFREE + 2, VECEMPTY = VECFULL + 2, DKDVDONE = VECEMPTY + 2, ACCFREE, DOTFREE, FINAL, NBAR
 };
 constexpr uint32_t kVecHalf = 3 * 64 * 4;  // lse2, delta, rq for 64 queries
-constexpr uint32_t kBar = kVec + 2 * kVecHalf;
+// per key row and query half: rk^2 / D * sum_i G_ij S_ij (the dk norm-backward coefficient)
+constexpr uint32_t kDot = kVec + 2 * kVecHalf;
+constexpr uint32_t kBar = kDot + 2 * 128 * 4;
 constexpr uint32_t kTmemPtr = kBar + NBAR * 8;
 constexpr uint32_t kAbort = kTmemPtr + 4;
-constexpr uint32_t kSmemBytes = kAbort + 4 + 1024;
+// No alignment slack: dynamic shared memory of a kernel without static shared
+// memory starts 1024-byte aligned; the kernel checks (DEV_LAYOUT) otherwise.
+constexpr uint32_t kSmemBytes = kAbort + 4;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Unit {
@@ -108,14 +112,16 @@ __device__ __forceinline__ Unit decode(const BwdParams& p, int u) {
 __device__ __forceinline__ uint32_t bar_addr(uint32_t sbase, int i) { return sbase + kBar + 8u * i; }
 
 // One 32-query chunk of a key row: P = 2^(S rq_i C_j - lse2_i) (zero outside the
-// band when MASKED), G = P (dP - delta_i) rq_i rk_j, both packed to bf16 pairs.
+// band when MASKED), G = P (dP - delta_i) rq_i rk_j, both packed to bf16 pairs,
+// and (dt0, dt1) += sum G S over the chunk (S: the raw logit q_i . k_j), so that
+// k_j . dK_acc_j = sum_i G_ij q_i . k_j is known without reading k again.
 // Two queries at a time in packed fp32x2 arithmetic.
 // vaddr: shared-memory address of this chunk's -lse2 entries; delta follows at
 // +256 bytes and rq at +512 bytes.
 template <bool MASKED>
 __device__ __forceinline__ void grad_chunk(const uint32_t (&sv)[32], const uint32_t (&dp)[32], uint32_t vaddr,
                                            float Cj, float rk, int c_lo, int c_hi, int cbase, uint32_t (&pk)[16],
-                                           uint32_t (&gk)[16]) {
+                                           uint32_t (&gk)[16], float& dt0, float& dt1) {
 #pragma unroll
   for (int e4 = 0; e4 < 8; ++e4) {
     const float4 L = lds_f4(vaddr + 16 * e4);  // -lse2
@@ -137,6 +143,7 @@ __device__ __forceinline__ void grad_chunk(const uint32_t (&sv)[32], const uint3
       fmul2(rr0, rr1, rv[2 * h], rv[2 * h + 1], rk, rk);  // rq_i rk_j
       fmul2(x0, x1, x0, x1, p0, p1);
       fmul2(x0, x1, x0, x1, rr0, rr1);
+      ffma2(dt0, dt1, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]), x0, x1, dt0, dt1);
       pk[e4 * 2 + h] = pack_bf16(p0, p1);
       gk[e4 * 2 + h] = pack_bf16(x0, x1);
     }
@@ -147,9 +154,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                const __grid_constant__ CUtensorMap tm_g, const BwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {  // uniform over the CTA: every thread returns before any barrier
+    if (threadIdx.x == 0) atomicOr(&g_status, DEV_LAYOUT);
+    return;
+  }
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kAbort);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int G = gridDim.x, cta = blockIdx.x;
@@ -158,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < NBAR; ++i) {
       uint32_t cnt = 1;
       if (i == DSREADY || i == DSREADY + 1 || i == VECFULL || i == VECFULL + 1 || i == VECEMPTY ||
-          i == VECEMPTY + 1 || i == ACCFREE)
+          i == VECEMPTY + 1 || i == ACCFREE || i == DOTFREE)
         cnt = 128;
       if (i == DSFREE || i == DSFREE + 1) cnt = 2;  // the MMA commit + the G^T store's read
       if (i == KVEMPTY) cnt = 1 + 256;  // the MMA commit + every compute thread once rk is read
@@ -380,6 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar_addr(sbase, KVEMPTY));  // done reading K from shared memory
         const float Cj = rk * p.scale * kLog2e;
         const size_t vbase = (size_t)U.bh * p.T_pad;
+        float dt0 = 0.f, dt1 = 0.f;
         for (int it = 0; it < U.N; ++it, ++qc) {
           const int qt = U.qlo + it;
           const int i0 = qt * 128 + 64 * a;  // first query of this half
@@ -425,15 +437,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
             uint32_t pk[16], gk[16];
             if (masked)
-              grad_chunk<true>(sv, dp, vaddr + 128 * c, Cj, rk, c_lo, c_hi, 32 * c, pk, gk);
+              grad_chunk<true>(sv, dp, vaddr + 128 * c, Cj, rk, c_lo, c_hi, 32 * c, pk, gk, dt0, dt1);
             else
-              grad_chunk<false>(sv, dp, vaddr + 128 * c, Cj, rk, c_lo, c_hi, 32 * c, pk, gk);
+              grad_chunk<false>(sv, dp, vaddr + 128 * c, Cj, rk, c_lo, c_hi, 32 * c, pk, gk, dt0, dt1);
             tmem_st16(tS + 16 * c, pk);
             // G^T row j, queries 32c..32c+31 of this half: 16-byte chunks 4c..4c+3
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4)
               sts128(ga + sw128(row, 4 * c + q4),
                      make_uint4(gk[4 * q4], gk[4 * q4 + 1], gk[4 * q4 + 2], gk[4 * q4 + 3]));
+          }
+          if (it + 1 == U.N) {
+            // this half's share of the dk coefficient, published before the last
+            // DSREADY (so the epilogue's wait for the final products covers it) and
+            // once the epilogue has taken the previous unit's (DOTFREE)
+            if (uidx > 0 &&
+                !__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DOTFREE), (uidx - 1) & 1, abort_flag))) {
+              ok = false;
+              break;
+            }
+            sts_f32(sbase + kDot + 4 * (128 * a + row), (dt0 + dt1) * rk * rk * (1.0f / 128.0f));
           }
           tmem_wait_st();
           fence_proxy_async_smem();
@@ -458,9 +481,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int j = U.kt * 128 + row;
         const size_t orow = (((size_t)U.b * p.T + (j < p.T ? j : 0)) * p.H + U.h) * 128;
         const bool jv = j < p.T;
-        // dk = scale (acc - rk^2 k (acc . k) / D), with k and rk from the raw key
-        // row, pulled towards L2 before the wait so that its latency overlaps the
-        // unit's last products
+        // dk = scale (acc - coef k), coef = rk^2 (acc . k) / D, with acc . k summed by
+        // the compute warpgroups as sum_i G_ij S_ij; the raw key row is pulled
+        // towards L2 before the wait so that its latency overlaps the last products
         {
           const uint4* krow = reinterpret_cast<const uint4*>(p.k + orow);
           if (jv) {
@@ -469,25 +492,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DKDVDONE), uidx & 1, abort_flag))) break;
           tc_fence_after();
-          float ss = 0.f, dot = 0.f;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t x[32];
-            tmem_ld32(tDK + 32 * c, x);
-            tmem_wait_ld();
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const uint4 v = jv ? __ldg(krow + 4 * c + q4) : make_uint4(0, 0, 0, 0);
-              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float k0 = bf16lo(w4[e]), k1 = bf16hi(w4[e]);
-                ss = fmaf(k0, k0, fmaf(k1, k1, ss));
-                dot = fmaf(__uint_as_float(x[8 * q4 + 2 * e]), k0, fmaf(__uint_as_float(x[8 * q4 + 2 * e + 1]), k1, dot));
-              }
-            }
-          }
-          const float coef = dot * (1.0f / 128.0f) / (ss * (1.0f / 128.0f) + p.eps);
+          const float coef = lds_f32(sbase + kDot + 4 * row) + lds_f32(sbase + kDot + 4 * (128 + row));
+          mbar_arrive(bar_addr(sbase, DOTFREE));
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t x[32];
