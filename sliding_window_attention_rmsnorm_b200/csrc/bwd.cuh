@@ -482,13 +482,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const size_t orow = (((size_t)U.b * p.T + (j < p.T ? j : 0)) * p.H + U.h) * 128;
         const bool jv = j < p.T;
         // dk = scale (acc - coef k), coef = rk^2 (acc . k) / D, with acc . k summed by
-        // the compute warpgroups as sum_i G_ij S_ij; the raw key row is pulled
-        // towards L2 before the wait so that its latency overlaps the last products
+        // the compute warpgroups as sum_i G_ij S_ij; the raw key row is loaded into
+        // registers before the wait, so its latency is hidden by the unit's products
         {
-          const uint4* krow = reinterpret_cast<const uint4*>(p.k + orow);
-          if (jv) {
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(krow));
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(krow + 8));
+          uint4 kv[16];
+          {
+            const uint4* krow = reinterpret_cast<const uint4*>(p.k + orow);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) kv[c] = jv ? __ldg(krow + c) : make_uint4(0, 0, 0, 0);
           }
           if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DKDVDONE), uidx & 1, abort_flag))) break;
           tc_fence_after();
@@ -501,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
-              const uint4 v = jv ? __ldg(krow + 4 * c + q4) : make_uint4(0, 0, 0, 0);
+              const uint4 v = kv[4 * c + q4];
               const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
               uint32_t o4[4];
 #pragma unroll
