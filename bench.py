@@ -107,12 +107,12 @@ def measured_peaks():
 # (profiles/attn_kernels_layer_s.md: S layer, B=8 T=2048 H=4), valid only while the
 # kernel's sources are byte-identical to the ones captured.
 CAPTURED_TRAFFIC = {
-    "bwd": {"bytes": 174437632,
-            "sources": {"bwd.cuh": "b98fc7bf9948fa328b45ad2eb9ff9249068b628cec76aa3456dfb33f6549994e",
-                        "sm100.cuh": "e8840c99391be84966b29d31a4e191b1191a0954bc2c199f8e03b6be6a2367b7"}},
-    "fwd": {"bytes": 52859904,
-            "sources": {"fwd.cuh": "78368305976e50f22ee65fe41bb9d099b5cfa324272e07d1dc7d2690e458d1ab",
-                        "sm100.cuh": "e8840c99391be84966b29d31a4e191b1191a0954bc2c199f8e03b6be6a2367b7"}},
+    "bwd": {"bytes": 164617984,
+            "sources": {"bwd.cuh": "80dbd11ac28e914c51d4ca0bd16e050baa3010c5dbe74cc803a65c8697b72375",
+                        "sm100.cuh": "2a6361b7a1592904700533a665955b9d2dc9fd96ab09bba3932c100f6798b5f7"}},
+    "fwd": {"bytes": 51727616,
+            "sources": {"fwd.cuh": "67fc8e52d48d48e820a1f31b8ab211c18e5217889256fc8d6106b7bc6aee1610",
+                        "sm100.cuh": "2a6361b7a1592904700533a665955b9d2dc9fd96ab09bba3932c100f6798b5f7"}},
 }
 
 
