@@ -122,7 +122,7 @@ enum {
 };
 
 /* on != 0: clear the record and, until called with on == 0, bracket every
- * kernel that ar_attn_fwd / ar_attn_bwd launch with CUDA events on the call's
+ * kernel that ar_attn_fwd, ar_attn_fwd_noalloc and ar_attn_bwd launch with CUDA events on the call's
  * stream (a few microseconds of host time per kernel).  on == 0 stops
  * recording and keeps what was recorded for ar_attn_timing_read.  Returns AR_OK. */
 int ar_attn_timing_enable(int on);

@@ -9,7 +9,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libar_attn.so")
 SOURCES = ["ar_attn.cu"]
-DEPS = ["ar_attn.cu", "sm100.cuh", "fwd.cuh", "bwd.cuh", "aux.cuh"]
+DEPS = ["ar_attn.cu", "sm100.cuh", "fwd.cuh", "bwd.cuh", "dq.cuh", "aux.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

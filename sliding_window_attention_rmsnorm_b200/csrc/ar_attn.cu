@@ -553,10 +553,18 @@ extern "C" int ar_attn_fwd_noalloc(const void* q, const void* k, const void* v, 
     return AR_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long long rows = (long long)B * T * H;
-  ar::fwd_prep_kernel<<<prep_grid(rows, sms), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(k), ck, B, T, H, T_pad,
-                                                            eps, scale * 1.4426950408889634f);
+  {
+    KernelTimer t(AR_KERNEL_FWD_PREP, s);
+    ar::fwd_prep_kernel<<<prep_grid(rows, sms), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(k), ck, B, T, H,
+                                                              T_pad, eps, scale * 1.4426950408889634f);
+    t.stop();
+  }
   const ar::FwdParams p = fwd_params(o, lse, ck, B, T, H, window, eps, scale);
   const int grid = p.n_units < sms ? p.n_units : sms;
-  launch_fwd(grid, s, tq, tk, tv, p, true);
+  {
+    KernelTimer t(AR_KERNEL_FWD, s);
+    launch_fwd(grid, s, tq, tk, tv, p, true);
+    t.stop();
+  }
   return cudaGetLastError() == cudaSuccess ? AR_OK : AR_ERR_CUDA;
 }

@@ -13,15 +13,18 @@
 // memory and rk_j from a per-key pre-pass (`ck`).  q and k are never rounded
 // after normalisation.
 //
-// CTA organisation (persistent, one CTA per SM, 384 threads):
+// CTA organisation (persistent, one CTA per SM, 512 threads):
 //   warps 0-3  softmax warpgroup 0: query tile 0 (rows r0..r0+127), one row per thread
 //   warps 4-7  softmax warpgroup 1: query tile 1 (rows r0+128..r0+255)
 //   warp 8     TMA producer: Q tiles, K tiles (3 stages), V tiles (2 stages)
 //   warp 9     MMA issuer: S_k = Q_k K^T into TMEM, O_k += P_k V with P_k read from TMEM
-//   warps 10-11 key factors: ck_j = rk_j * scale * log2(e) of each K tile, from the
-//              tile in shared memory, into a 4-slot ring read by the softmax
+//   warps 10-11 idle
+//   warps 12-15 key factors: ck_j = rk_j * scale * log2(e) of each K tile, one key
+//              row per thread, from the tile in shared memory into a 4-slot ring
+//              read by the softmax.  One warp sits on each SM sub-partition, so
+//              this work takes issue slots evenly from the softmax warps beside it
 //              (kCkGlobal: read instead from a [B*H, T_pad] vector in global memory,
-//              loaded with the V tile into a slot per V stage; warps 10-11 then idle)
+//              loaded with the V tile into a slot per V stage; warps 12-15 then idle)
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P_k (bf16
 // pairs) overwrites the first 64 columns of S_k.  The MMA issue order
 // S0 S1 | PV0 S0' PV1 S1' | ... lets one warpgroup's softmax run while the
@@ -66,11 +69,14 @@ struct FwdParams {
 };
 
 namespace fwd {
-constexpr int kThreads = 384;
-// Launch budget 168 registers x 384 threads; warpgroup 2 (TMA, MMA, 2 idle
-// warps) drops to 104 so warpgroups 0-1 can rise to 200: 256*200 + 128*104 = 168*384.
-constexpr int kRegsLow = 104, kRegsHigh = 200, kLaunchRegs = 168;
-static_assert(256 * kRegsHigh + 128 * kRegsLow <= kLaunchRegs * kThreads, "register split exceeds the launch budget");
+constexpr int kThreads = 512;
+// Launch budget 128 registers x 512 threads; warpgroup 2 (TMA, MMA, 2 idle
+// warps) drops to 104 and warpgroup 3 (key factors) to 40 so warpgroups 0-1 can
+// rise to 184: 256*184 + 128*104 + 128*40 = 128*512.  (The running-max softmax
+// spills a few registers at 184; the fixed-offset one does not.)
+constexpr int kRegsLow = 104, kRegsCk = 40, kRegsHigh = 184, kLaunchRegs = 128;
+static_assert(256 * kRegsHigh + 128 * kRegsLow + 128 * kRegsCk <= kLaunchRegs * kThreads,
+              "register split exceeds the launch budget");
 constexpr uint32_t kTile = 32768, kHalf = 16384;
 // Stage counts: a K tile is needed first (S = Q K^T) and its loads, which take
 // ~5000 cycles under load, were what held the pipeline with two stages; V tiles
@@ -92,7 +98,7 @@ enum {
   SFULL = VEMPTY + kVStages, PFULL = SFULL + 2, ODONE = PFULL + 2, OFREE = ODONE + 2,
   CKFULL = OFREE + 2, FINAL = CKFULL + kCkSlots, NBAR
 };
-constexpr int kCkThreads = 64;  // warps 10-11
+constexpr int kCkThreads = 128;  // warps 12-15
 constexpr uint32_t kBar = kCK + kCkSlots * 512;
 constexpr uint32_t kTmemPtr = kBar + NBAR * 8;
 constexpr uint32_t kAbort = kTmemPtr + 4;
@@ -179,7 +185,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + kTmemPtr);
 
-  if (warp >= 8) {
+  if (warp >= 12) {
+    regs_dec<kRegsCk>();
+    if (!kCkGlobal) {
+      // ---------------------------------------------------------- key factors
+      // Tile kv's factors go to ring slot kv % kCkSlots (free: see kCkSlots).
+      const int row = threadIdx.x - 384;  // key row within the tile
+      uint32_t kv = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int u = unit_index(cta, r, G);
+        if (u >= p.n_units) break;
+        const Unit U = decode(p, u);
+        for (int it = 0; it < U.N; ++it, ++kv) {
+          const int n = U.hi_u - it;
+          const int st = kv % kKStages, ph = (kv / kKStages) & 1;
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, KFULL + st), ph, abort_flag))) {
+            ok = false;
+            break;
+          }
+          const uint32_t kt = sbase + kK + st * kTile;
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < 16; ++c) {  // 16-byte chunk c of the row
+            const uint4 x = lds128(kt + (c >> 3) * kHalf + sw128(row, c & 7));
+            const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float a = bf16lo(w4[e]), b = bf16hi(w4[e]);
+              ffma2(s0, s1, a, b, a, b, s0, s1);
+            }
+          }
+          const float ck = (n * 128 + row < p.T) ? rsqrtf((s0 + s1) * (1.0f / 128.0f) + p.eps) * p.cscale : 0.f;
+          sts_f32(sbase + kCK + (kv % kCkSlots) * 512 + 4 * row, ck);
+          mbar_arrive(bar_addr(sbase, KEMPTY + st));  // done reading the K tile
+          mbar_arrive(bar_addr(sbase, CKFULL + kv % kCkSlots));
+        }
+      }
+    }
+  } else if (warp >= 8) {
     regs_dec<kRegsLow>();
     if (warp == 8 && lane == 0) {
       // ---------------------------------------------------------- TMA producer
@@ -229,51 +273,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kVStages; ++s)
           if (last_v_par[s] >= 0) mbar_wait(bar_addr(sbase, VFULL + s), last_v_par[s], &never);
         if (last_q_par >= 0) mbar_wait(bar_addr(sbase, QFULL), last_q_par, &never);
-      }
-    } else if (!kCkGlobal && warp >= 10) {
-      // ---------------------------------------------------------- key factors
-      // Tile kv's factors go to ring slot kv % kCkSlots (free: see kCkSlots).
-      const int tid = threadIdx.x - 320;
-      uint32_t kv = 0;
-      bool ok = true;
-      for (int r = 0; ok; ++r) {
-        const int u = unit_index(cta, r, G);
-        if (u >= p.n_units) break;
-        const Unit U = decode(p, u);
-        for (int it = 0; it < U.N; ++it, ++kv) {
-          const int n = U.hi_u - it;
-          const int st = kv % kKStages, ph = (kv / kKStages) & 1;
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, KFULL + st), ph, abort_flag))) {
-            ok = false;
-            break;
-          }
-          const uint32_t kt = sbase + kK + st * kTile;
-          const uint32_t slot = sbase + kCK + (kv % kCkSlots) * 512;
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int row = tid + 64 * h2;
-            float ss[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                const uint4 v = lds128(kt + hf * kHalf + sw128(row, c));
-                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float a = bf16lo(w4[e]), b2 = bf16hi(w4[e]);
-                  ss[e] = fmaf(a, a, ss[e]);
-                  ss[e] = fmaf(b2, b2, ss[e]);
-                }
-              }
-            const float ck = (n * 128 + row < p.T)
-                                 ? rsqrtf((ss[0] + ss[1] + ss[2] + ss[3]) * (1.0f / 128.0f) + p.eps) * p.cscale
-                                 : 0.f;
-            sts_f32(slot + 4 * row, ck);
-          }
-          mbar_arrive(bar_addr(sbase, KEMPTY + st));  // done reading the K tile
-          mbar_arrive(bar_addr(sbase, CKFULL + kv % kCkSlots));
-        }
       }
     } else if (warp == 9 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
