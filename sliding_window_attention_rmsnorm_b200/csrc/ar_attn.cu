@@ -395,7 +395,7 @@ int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, cons
     d.H = H;
     d.w = w;
     d.nq = nk;
-    d.n_units = n_bh * ((nk + 1) / 2);  // units of two query tiles
+    d.n_units = n_bh * nk;  // units of one query tile
     d.bh0 = bh0;
     d.n_bh = n_bh;
     d.nb = nb;

@@ -6,25 +6,26 @@
 // the attention product as in the "autoresearch" README (gitee), section 7.3).
 //
 // The backward main kernel stores, for every (query tile, key tile) pair of the
-// band, the bf16 tile G^T with G_ij = dS_ij rq_i rk_j.  Here one CTA owns two
-// consecutive 128-query tiles at a time (a unit) and accumulates, in TMEM,
+// band, the bf16 tile G^T with G_ij = dS_ij rq_i rk_j.  Here one CTA owns one
+// 128-query tile at a time (a unit) and accumulates, in TMEM,
 //   acc_i = sum_j G_ij k_j = rq_i dqhat_i / scale      (raw bf16 k rows)
-// over each tile's band, then finishes dq_i = scale (acc_i - c_i q_i) with
-// c_i = (acc_i . q_i) / D / (mean q_i^2 + eps) and writes it as bf16.  The two
-// tiles' bands overlap in all but one key tile, so each K tile is loaded once
-// for both: the kernel streams 32 KB per G tile plus 32 KB per K tile, which
-// is what bounds it (the SM's TMA ingest, about 64 bytes per clock).
+// over the tile's band, then finishes dq_i = scale (acc_i - c_i q_i) with
+// c_i = (acc_i . q_i) / D / (mean q_i^2 + eps) and writes it as bf16.  Per key
+// tile of the band the kernel streams a 32 KB G tile (from DRAM) and the 32 KB
+// K tile (mostly from L2).  Units of one query tile, rather than two that share
+// their K tiles, split the work into finer pieces, so the persistent CTAs end
+// closer together on banded layers.
 //
 // CTA organisation (persistent, one CTA per SM, 224 threads):
-//   warps 0-3  epilogue warpgroup: one query row per thread, tile 0 then tile 1
+//   warps 0-3  epilogue warpgroup: one query row per thread
 //   warp 4     TMA producer of the G tiles (two 64-query halves each; 4 stages)
 //   warp 5     MMA issuer
 //   warp 6     TMA producer of the K tiles (3 stages)
-// TMEM (512 columns): accumulators for the unit's two tiles, double-buffered
-// (column 256 * buffer + 128 * tile), so one unit's epilogue overlaps the next
-// unit's products.  The product is acc (M = 128 queries, N = 128 features,
-// K = 16 keys per step) with A = G read from the G^T tile (queries contiguous:
-// MN-major) and B = the K tile (features contiguous: MN-major).
+// TMEM (512 columns): four 128-column accumulators, one per unit in flight, so
+// the epilogues of short units overlap the next units' products.  The product
+// is acc (M = 128 queries, N = 128 features, K = 16 keys per step) with A = G
+// read from the G^T tile (queries contiguous: MN-major) and B = the K tile
+// (features contiguous: MN-major).
 #pragma once
 #include "sm100.cuh"
 
@@ -36,7 +37,7 @@ struct DqParams {
   int B, T, H;
   int w;           // left window (w >= T means full causal)
   int nq;          // query tiles per head
-  int n_units;     // n_bh * ceil(nq / 2)
+  int n_units;     // n_bh * nq
   int bh0, n_bh;   // heads processed by this launch (as in the backward kernel)
   int nb;          // key tiles in one query tile's band (as in the backward kernel)
   int pairs_head;  // G tiles per head
@@ -47,10 +48,11 @@ namespace dqk {
 constexpr int kThreads = 224;
 constexpr uint32_t kTile = 32768, kHalf = 16384;
 constexpr int kGStages = 4, kKStages = 3;
+constexpr int kAcc = 4;  // TMEM accumulators (128 columns each)
 constexpr uint32_t kG = 0, kK = kGStages * kTile;
 enum {
   GFULL = 0, GEMPTY = GFULL + kGStages, KFULL = GEMPTY + kGStages, KEMPTY = KFULL + kKStages,
-  ACCFULL = KEMPTY + kKStages, ACCFREE = ACCFULL + 2, FINAL = ACCFREE + 2, NBAR
+  ACCFULL = KEMPTY + kKStages, ACCFREE = ACCFULL + kAcc, FINAL = ACCFREE + kAcc, NBAR
 };
 constexpr uint32_t kBar = kK + kKStages * kTile;
 constexpr uint32_t kTmemPtr = kBar + NBAR * 8;
@@ -58,36 +60,25 @@ constexpr uint32_t kAbort = kTmemPtr + 4;
 constexpr uint32_t kSmemBytes = kAbort + 4 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-// A unit: query tiles q0 = 2 qp and q1 = q0 + 1 (q1 only if has1) of one head;
-// key tiles kt = khi down to klo, where tile t uses kt in [lo[t], hi[t]].
+// A unit: query tile qt of one head, with key tiles kt = hi (= qt) down to lo.
 struct Unit {
-  int hl, bh, b, h, q0, has1, khi, klo, lo[2], hi[2];
-  __device__ bool in(int t, int kt) const { return (t == 0 || has1) && kt >= lo[t] && kt <= hi[t]; }
+  int hl, bh, b, h, qt, lo, hi;
 };
 
 __device__ __forceinline__ int unit_index(int cta, int round, int G) {
   return round * G + ((round & 1) ? (G - 1 - cta) : cta);
 }
 
-// Units are (head, pair of query tiles), later pairs (longer bands) first.
+// Units are (head, query tile), later tiles (longer bands) first.
 __device__ __forceinline__ Unit decode(const DqParams& p, int u) {
   Unit U;
-  const int npairs = (p.nq + 1) / 2;
-  const int qp = npairs - 1 - u / p.n_bh;
   U.hl = u % p.n_bh;
   U.bh = p.bh0 + U.hl;
   U.b = U.bh / p.H;
   U.h = U.bh % p.H;
-  U.q0 = 2 * qp;
-  U.has1 = U.q0 + 1 < p.nq;
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int qt = U.q0 + t;
-    U.lo[t] = max(0, qt * 128 - p.w) / 128;
-    U.hi[t] = qt;
-  }
-  U.klo = U.lo[0];
-  U.khi = U.has1 ? U.hi[1] : U.hi[0];
+  U.qt = p.nq - 1 - u / p.n_bh;
+  U.lo = max(0, U.qt * 128 - p.w) / 128;
+  U.hi = U.qt;
   return U;
 }
 
@@ -110,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int G = gridDim.x, cta = blockIdx.x;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NBAR; ++i) mbar_init(bar_addr(sbase, i), (i == ACCFREE || i == ACCFREE + 1) ? 128 : 1);
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar_addr(sbase, i), (i >= ACCFREE && i < ACCFREE + kAcc) ? 128 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -130,8 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 4 || warp == 6) {
     if (lane == 0) {
       // ---------------------------------------------------------- TMA producers: G (warp 4), K (warp 6)
-      // Both walk the unit's key tiles newest first; the G producer loads, per key
-      // tile, the G tile of each query tile whose band holds it (tile 0 first).
+      // Both walk the unit's key tiles newest first.
       const bool is_g = warp == 4;
       const int nst = is_g ? kGStages : kKStages;
       const int full = is_g ? GFULL : KFULL, empty = is_g ? GEMPTY : KEMPTY;
@@ -142,28 +132,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = unit_index(cta, r, G);
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
-        for (int kt = U.khi; kt >= U.klo && ok; --kt) {
-          for (int t = 0; t < (is_g ? 2 : 1); ++t) {
-            if (is_g && !U.in(t, kt)) continue;
-            const int s = c % nst, ph = (c / nst) & 1;
-            if (!mbar_wait(bar_addr(sbase, empty + s), ph ^ 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            mbar_expect_tx(bar_addr(sbase, full + s), kTile);
-            if (is_g) {
-              const long long slot = g_slot(p, U.hl, U.q0 + t, kt);
-              for (int hf = 0; hf < 2; ++hf)
-                tma_load_2d(sbase + kG + s * kTile + hf * kHalf, &tm_g, bar_addr(sbase, full + s), 0,
-                            (int)((2 * slot + hf) * 128));
-            } else {
-              for (int hf = 0; hf < 2; ++hf)
-                tma_load_4d(sbase + kK + s * kTile + hf * kHalf, &tm_k, bar_addr(sbase, full + s), hf * 64, U.h,
-                            kt * 128, U.b);
-            }
-            last_par[s] = ph;
-            ++c;
+        for (int kt = U.hi; kt >= U.lo; --kt, ++c) {
+          const int s = c % nst, ph = (c / nst) & 1;
+          if (!mbar_wait(bar_addr(sbase, empty + s), ph ^ 1, abort_flag)) {
+            ok = false;
+            break;
           }
+          mbar_expect_tx(bar_addr(sbase, full + s), kTile);
+          if (is_g) {
+            const long long slot = g_slot(p, U.hl, U.qt, kt);
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_2d(sbase + kG + s * kTile + hf * kHalf, &tm_g, bar_addr(sbase, full + s), 0,
+                          (int)((2 * slot + hf) * 128));
+          } else {
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_4d(sbase + kK + s * kTile + hf * kHalf, &tm_k, bar_addr(sbase, full + s), hf * 64, U.h,
+                          kt * 128, U.b);
+          }
+          last_par[s] = ph;
         }
       }
       if (*abort_flag) {
@@ -184,30 +170,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = unit_index(cta, r, G);
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
-        const int ab = uidx & 1;
-        if (uidx >= 2 && !mbar_wait(bar_addr(sbase, ACCFREE + ab), ((uidx >> 1) - 1) & 1, abort_flag)) break;
-        for (int kt = U.khi; kt >= U.klo && ok; --kt, ++ck) {
+        const int ab = uidx % kAcc;
+        if (uidx >= kAcc && !mbar_wait(bar_addr(sbase, ACCFREE + ab), (uidx / kAcc - 1) & 1, abort_flag)) break;
+        for (int kt = U.hi; kt >= U.lo; --kt, ++ck, ++cg) {
           const int ks = ck % kKStages, kph = (ck / kKStages) & 1;
-          if (!mbar_wait(bar_addr(sbase, KFULL + ks), kph, abort_flag)) {
+          const int gs = cg % kGStages, gph = (cg / kGStages) & 1;
+          if (!mbar_wait(bar_addr(sbase, KFULL + ks), kph, abort_flag) ||
+              !mbar_wait(bar_addr(sbase, GFULL + gs), gph, abort_flag)) {
             ok = false;
             break;
           }
-          for (int t = 0; t < 2; ++t) {
-            if (!U.in(t, kt)) continue;
-            const int gs = cg % kGStages, gph = (cg / kGStages) & 1;
-            if (!mbar_wait(bar_addr(sbase, GFULL + gs), gph, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const bool first = kt == U.hi[t];
+          tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tbase + 256 * ab + 128 * t, sdesc_add(dA, gs * kTile + kk * 2048),
-                     sdesc_add(dB, ks * kTile + kk * 2048), id, (!first || kk > 0) ? 1u : 0u);
-            mma_commit(bar_addr(sbase, GEMPTY + gs));
-            ++cg;
-          }
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tbase + 128 * ab, sdesc_add(dA, gs * kTile + kk * 2048), sdesc_add(dB, ks * kTile + kk * 2048),
+                   id, (kt < U.hi || kk > 0) ? 1u : 0u);
+          mma_commit(bar_addr(sbase, GEMPTY + gs));
           mma_commit(bar_addr(sbase, KEMPTY + ks));
         }
         if (!ok) break;
@@ -228,9 +206,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int u = unit_index(cta, r, G);
       if (u >= p.n_units) break;
       const Unit U = decode(p, u);
-      const int ab = uidx & 1;
-      for (int t = 0; t < 1 + U.has1; ++t) {
-        const int i = (U.q0 + t) * 128 + row;
+      const int ab = uidx % kAcc;
+      {
+        const int i = U.qt * 128 + row;
         const bool iv = i < p.T;
         const size_t orow = (((size_t)U.b * p.T + (iv ? i : 0)) * p.H + U.h) * 128;
         // the whole q row, loaded before the wait for the accumulator so that its
@@ -241,13 +219,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 16; ++c) qv[c] = iv ? __ldg(qrow + c) : make_uint4(0, 0, 0, 0);
         }
-        if (t == 0 &&
-            !__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, ACCFULL + ab), (uidx >> 1) & 1, abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, ACCFULL + ab), (uidx / kAcc) & 1, abort_flag))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t tA = tbase + 256 * ab + 128 * t + lane_off;
+        const uint32_t tA = tbase + 128 * ab + lane_off;
         // pass 1: (acc . q) and sum q^2
         float ss = 0.f, dot = 0.f;
 #pragma unroll

@@ -209,12 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
           for (int c = 0; c < 16; ++c) {  // 16-byte chunk c of the row
             const uint4 x = lds128(kt + (c >> 3) * kHalf + sw128(row, c & 7));
-            const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float a = bf16lo(w4[e]), b = bf16hi(w4[e]);
-              ffma2(s0, s1, a, b, a, b, s0, s1);
-            }
+            fma_sq_bf16x2_f32(s0, s1, x.x);
+            fma_sq_bf16x2_f32(s0, s1, x.y);
+            fma_sq_bf16x2_f32(s0, s1, x.z);
+            fma_sq_bf16x2_f32(s0, s1, x.w);
           }
           const float ck = (n * 128 + row < p.T) ? rsqrtf((s0 + s1) * (1.0f / 128.0f) + p.eps) * p.cscale : 0.f;
           sts_f32(sbase + kCK + (kv % kCkSlots) * 512 + 4 * row, ck);
@@ -481,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   }
                   fadd2(l0, l1, p0, p1);
                   const uint32_t pp = pack_bf16(p0, p1);
-                  fadd2(lr0, lr1, bf16lo(pp), bf16hi(pp));
+                  add_bf16x2_f32(lr0, lr1, pp);
                   pk[2 * j4 + h2] = pp;
                 }
               }

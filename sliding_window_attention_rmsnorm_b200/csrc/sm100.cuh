@@ -338,6 +338,20 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 __device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+// c0 += lo, c1 += hi for the two bf16 halves of u: mixed-precision adds (bf16
+// operand, f32 accumulator, one rounding each), the same values as converting
+// the halves to f32 first, without the conversions.
+__device__ __forceinline__ void add_bf16x2_f32(float& c0, float& c1, uint32_t u) {
+  asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %2;\n add.rn.f32.bf16 %0, lo, %0;\n add.rn.f32.bf16 %1, hi, %1;\n}"
+      : "+f"(c0), "+f"(c1)
+      : "r"(u));
+}
+// c0 += lo * lo, c1 += hi * hi (the products are exact in f32; one rounding each)
+__device__ __forceinline__ void fma_sq_bf16x2_f32(float& c0, float& c1, uint32_t u) {
+  asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %2;\n fma.rn.f32.bf16 %0, lo, lo, %0;\n fma.rn.f32.bf16 %1, hi, hi, %1;\n}"
+      : "+f"(c0), "+f"(c1)
+      : "r"(u));
+}
 
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` inside a 128-byte-swizzled
 // tile of 128-byte rows (the layout TMA writes with SWIZZLE_128B).
