@@ -150,6 +150,7 @@ ar::FwdParams fwd_params(void* o, float* lse, const float* ck, int B, int T, int
   p.eps = eps;
   p.bound = scale * 128.0f * 1.4426950408889634f;
   p.cscale = scale * 1.4426950408889634f;
+  p.wide = aligned(o, 32);
   return p;
 }
 
@@ -381,6 +382,7 @@ int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, cons
     p.pairs_head = (int)ph;
     p.eps = eps;
     p.scale = scale;
+    p.wide = aligned(dk, 32) && aligned(dv, 32);
     {
       KernelTimer t(AR_KERNEL_BWD, s);
       ar::bwd::bwd_kernel<<<std::min(p.n_units, sms), ar::bwd::kThreads, ar::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo,
@@ -402,6 +404,7 @@ int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, cons
     d.pairs_head = (int)ph;
     d.eps = eps;
     d.scale = scale;
+    d.wide = aligned(dq, 32);
     {
       KernelTimer t(AR_KERNEL_DQ, s);
       ar::dqk::dq_kernel<<<std::min(d.n_units, sms), ar::dqk::kThreads, ar::dqk::kSmemBytes, s>>>(tg, tk, d);

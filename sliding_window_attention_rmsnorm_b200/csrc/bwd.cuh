@@ -54,6 +54,7 @@ struct BwdParams {
   int nb;          // key tiles in one query tile's band: min(nk, floor((w + 127) / 128) + 1)
   int pairs_head;  // G tiles per head: sum over query tiles of min(qt + 1, nb)
   float eps, scale;
+  int wide;  // dk and dv are 32-byte aligned: rows are written with 256-bit stores
 };
 
 // Slot of the G tile of (query tile qt, key tile kt) of the launch's head
@@ -500,19 +501,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t x[32];
             tmem_ld32(tDK + 32 * c, x);
             tmem_wait_ld();
+            uint32_t pk[16];
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
               const uint4 v = kv[4 * c + q4];
               const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-              uint32_t o4[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const float g0 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e]) - coef * bf16lo(w4[e]));
                 const float g1 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e + 1]) - coef * bf16hi(w4[e]));
-                o4[e] = pack_bf16(g0, g1);
+                pk[4 * q4 + e] = pack_bf16(g0, g1);
               }
-              if (jv)
-                *reinterpret_cast<uint4*>(p.dk + orow + 32 * c + 8 * q4) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            }
+            if (jv) {
+              stg32B(p.dk + orow + 32 * c, pk, p.wide);
+              stg32B(p.dk + orow + 32 * c + 16, pk + 8, p.wide);
             }
           }
         }
@@ -525,9 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]));
           if (jv) {
-            uint4* d = reinterpret_cast<uint4*>(p.dv + orow + 32 * c);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) d[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            stg32B(p.dv + orow + 32 * c, pk, p.wide);
+            stg32B(p.dv + orow + 32 * c + 16, pk + 8, p.wide);
           }
         }
         tc_fence_before();

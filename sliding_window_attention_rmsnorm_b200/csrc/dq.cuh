@@ -42,6 +42,7 @@ struct DqParams {
   int nb;          // key tiles in one query tile's band (as in the backward kernel)
   int pairs_head;  // G tiles per head
   float eps, scale;
+  int wide;        // dq is 32-byte aligned: rows are written with 256-bit stores
 };
 
 namespace dqk {
@@ -251,19 +252,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t x[32];
           tmem_ld32(tA + 32 * cc, x);
           tmem_wait_ld();
+          uint32_t pk[16];
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             const uint4 v = qv[4 * cc + q4];
             const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-            uint32_t o4[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float g0 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e]) - coef * bf16lo(w4[e]));
               const float g1 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e + 1]) - coef * bf16hi(w4[e]));
-              o4[e] = pack_bf16(g0, g1);
+              pk[4 * q4 + e] = pack_bf16(g0, g1);
             }
-            if (iv)
-              *reinterpret_cast<uint4*>(p.dq + orow + 32 * cc + 8 * q4) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+          }
+          if (iv) {
+            stg32B(p.dq + orow + 32 * cc, pk, p.wide);
+            stg32B(p.dq + orow + 32 * cc + 16, pk + 8, p.wide);
           }
         }
       }

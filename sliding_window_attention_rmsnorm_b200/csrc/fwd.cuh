@@ -66,6 +66,7 @@ struct FwdParams {
   float eps;
   float bound;       // scale * D * log2(e): the largest |logit| in log2 units
   float cscale;      // scale * log2(e)
+  int wide;          // o is 32-byte aligned: rows are written with 256-bit stores
 };
 
 namespace fwd {
@@ -606,9 +607,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[e] = pack_bf16(a0, a1);
         }
         if (iv) {
-          uint4* d = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) d[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          stg32B(orow + 32 * c, pk, p.wide);
+          stg32B(orow + 32 * c + 16, pk + 8, p.wide);
         }
       }
       tc_fence_before();

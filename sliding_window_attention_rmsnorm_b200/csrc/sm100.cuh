@@ -353,6 +353,22 @@ __device__ __forceinline__ void fma_sq_bf16x2_f32(float& c0, float& c1, uint32_t
       : "r"(u));
 }
 
+// 32 bytes (w[0..7]) to global memory at dst: one 256-bit store when `wide`
+// (dst 32-byte aligned), else two 128-bit stores (dst 16-byte aligned).  A warp
+// whose lanes each write a different row touches one 32-byte sector per lane
+// either way; the wide form needs half the store instructions.
+__device__ __forceinline__ void stg32B(void* dst, const uint32_t* w, bool wide) {
+  if (wide) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
+                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+  } else {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+    d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` inside a 128-byte-swizzled
 // tile of 128-byte rows (the layout TMA writes with SWIZZLE_128B).
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t c) { return r * 128u + ((c ^ (r & 7u)) << 4); }

@@ -241,3 +241,27 @@ def test_masked_positions_zero_gradient_on_gpu():
     outside = [j for j in range(T) if not (i0 - w <= j <= i0)]
     assert np.all(g["dk"][:, outside] == 0) and np.all(g["dv"][:, outside] == 0)
     assert np.all(g["dq"][:, np.arange(T) != i0] == 0)
+
+
+def test_outputs_16_byte_aligned_match_aligned_outputs():
+    """Outputs that start 16 bytes past a 32-byte boundary take the 128-bit
+    store path of the epilogues; every value matches the 256-bit path bitwise."""
+    B, T, H, w = 2, 300, 3, 100
+    x = synth.layer_inputs(17, 0, B, T, H, 128)
+    q, k, v, dO = (x[r].cuda() for r in ("q", "k", "v", "dO"))
+    n = B * T * H * 128
+
+    def offset_out():
+        buf = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")
+        t = buf[8:].view(B, T, H, 128)  # 8 bf16 = 16 bytes past the allocation's start
+        assert t.data_ptr() % 32 == 16
+        return t
+
+    o_ref, lse_ref = attn.fwd(q, k, v, w)
+    g_ref = attn.bwd(q, k, v, o_ref, dO, lse_ref, w)
+    o, lse = attn.fwd(q, k, v, w, out=offset_out())
+    g = attn.bwd(q, k, v, o, dO, lse, w, dq=offset_out(), dk=offset_out(), dv=offset_out())
+    attn.sync_status()
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+    for a, b in zip(g, g_ref):
+        assert torch.equal(a, b)
