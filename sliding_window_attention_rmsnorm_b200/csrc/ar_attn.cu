@@ -383,6 +383,7 @@ int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, cons
     p.eps = eps;
     p.scale = scale;
     p.wide = aligned(dk, 32) && aligned(dv, 32);
+    p.wide_k = aligned(k, 32);
     {
       KernelTimer t(AR_KERNEL_BWD, s);
       ar::bwd::bwd_kernel<<<std::min(p.n_units, sms), ar::bwd::kThreads, ar::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo,
@@ -405,6 +406,7 @@ int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, cons
     d.eps = eps;
     d.scale = scale;
     d.wide = aligned(dq, 32);
+    d.wide_q = aligned(q, 32);
     {
       KernelTimer t(AR_KERNEL_DQ, s);
       ar::dqk::dq_kernel<<<std::min(d.n_units, sms), ar::dqk::kThreads, ar::dqk::kSmemBytes, s>>>(tg, tk, d);

@@ -54,7 +54,8 @@ struct BwdParams {
   int nb;          // key tiles in one query tile's band: min(nk, floor((w + 127) / 128) + 1)
   int pairs_head;  // G tiles per head: sum over query tiles of min(qt + 1, nb)
   float eps, scale;
-  int wide;  // dk and dv are 32-byte aligned: rows are written with 256-bit stores
+  int wide;    // dk and dv are 32-byte aligned: rows are written with 256-bit stores
+  int wide_k;  // k is 32-byte aligned: key rows are read with 256-bit loads
 };
 
 // Slot of the G tile of (query tile qt, key tile kt) of the launch's head
@@ -490,7 +491,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           {
             const uint4* krow = reinterpret_cast<const uint4*>(p.k + orow);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) kv[c] = jv ? __ldg(krow + c) : make_uint4(0, 0, 0, 0);
+            for (int c = 0; c < 16; c += 2) {
+              if (jv) {
+                ldg32B(krow + c, kv[c], kv[c + 1], p.wide_k);
+              } else {
+                kv[c] = make_uint4(0, 0, 0, 0);
+                kv[c + 1] = kv[c];
+              }
+            }
           }
           if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DKDVDONE), uidx & 1, abort_flag))) break;
           tc_fence_after();

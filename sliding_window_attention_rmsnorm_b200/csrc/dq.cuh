@@ -43,6 +43,7 @@ struct DqParams {
   int pairs_head;  // G tiles per head
   float eps, scale;
   int wide;        // dq is 32-byte aligned: rows are written with 256-bit stores
+  int wide_q;      // q is 32-byte aligned: query rows are read with 256-bit loads
 };
 
 namespace dqk {
@@ -218,7 +219,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
           const uint4* qrow = reinterpret_cast<const uint4*>(p.q + orow);
 #pragma unroll
-          for (int c = 0; c < 16; ++c) qv[c] = iv ? __ldg(qrow + c) : make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < 16; c += 2) {
+            if (iv) {
+              ldg32B(qrow + c, qv[c], qv[c + 1], p.wide_q);
+            } else {
+              qv[c] = make_uint4(0, 0, 0, 0);
+              qv[c + 1] = qv[c];
+            }
+          }
         }
         if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, ACCFULL + ab), (uidx / kAcc) & 1, abort_flag))) {
           ok = false;

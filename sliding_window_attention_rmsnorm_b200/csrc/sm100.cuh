@@ -369,6 +369,19 @@ __device__ __forceinline__ void stg32B(void* dst, const uint32_t* w, bool wide) 
   }
 }
 
+// 32 bytes from global memory at src (read-only for the kernel's lifetime) into
+// a, b: one 256-bit load when `wide` (src 32-byte aligned), else two 128-bit loads.
+__device__ __forceinline__ void ldg32B(const void* src, uint4& a, uint4& b, bool wide) {
+  if (wide) {
+    asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(src));
+  } else {
+    a = __ldg(reinterpret_cast<const uint4*>(src));
+    b = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+  }
+}
+
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` inside a 128-byte-swizzled
 // tile of 128-byte rows (the layout TMA writes with SWIZZLE_128B).
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t c) { return r * 128u + ((c ^ (r & 7u)) << 4); }

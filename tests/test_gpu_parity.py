@@ -243,24 +243,28 @@ def test_masked_positions_zero_gradient_on_gpu():
     assert np.all(g["dq"][:, np.arange(T) != i0] == 0)
 
 
-def test_outputs_16_byte_aligned_match_aligned_outputs():
-    """Outputs that start 16 bytes past a 32-byte boundary take the 128-bit
-    store path of the epilogues; every value matches the 256-bit path bitwise."""
+def test_16_byte_aligned_tensors_match_aligned_ones():
+    """Tensors that start 16 bytes past a 32-byte boundary take the 128-bit load
+    and store paths of the epilogues; every value matches the 256-bit paths
+    bitwise."""
     B, T, H, w = 2, 300, 3, 100
     x = synth.layer_inputs(17, 0, B, T, H, 128)
     q, k, v, dO = (x[r].cuda() for r in ("q", "k", "v", "dO"))
     n = B * T * H * 128
 
-    def offset_out():
+    def offset(src=None):
         buf = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")
         t = buf[8:].view(B, T, H, 128)  # 8 bf16 = 16 bytes past the allocation's start
         assert t.data_ptr() % 32 == 16
+        if src is not None:
+            t.copy_(src)
         return t
 
     o_ref, lse_ref = attn.fwd(q, k, v, w)
     g_ref = attn.bwd(q, k, v, o_ref, dO, lse_ref, w)
-    o, lse = attn.fwd(q, k, v, w, out=offset_out())
-    g = attn.bwd(q, k, v, o, dO, lse, w, dq=offset_out(), dk=offset_out(), dv=offset_out())
+    qo, ko, vo, dOo = offset(q), offset(k), offset(v), offset(dO)
+    o, lse = attn.fwd(qo, ko, vo, w, out=offset())
+    g = attn.bwd(qo, ko, vo, o, dOo, lse, w, dq=offset(), dk=offset(), dv=offset())
     attn.sync_status()
     assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
     for a, b in zip(g, g_ref):
