@@ -107,12 +107,12 @@ def measured_peaks():
 # (profiles/attn_kernels_layer_s.md: S layer, B=8 T=2048 H=4), valid only while the
 # kernel's sources are byte-identical to the ones captured.
 CAPTURED_TRAFFIC = {
-    "bwd": {"bytes": 164986880,
-            "sources": {"bwd.cuh": "80dbd11ac28e914c51d4ca0bd16e050baa3010c5dbe74cc803a65c8697b72375",
-                        "sm100.cuh": "1f75d6b366e1dd63f0d435e45d60e33b7e6c830520b43fb92a71525c55af7687"}},
-    "fwd": {"bytes": 52677376,
-            "sources": {"fwd.cuh": "87059832b70c5f7fd6619e7fbc79e22377e1a1e2df087d3b89a5bf775b619044",
-                        "sm100.cuh": "1f75d6b366e1dd63f0d435e45d60e33b7e6c830520b43fb92a71525c55af7687"}},
+    "bwd": {"bytes": 167386112,
+            "sources": {"bwd.cuh": "4f1cda0699923ec45c81c71364d9c8f0aa436e52416facee433476de96112dd2",
+                        "sm100.cuh": "cea2fd62bb5f0b803ae6ea4e5190ce97adea9f5b5598bee2001819a0a7ba2e12"}},
+    "fwd": {"bytes": 52466944,
+            "sources": {"fwd.cuh": "8c5d56f92488669952d28517e8ebf289df8e697f2acea0cd6dd4306d3afa92b1",
+                        "sm100.cuh": "cea2fd62bb5f0b803ae6ea4e5190ce97adea9f5b5598bee2001819a0a7ba2e12"}},
 }
 
 
