@@ -22,8 +22,10 @@
  *     sees only itself.
  *   - eps >= 0 and finite; scale > 0 and finite (usually 1/sqrt(D)).
  *   - All pointers are DEVICE pointers of the current CUDA device, 16-byte
- *     aligned (the kernels read them with TMA).  The caller owns every buffer;
- *     the library never frees or retains caller memory.
+ *     aligned (the kernels read them with TMA).  32-byte aligned o, dq, dk, dv
+ *     (and q, k) are written (read) by the epilogues with 256-bit accesses,
+ *     which is faster; results are identical either way.  The caller owns
+ *     every buffer; the library never frees or retains caller memory.
  *   - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Calls only enqueue work and return; results are ready when the stream is.
  *   - Return value: AR_OK (0) or a negative AR_ERR_* code.  No exception or
