@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="stack8")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    ap.add_argument("--ref-seconds", type=float, default=60.0,
+                    help="--impl reference: oracle time budget for the whole run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -220,7 +222,7 @@ def run_reference(args, wl, rank, world):
     if rank != 0:
         return
     from oracle import oracle as orc
-    per_step = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    per_step = max(1.0, args.ref_seconds / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         oracle_sample(wl, 0.0)
     flops, secs, desc, threads = 0.0, 0.0, "", orc.num_threads()
@@ -240,6 +242,22 @@ def run_reference(args, wl, rank, world):
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- multi-rank helpers
+def max_over_ranks(dist, x, device):
+    """x maximised over all ranks (x itself in a single process)."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world, flops_per_rank_step, ms_per_step):
+    """Whole-job rate: every rank runs the same step, timed by the slowest rank."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
 
 
 # ---------------------------------------------------------------- our CUDA path
@@ -294,16 +312,13 @@ def run_ours(args, wl, rank, world, dist):
     attn.timing_enable(False)
     attn.sync_status()
     kern = attn.timing_read()
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(dist, ms, "cuda")
     clocks = None
     if sampler is not None:
         sampler.stop()
         clocks = sampler.summary(t_wall0, t_wall1)
 
-    value = world * (fwd_f + bwd_f) / (ms * 1e-3) / 1e12
+    value = job_tflops(world, fwd_f + bwd_f, ms)
     peaks = measured_peaks()
 
     # roofline of the dominant kernel: counted FLOPs per launch over its event-timed mean duration
@@ -358,13 +373,10 @@ def run_ours(args, wl, rank, world, dist):
         a1.record(stream)
         torch.cuda.synchronize()
         ms_e2e = a0.elapsed_time(a1) / args.e2e_steps
-        if dist is not None:
-            t = torch.tensor([ms_e2e], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = max_over_ranks(dist, ms_e2e, "cuda")
         h2d = sum(t.numel() * t.element_size() for x in pinned for t in x.values())
         d2h = sum(t.numel() * t.element_size() for x in outs_h for t in x.values())
-        e2e = {"value": world * (fwd_f + bwd_f) / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_tflops(world, fwd_f + bwd_f, ms_e2e), "unit": "TFLOP/s",
                "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     cpu = None
