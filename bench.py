@@ -113,7 +113,7 @@ CAPTURED_TRAFFIC = {
             "sources": {"bwd.cuh": "4f1cda0699923ec45c81c71364d9c8f0aa436e52416facee433476de96112dd2",
                         "sm100.cuh": "cea2fd62bb5f0b803ae6ea4e5190ce97adea9f5b5598bee2001819a0a7ba2e12"}},
     "fwd": {"bytes": 52466944,
-            "sources": {"fwd.cuh": "8c5d56f92488669952d28517e8ebf289df8e697f2acea0cd6dd4306d3afa92b1",
+            "sources": {"fwd.cuh": "ecbb304d05850280362d603c41d992a6d553bd89550841fb6f32b88b8a386768",
                         "sm100.cuh": "cea2fd62bb5f0b803ae6ea4e5190ce97adea9f5b5598bee2001819a0a7ba2e12"}},
 }
 

@@ -10,8 +10,8 @@
 // The norm is folded into the logits as a rank-1 scale: the tensor core
 // multiplies the raw bf16 q and k, and the softmax warps apply
 // rq_i * (rk_j * scale * log2 e), where rq_i comes from the Q tile in shared
-// memory and rk_j from a per-key pre-pass (`ck`).  q and k are never rounded
-// after normalisation.
+// memory and the per-key factor (`ck`) from the K tile, computed by the
+// key-factor warps below.  q and k are never rounded after normalisation.
 //
 // CTA organisation (persistent, one CTA per SM, 512 threads):
 //   warps 0-3  softmax warpgroup 0: query tile 0 (rows r0..r0+127), one row per thread
