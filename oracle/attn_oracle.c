@@ -18,14 +18,21 @@
  *     and section 5.2.2 "sliding window attention").  window < 0 means no
  *     left limit (full causal).
  *   - the analytic backward of both, with the RMSNorm gradient.
+ *   - grouped K/V heads (n_kv_head < n_head: "autoresearch" README, section 7.3,
+ *     where n_kv_head may be smaller than n_head, and section 10.2.1, item 4,
+ *     n_kv_head = n_head / 2): query head h reads K/V head h / (H / Hkv), as in
+ *     FlashAttention's grouped-query convention, and dk, dv of a K/V head sum
+ *     the contributions of every query head of its group.  Hkv = H is plain
+ *     multi-head attention.
  *
  * Everything is the plain definition written out in fp64: two-pass softmax
  * (max, then sum), delta computed as sum_j P_ij dP_ij (not as dO.o), and the
  * key-side gradients computed column by column.  No tiling, no fusion, no
  * online softmax.
  *
- * Layouts: q, k, v, o, dO, dq, dk, dv are [B, T, H, D] row-major fp64;
- * lse and delta are [B, H, T].  Work is split over (head, row) with OpenMP.
+ * Layouts: q, o, dO, dq are [B, T, H, D] row-major fp64; k, v, dk, dv are
+ * [B, T, Hkv, D]; lse and delta are [B, H, T].  Work is split over (head, row)
+ * with OpenMP.
  *
  * Parity status: every function here is pinned by the CPU tests
  * (library cross-check, finite differences, closed forms, invariants).
@@ -86,13 +93,17 @@ static double dot(const double *a, const double *b, long D) {
     return s;
 }
 
-/* Per-head views: row t of head (b, h) starts at ((b*T + t)*H + h)*D. */
-#define ROW(ptr, b, t, h) ((ptr) + ((((long)(b) * T + (t)) * H + (h)) * D))
+/* Per-head views: row t of head (b, h) of a tensor with NH heads starts at
+ * ((b*T + t)*NH + h)*D.  ROW is a query-side tensor (H heads), KROW a K/V-side
+ * tensor (Hkv heads). */
+#define ROWN(ptr, b, t, h, NH) ((ptr) + ((((long)(b) * T + (t)) * (NH) + (h)) * D))
+#define ROW(ptr, b, t, h) ROWN(ptr, b, t, h, H)
+#define KROW(ptr, b, t, h) ROWN(ptr, b, t, h, Hkv)
 
-/* Normalise all rows of one head of x into xh (T x D contiguous), r into rr. */
-static void norm_head(const double *x, long b, long h, long T, long H, long D, double eps,
+/* Normalise all rows of one head of x (NH heads) into xh (T x D contiguous), r into rr. */
+static void norm_head(const double *x, long b, long h, long T, long NH, long D, double eps,
                       double *xh, double *rr) {
-    for (long t = 0; t < T; ++t) rr[t] = rms_row(ROW(x, b, t, h), D, eps, xh + t * D);
+    for (long t = 0; t < T; ++t) rr[t] = rms_row(ROWN(x, b, t, h, NH), D, eps, xh + t * D);
 }
 
 /* Softmax statistics of query row i: returns lse_i; s_ij over visible keys. */
@@ -112,22 +123,24 @@ static double row_lse(const double *qh, const double *kh, long i, long w, long D
 }
 
 /*
- * Forward for the heads listed in `heads` (flat b*H + h indices; NULL means
- * all B*H heads).  Writes o [B,T,H,D] and lse [B,H,T] for those heads only.
+ * Forward for the query heads listed in `heads` (flat b*H + h indices; NULL
+ * means all B*H heads).  Writes o [B,T,H,D] and lse [B,H,T] for those heads
+ * only.  k and v have Hkv heads (H a multiple of Hkv).
  */
-void oracle_attn_fwd(const double *q, const double *k, const double *v,
-                     long B, long T, long H, long D, long window, double eps, double scale,
-                     double *o, double *lse, const long *heads, long n_heads) {
+void oracle_attn_fwd_gqa(const double *q, const double *k, const double *v,
+                         long B, long T, long H, long Hkv, long D, long window, double eps, double scale,
+                         double *o, double *lse, const long *heads, long n_heads) {
     long nh = heads ? n_heads : B * H;
+    long grp = H / Hkv;
     double *qh = (double *)malloc(sizeof(double) * T * D);
     double *kh = (double *)malloc(sizeof(double) * T * D);
     double *rq = (double *)malloc(sizeof(double) * T);
     double *rk = (double *)malloc(sizeof(double) * T);
     for (long n = 0; n < nh; ++n) {
         long bh = heads ? heads[n] : n;
-        long b = bh / H, h = bh % H;
+        long b = bh / H, h = bh % H, hk = h / grp;
         norm_head(q, b, h, T, H, D, eps, qh, rq);
-        norm_head(k, b, h, T, H, D, eps, kh, rk);
+        norm_head(k, b, hk, T, Hkv, D, eps, kh, rk);
 #pragma omp parallel for schedule(dynamic, 4)
         for (long i = 0; i < T; ++i) {
             double L = row_lse(qh, kh, i, window, D, scale);
@@ -136,7 +149,7 @@ void oracle_attn_fwd(const double *q, const double *k, const double *v,
             for (long d = 0; d < D; ++d) oi[d] = 0.0;
             for (long j = first_key(i, window); j <= i; ++j) {
                 double p = exp(scale * dot(qh + i * D, kh + j * D, D) - L);
-                const double *vj = ROW(v, b, j, h);
+                const double *vj = KROW(v, b, j, hk);
                 for (long d = 0; d < D; ++d) oi[d] += p * vj[d];
             }
         }
@@ -144,78 +157,105 @@ void oracle_attn_fwd(const double *q, const double *k, const double *v,
     free(qh); free(kh); free(rq); free(rk);
 }
 
-/*
- * Backward for the listed heads.  Recomputes the forward statistics, then:
- *   dV_j = sum_i P_ij dO_i ; dP_ij = dO_i . v_j ; delta_i = sum_j P_ij dP_ij ;
- *   dS_ij = P_ij (dP_ij - delta_i) ;
- *   dqhat_i = scale sum_j dS_ij khat_j ; dkhat_j = scale sum_i dS_ij qhat_i ;
- *   dq, dk through the RMSNorm gradient.
- * Also returns lse and delta [B,H,T] (may be NULL).
- */
-void oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dO,
+void oracle_attn_fwd(const double *q, const double *k, const double *v,
                      long B, long T, long H, long D, long window, double eps, double scale,
-                     double *dq, double *dk, double *dv, double *lse_out, double *delta_out,
-                     const long *heads, long n_heads) {
-    long nh = heads ? n_heads : B * H;
+                     double *o, double *lse, const long *heads, long n_heads) {
+    oracle_attn_fwd_gqa(q, k, v, B, T, H, H, D, window, eps, scale, o, lse, heads, n_heads);
+}
+
+/*
+ * Backward for the K/V heads listed in `heads` (flat b*Hkv + hk indices; NULL
+ * means all B*Hkv heads), and for every query head of their groups.
+ * Recomputes the forward statistics of each query head h, then:
+ *   dV_j = sum_h sum_i P_ij dO_i ; dP_ij = dO_i . v_j ; delta_i = sum_j P_ij dP_ij ;
+ *   dS_ij = P_ij (dP_ij - delta_i) ;
+ *   dqhat_i = scale sum_j dS_ij khat_j ; dkhat_j = scale sum_h sum_i dS_ij qhat_i ;
+ *   dq, dk through the RMSNorm gradient (sum_h over the query heads of the
+ *   K/V head's group; a single head when Hkv = H).
+ * Also returns lse and delta [B,H,T] of those query heads (may be NULL).
+ */
+void oracle_attn_bwd_gqa(const double *q, const double *k, const double *v, const double *dO,
+                         long B, long T, long H, long Hkv, long D, long window, double eps, double scale,
+                         double *dq, double *dk, double *dv, double *lse_out, double *delta_out,
+                         const long *heads, long n_heads) {
+    long nh = heads ? n_heads : B * Hkv;
+    long grp = H / Hkv;
     double *qh = (double *)malloc(sizeof(double) * T * D);
     double *kh = (double *)malloc(sizeof(double) * T * D);
     double *rq = (double *)malloc(sizeof(double) * T);
     double *rk = (double *)malloc(sizeof(double) * T);
     double *L = (double *)malloc(sizeof(double) * T);
     double *delta = (double *)malloc(sizeof(double) * T);
+    double *gk = (double *)malloc(sizeof(double) * T * D);  /* dkhat_j, summed over the group */
     for (long n = 0; n < nh; ++n) {
-        long bh = heads ? heads[n] : n;
-        long b = bh / H, h = bh % H;
-        norm_head(q, b, h, T, H, D, eps, qh, rq);
-        norm_head(k, b, h, T, H, D, eps, kh, rk);
-        /* Row pass: lse_i, delta_i, dq_i. */
-#pragma omp parallel for schedule(dynamic, 4)
-        for (long i = 0; i < T; ++i) {
-            const double *dOi = ROW(dO, b, i, h);
-            long j0 = first_key(i, window);
-            double Li = row_lse(qh, kh, i, window, D, scale);
-            double di = 0.0;
-            for (long j = j0; j <= i; ++j) {
-                double p = exp(scale * dot(qh + i * D, kh + j * D, D) - Li);
-                di += p * dot(dOi, ROW(v, b, j, h), D);
-            }
-            L[i] = Li;
-            delta[i] = di;
-            double *g = (double *)malloc(sizeof(double) * D);
-            for (long d = 0; d < D; ++d) g[d] = 0.0;
-            for (long j = j0; j <= i; ++j) {
-                double p = exp(scale * dot(qh + i * D, kh + j * D, D) - Li);
-                double ds = p * (dot(dOi, ROW(v, b, j, h), D) - di);
-                for (long d = 0; d < D; ++d) g[d] += scale * ds * kh[j * D + d];
-            }
-            rms_row_bwd(g, qh + i * D, rq[i], D, ROW(dq, b, i, h));
-            free(g);
-        }
-        /* Column pass: dv_j, dk_j (needs every lse_i and delta_i). */
-#pragma omp parallel for schedule(dynamic, 4)
+        long bhk = heads ? heads[n] : n;
+        long b = bhk / Hkv, hk = bhk % Hkv;
+        norm_head(k, b, hk, T, Hkv, D, eps, kh, rk);
+        for (long t = 0; t < T * D; ++t) gk[t] = 0.0;
         for (long j = 0; j < T; ++j) {
-            double *g = (double *)malloc(sizeof(double) * D);
-            double *dvj = ROW(dv, b, j, h);
-            const double *vj = ROW(v, b, j, h);
-            for (long d = 0; d < D; ++d) { g[d] = 0.0; dvj[d] = 0.0; }
-            long i1 = last_query(j, window, T);
-            for (long i = j; i <= i1; ++i) {
-                if (!visible(i, j, window)) continue;
+            double *dvj = KROW(dv, b, j, hk);
+            for (long d = 0; d < D; ++d) dvj[d] = 0.0;
+        }
+        for (long h = hk * grp; h < (hk + 1) * grp; ++h) {
+            norm_head(q, b, h, T, H, D, eps, qh, rq);
+            /* Row pass: lse_i, delta_i, dq_i. */
+#pragma omp parallel for schedule(dynamic, 4)
+            for (long i = 0; i < T; ++i) {
                 const double *dOi = ROW(dO, b, i, h);
-                double p = exp(scale * dot(qh + i * D, kh + j * D, D) - L[i]);
-                double ds = p * (dot(dOi, vj, D) - delta[i]);
-                for (long d = 0; d < D; ++d) {
-                    dvj[d] += p * dOi[d];
-                    g[d] += scale * ds * qh[i * D + d];
+                long j0 = first_key(i, window);
+                double Li = row_lse(qh, kh, i, window, D, scale);
+                double di = 0.0;
+                for (long j = j0; j <= i; ++j) {
+                    double p = exp(scale * dot(qh + i * D, kh + j * D, D) - Li);
+                    di += p * dot(dOi, KROW(v, b, j, hk), D);
+                }
+                L[i] = Li;
+                delta[i] = di;
+                double *g = (double *)malloc(sizeof(double) * D);
+                for (long d = 0; d < D; ++d) g[d] = 0.0;
+                for (long j = j0; j <= i; ++j) {
+                    double p = exp(scale * dot(qh + i * D, kh + j * D, D) - Li);
+                    double ds = p * (dot(dOi, KROW(v, b, j, hk), D) - di);
+                    for (long d = 0; d < D; ++d) g[d] += scale * ds * kh[j * D + d];
+                }
+                rms_row_bwd(g, qh + i * D, rq[i], D, ROW(dq, b, i, h));
+                free(g);
+            }
+            /* Column pass: this query head's share of dv_j and dkhat_j (needs
+             * every lse_i and delta_i of the head). */
+#pragma omp parallel for schedule(dynamic, 4)
+            for (long j = 0; j < T; ++j) {
+                double *g = gk + j * D;
+                double *dvj = KROW(dv, b, j, hk);
+                const double *vj = KROW(v, b, j, hk);
+                long i1 = last_query(j, window, T);
+                for (long i = j; i <= i1; ++i) {
+                    if (!visible(i, j, window)) continue;
+                    const double *dOi = ROW(dO, b, i, h);
+                    double p = exp(scale * dot(qh + i * D, kh + j * D, D) - L[i]);
+                    double ds = p * (dot(dOi, vj, D) - delta[i]);
+                    for (long d = 0; d < D; ++d) {
+                        dvj[d] += p * dOi[d];
+                        g[d] += scale * ds * qh[i * D + d];
+                    }
                 }
             }
-            rms_row_bwd(g, kh + j * D, rk[j], D, ROW(dk, b, j, h));
-            free(g);
+            for (long i = 0; i < T; ++i) {
+                if (lse_out) lse_out[(b * H + h) * T + i] = L[i];
+                if (delta_out) delta_out[(b * H + h) * T + i] = delta[i];
+            }
         }
-        for (long i = 0; i < T; ++i) {
-            if (lse_out) lse_out[(b * H + h) * T + i] = L[i];
-            if (delta_out) delta_out[(b * H + h) * T + i] = delta[i];
-        }
+        /* dk through the RMSNorm gradient of the summed dkhat. */
+#pragma omp parallel for schedule(static)
+        for (long j = 0; j < T; ++j) rms_row_bwd(gk + j * D, kh + j * D, rk[j], D, KROW(dk, b, j, hk));
     }
-    free(qh); free(kh); free(rq); free(rk); free(L); free(delta);
+    free(qh); free(kh); free(rq); free(rk); free(L); free(delta); free(gk);
+}
+
+void oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dO,
+                     long B, long T, long H, long D, long window, double eps, double scale,
+                     double *dq, double *dk, double *dv, double *lse_out, double *delta_out,
+                     const long *heads, long n_heads) {
+    oracle_attn_bwd_gqa(q, k, v, dO, B, T, H, H, D, window, eps, scale, dq, dk, dv, lse_out, delta_out,
+                        heads, n_heads);
 }

@@ -66,6 +66,88 @@ def test_matches_torch_sdpa_fp64(B, T, H, D, window):
         np.testing.assert_allclose(a, b, rtol=0, atol=1e-10, err_msg=name)
 
 
+def torch_reference_gqa(q, k, v, dO, window, eps, scale):
+    """Grouped K/V heads through the same textbook composition: each K/V head is
+    repeated for the query heads of its group (query head h reads K/V head
+    h // (H // Hkv)), so autograd sums dk, dv over the group."""
+    H, Hkv = q.shape[2], k.shape[2]
+    kt, vt = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (k, v))
+    kr, vr = (x.repeat_interleave(H // Hkv, dim=2) for x in (kt, vt))
+    qt, dOt = (torch.tensor(x, dtype=torch.float64) for x in (q, dO))
+    qt.requires_grad_(True)
+    B, T, _, D = q.shape
+    qh = F.rms_norm(qt, (D,), eps=eps).transpose(1, 2)
+    kh = F.rms_norm(kr, (D,), eps=eps).transpose(1, 2)
+    i = torch.arange(T)[:, None]
+    j = torch.arange(T)[None, :]
+    mask = (j <= i) & ((i - j <= window) if window >= 0 else torch.ones_like(j <= i))
+    o = F.scaled_dot_product_attention(qh, kh, vr.transpose(1, 2), attn_mask=mask, scale=scale).transpose(1, 2)
+    (o * dOt).sum().backward()
+    return o.detach().numpy(), qt.grad.numpy(), kt.grad.numpy(), vt.grad.numpy()
+
+
+@pytest.mark.parametrize("B,T,H,Hkv,D,window", [
+    (1, 9, 2, 1, 8, -1), (2, 21, 4, 2, 16, 4), (1, 40, 6, 3, 128, 0), (1, 48, 4, 1, 64, 11),
+])
+def test_grouped_kv_heads_match_torch_sdpa_fp64(B, T, H, Hkv, D, window):
+    eps, scale = 1e-6, 1.0 / math.sqrt(D)
+    q, dO = rand((B, T, H, D), 40), rand((B, T, H, D), 41)
+    k, v = rand((B, T, Hkv, D), 42), rand((B, T, Hkv, D), 43)
+    ro, rdq, rdk, rdv = torch_reference_gqa(q, k, v, dO, window, eps, scale)
+    o, _ = orc.attn_fwd(q, k, v, window, eps, scale)
+    g = orc.attn_bwd(q, k, v, dO, window, eps, scale)
+    for name, a, b in [("o", o, ro), ("dq", g["dq"], rdq), ("dk", g["dk"], rdk), ("dv", g["dv"], rdv)]:
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-10, err_msg=name)
+
+
+def test_grouped_kv_heads_finite_differences():
+    """dk, dv of a shared K/V head against central differences of the forward."""
+    B, T, H, Hkv, D, window, eps = 1, 7, 4, 2, 4, 3, 1e-6
+    scale = 1.0 / math.sqrt(D)
+    q, dO = rand((B, T, H, D), 50), rand((B, T, H, D), 51)
+    k, v = rand((B, T, Hkv, D), 52), rand((B, T, Hkv, D), 53)
+    g = orc.attn_bwd(q, k, v, dO, window, eps, scale)
+
+    def loss(k_, v_):
+        o, _ = orc.attn_fwd(q, k_, v_, window, eps, scale)
+        return float(np.sum(o * dO))
+
+    h = 1e-6
+    for name, src in (("dk", 0), ("dv", 1)):
+        an = g[name]
+        gmax = np.abs(an).max()
+        for f in range(k.size):
+            args = [k.copy(), v.copy()]
+            args[src].flat[f] += h
+            lp = loss(*args)
+            args[src].flat[f] -= 2 * h
+            lm = loss(*args)
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - an.flat[f]) <= 1e-6 * (abs(an.flat[f]) + gmax), (name, f, fd, an.flat[f])
+
+
+def test_grouped_kv_heads_equal_duplicated_heads():
+    """Grouped K/V heads give the multi-head result on K/V duplicated per query
+    head, with dk, dv summed over each group; a K/V-head subset matches."""
+    B, T, H, Hkv, D, w = 2, 30, 6, 2, 16, 9
+    q, dO = rand((B, T, H, D), 60), rand((B, T, H, D), 61)
+    k, v = rand((B, T, Hkv, D), 62), rand((B, T, Hkv, D), 63)
+    kd, vd = np.repeat(k, H // Hkv, axis=2), np.repeat(v, H // Hkv, axis=2)
+    o, lse = orc.attn_fwd(q, k, v, w)
+    od, lsed = orc.attn_fwd(q, kd, vd, w)
+    np.testing.assert_allclose(o, od, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, lsed, rtol=0, atol=1e-13)
+    g, gd = orc.attn_bwd(q, k, v, dO, w), orc.attn_bwd(q, kd, vd, dO, w)
+    np.testing.assert_allclose(g["dq"], gd["dq"], rtol=0, atol=1e-12)
+    for n in ("dk", "dv"):
+        summed = gd[n].reshape(B, T, Hkv, H // Hkv, D).sum(axis=3)
+        np.testing.assert_allclose(g[n], summed, rtol=0, atol=1e-12)
+    sub = orc.attn_bwd(q, k, v, dO, w, heads=[1 * Hkv + 1])  # b = 1, K/V head 1
+    np.testing.assert_array_equal(sub["dk"][1, :, 1], g["dk"][1, :, 1])
+    np.testing.assert_array_equal(sub["dq"][1, :, 3:6], g["dq"][1, :, 3:6])
+    assert np.isnan(sub["dk"][0]).all()
+
+
 def test_delta_equals_rowsum_dO_o():
     """delta is computed as sum_j P dP; it must equal the row sum of dO*o."""
     B, T, H, D, w = 1, 30, 2, 16, 7
