@@ -95,6 +95,25 @@ int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, cons
                 int B, int T, int H, int D, int window, float eps, float scale,
                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* Grouped K/V heads ("autoresearch" README on gitee, section 7.3: n_kv_head
+ * may be smaller than n_head; section 10.2.1, item 4: n_kv_head = n_head / 2).
+ * k, v, dk, dv are [B, T, Hkv, D] with Hkv dividing H; q, o, dO, dq stay
+ * [B, T, H, D] and lse [B, H, T].  Query head h attends with K/V head
+ * h / (H / Hkv) (consecutive query heads share a K/V head, as in
+ * FlashAttention), and dk, dv of a K/V head sum the gradients of every query
+ * head of its group.  Hkv = H gives exactly ar_attn_fwd / ar_attn_bwd (which
+ * call these).  AR_ERR_SHAPE if Hkv < 1 or Hkv does not divide H; otherwise
+ * arguments, errors and the workspace contract are those of the functions
+ * above.  The backward processes whole groups per launch, so its workspace
+ * holds the G tiles of at least one group of H / Hkv query heads. */
+int ar_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int B, int T, int H, int Hkv, int D, int window, float eps, float scale, void* stream);
+size_t ar_attn_bwd_gqa_workspace_bytes(int B, int T, int H, int Hkv, int D);
+int ar_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                    const float* lse, void* dq, void* dk, void* dv,
+                    int B, int T, int H, int Hkv, int D, int window, float eps, float scale,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears this device's status word.
  * Returns AR_OK, AR_ERR_TIMEOUT if a kernel abandoned a wait since the last
  * call, or AR_ERR_CUDA if the synchronisation itself failed. */

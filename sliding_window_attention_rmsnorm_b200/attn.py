@@ -61,6 +61,12 @@ def lib():
         L.ar_attn_timing_enable.restype = i
         L.ar_attn_timing_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
         L.ar_attn_timing_read.restype = i
+        L.ar_attn_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, vp]
+        L.ar_attn_fwd_gqa.restype = i
+        L.ar_attn_bwd_gqa_workspace_bytes.argtypes = [i, i, i, i, i]
+        L.ar_attn_bwd_gqa_workspace_bytes.restype = sz
+        L.ar_attn_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, vp, sz, vp]
+        L.ar_attn_bwd_gqa.restype = i
         _lib = L
     return _lib
 
@@ -90,6 +96,17 @@ def _check_inputs(*ts):
             raise ValueError("q, k, v (and o, dO) must have the same shape")
 
 
+def _check_qkv(q, k, v):
+    """q [B, T, H, D]; k, v [B, T, Hkv, D] with Hkv dividing H.  Returns Hkv."""
+    _check_inputs(q)
+    _check_inputs(k, v)
+    B, T, H, D = q.shape
+    Hkv = k.shape[2]
+    if k.shape[0] != B or k.shape[1] != T or k.shape[3] != D or H % Hkv:
+        raise ValueError("k, v must be [B, T, Hkv, D] with Hkv dividing q's head count")
+    return Hkv
+
+
 def default_scale(D: int) -> float:
     return 1.0 / math.sqrt(D)
 
@@ -98,22 +115,31 @@ def fwd_workspace_bytes(B, T, H, D) -> int:
     return int(lib().ar_attn_fwd_workspace_bytes(B, T, H, D))
 
 
-def bwd_workspace_bytes(B, T, H, D) -> int:
-    return int(lib().ar_attn_bwd_workspace_bytes(B, T, H, D))
+def bwd_workspace_bytes(B, T, H, D, Hkv=None) -> int:
+    if Hkv is None or Hkv == H:
+        return int(lib().ar_attn_bwd_workspace_bytes(B, T, H, D))
+    return int(lib().ar_attn_bwd_gqa_workspace_bytes(B, T, H, Hkv, D))
 
 
 def fwd(q, k, v, window: int, eps: float = 1e-6, scale=None, out=None, lse=None, workspace=None):
     """o, lse = attention(norm(q), norm(k), v) over the band 0 <= i - j <= window.
 
-    q, k, v: bf16 CUDA tensors [B, T, H, 128].  Returns o (bf16, same shape)
-    and lse (fp32 [B, H, T]).  Enqueued on torch's current stream.
+    q: bf16 CUDA tensor [B, T, H, 128]; k, v: [B, T, Hkv, 128] with Hkv
+    dividing H (Hkv < H: grouped K/V heads, query head h reads K/V head
+    h // (H // Hkv)).  Returns o (bf16, like q) and lse (fp32 [B, H, T]).
+    Enqueued on torch's current stream.
     """
-    _check_inputs(q, k, v)
+    Hkv = _check_qkv(q, k, v)
     B, T, H, D = q.shape
     if scale is None:
         scale = default_scale(D)
     o = torch.empty_like(q) if out is None else out
     lse_t = torch.empty((B, H, T), dtype=torch.float32, device=q.device) if lse is None else lse
+    if Hkv != H:
+        st = lib().ar_attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, T, H, Hkv, D, int(window),
+                                   float(eps), float(scale), _stream())
+        _check(st, "ar_attn_fwd_gqa")
+        return o, lse_t
     if workspace is None:
         workspace = torch.empty(max(fwd_workspace_bytes(B, T, H, D), 1), dtype=torch.uint8, device=q.device)
     st = lib().ar_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, T, H, D, int(window),
@@ -124,18 +150,29 @@ def fwd(q, k, v, window: int, eps: float = 1e-6, scale=None, out=None, lse=None,
 
 def bwd(q, k, v, o, dO, lse, window: int, eps: float = 1e-6, scale=None, dq=None, dk=None, dv=None,
         workspace=None):
-    """dq, dk, dv of the forward above, given the upstream gradient dO."""
-    _check_inputs(q, k, v, o, dO)
+    """dq, dk, dv of the forward above, given the upstream gradient dO.
+
+    With grouped K/V heads, dk and dv ([B, T, Hkv, 128]) sum the gradients of
+    every query head of their group.
+    """
+    Hkv = _check_qkv(q, k, v)
+    _check_inputs(q, o, dO)
     B, T, H, D = q.shape
     if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, H, T)):
         raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, H, T]")
     if scale is None:
         scale = default_scale(D)
     dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
     if workspace is None:
-        workspace = torch.empty(bwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(bwd_workspace_bytes(B, T, H, D, Hkv), dtype=torch.uint8, device=q.device)
+    if Hkv != H:
+        st = lib().ar_attn_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq), _ptr(dk),
+                                   _ptr(dv), B, T, H, Hkv, D, int(window), float(eps), float(scale),
+                                   _ptr(workspace), workspace.numel(), _stream())
+        _check(st, "ar_attn_bwd_gqa")
+        return dq, dk, dv
     st = lib().ar_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
                            B, T, H, D, int(window), float(eps), float(scale), _ptr(workspace), workspace.numel(),
                            _stream())

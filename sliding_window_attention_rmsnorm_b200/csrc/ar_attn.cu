@@ -121,6 +121,9 @@ int check_args(float eps, float scale) {
 
 int effective_window(int window, int T) { return (window < 0 || window >= T - 1) ? T : window; }
 
+// Grouped K/V heads: Hkv divides H (Hkv = H is multi-head attention).
+int check_kv_heads(int H, int Hkv) { return (Hkv >= 1 && Hkv <= H && H % Hkv == 0) ? AR_OK : AR_ERR_SHAPE; }
+
 // [B, T, H, 128] bf16 viewed as a 4-D tensor (d, h, t, b); boxes of 64 x 1 x 128 x 1
 // land as 128 rows of 128 bytes with the 128-byte swizzle the MMA descriptors expect.
 int make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
@@ -134,8 +137,8 @@ int make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
   return r == CUDA_SUCCESS ? AR_OK : AR_ERR_CUDA;
 }
 
-ar::FwdParams fwd_params(void* o, float* lse, const float* ck, int B, int T, int H, int window, float eps,
-                         float scale) {
+ar::FwdParams fwd_params(void* o, float* lse, const float* ck, int B, int T, int H, int Hkv, int window,
+                         float eps, float scale) {
   ar::FwdParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -143,6 +146,7 @@ ar::FwdParams fwd_params(void* o, float* lse, const float* ck, int B, int T, int
   p.B = B;
   p.T = T;
   p.H = H;
+  p.grp = H / Hkv;
   p.T_pad = (T + 127) / 128 * 128;
   p.w = effective_window(window, T);
   p.nqp = (T + 255) / 256;
@@ -185,11 +189,13 @@ long long g_pairs_head(int T, int nb) {
   return nq <= nb ? nq * (nq + 1) / 2 : (long long)nb * (nb + 1) / 2 + (nq - nb) * nb;
 }
 size_t g_head_bytes(int T, int nb) { return (size_t)g_pairs_head(T, nb) * kGTile; }
-// Heads whose G tiles the workspace holds at once, sized for the widest band (full causal).
-size_t g_heads_cap(int B, int T, int H) {
+// Query heads whose G tiles the workspace holds at once, sized for the widest
+// band (full causal): whole groups of grp query heads (the heads that share a
+// K/V head are processed by one launch), at least one group.
+size_t g_heads_cap(int B, int T, int H, int grp) {
   const size_t per = g_head_bytes(T, (T + 127) / 128);
-  size_t n = kGBufferCap / per;
-  if (n < 1) n = 1;
+  size_t n = kGBufferCap / per / grp * grp;
+  if (n < (size_t)grp) n = grp;
   const size_t bh = (size_t)B * H;
   return n < bh ? n : bh;
 }
@@ -274,28 +280,31 @@ size_t ar_attn_fwd_workspace_bytes(int B, int T, int H, int D) {
   return 0;  // the forward kernel derives the per-key norm factors itself
 }
 
-size_t ar_attn_bwd_workspace_bytes(int B, int T, int H, int D) {
-  if (check_shape(B, T, H, D) != AR_OK) return 0;
-  return 3 * vec_bytes(B, T, H) + g_heads_cap(B, T, H) * g_head_bytes(T, (T + 127) / 128);
+size_t ar_attn_bwd_gqa_workspace_bytes(int B, int T, int H, int Hkv, int D) {
+  if (check_shape(B, T, H, D) != AR_OK || check_kv_heads(H, Hkv) != AR_OK) return 0;
+  return 3 * vec_bytes(B, T, H) + g_heads_cap(B, T, H, H / Hkv) * g_head_bytes(T, (T + 127) / 128);
 }
 
-int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T, int H, int D,
-                int window, float eps, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+size_t ar_attn_bwd_workspace_bytes(int B, int T, int H, int D) { return ar_attn_bwd_gqa_workspace_bytes(B, T, H, H, D); }
+
+int ar_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T, int H, int Hkv,
+                    int D, int window, float eps, float scale, void* stream) {
   if (!q || !k || !v || !o || !lse) return AR_ERR_NULL;
   int st = check_shape(B, T, H, D);
   if (st != AR_OK) return st;
+  if ((st = check_kv_heads(H, Hkv)) != AR_OK) return st;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return AR_ERR_ALIGN;
   if ((st = check_args(eps, scale)) != AR_OK) return st;
-  (void)workspace, (void)workspace_bytes;  // no scratch needed: see ar_attn_fwd_workspace_bytes
   int sms = 0;
   if ((st = device_setup(&sms)) != AR_OK) return st;
 
   CUtensorMap tq, tk, tv;
-  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, H) != AR_OK || make_map(&tv, v, B, T, H) != AR_OK)
+  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, Hkv) != AR_OK ||
+      make_map(&tv, v, B, T, Hkv) != AR_OK)
     return AR_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const ar::FwdParams p = fwd_params(o, lse, nullptr, B, T, H, window, eps, scale);
+  const ar::FwdParams p = fwd_params(o, lse, nullptr, B, T, H, Hkv, window, eps, scale);
   const int grid = p.n_units < sms ? p.n_units : sms;
   {
     KernelTimer t(AR_KERNEL_FWD, s);
@@ -305,30 +314,38 @@ int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
   return cudaGetLastError() == cudaSuccess ? AR_OK : AR_ERR_CUDA;
 }
 
-int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
-                void* dq, void* dk, void* dv, int B, int T, int H, int D, int window, float eps, float scale,
-                void* workspace, size_t workspace_bytes, void* stream) {
+int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T, int H, int D,
+                int window, float eps, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  (void)workspace, (void)workspace_bytes;  // no scratch needed: see ar_attn_fwd_workspace_bytes
+  return ar_attn_fwd_gqa(q, k, v, o, lse, B, T, H, H, D, window, eps, scale, stream);
+}
+
+int ar_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                    void* dq, void* dk, void* dv, int B, int T, int H, int Hkv, int D, int window, float eps,
+                    float scale, void* workspace, size_t workspace_bytes, void* stream) {
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return AR_ERR_NULL;
   int st = check_shape(B, T, H, D);
   if (st != AR_OK) return st;
+  if ((st = check_kv_heads(H, Hkv)) != AR_OK) return st;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
       !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
     return AR_ERR_ALIGN;
   if ((st = check_args(eps, scale)) != AR_OK) return st;
-  const size_t need = ar_attn_bwd_workspace_bytes(B, T, H, D);
+  const size_t need = ar_attn_bwd_gqa_workspace_bytes(B, T, H, Hkv, D);
   if (workspace && workspace_bytes < need) return AR_ERR_WORKSPACE;
   if (workspace && !aligned(workspace, 256)) return AR_ERR_ALIGN;
   int sms = 0;
   if ((st = device_setup(&sms)) != AR_OK) return st;
 
   CUtensorMap tq, tk, tv, tdo;
-  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, H) != AR_OK ||
-      make_map(&tv, v, B, T, H) != AR_OK || make_map(&tdo, dO, B, T, H) != AR_OK)
+  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, Hkv) != AR_OK ||
+      make_map(&tv, v, B, T, Hkv) != AR_OK || make_map(&tdo, dO, B, T, H) != AR_OK)
     return AR_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   void* ws = workspace;
   if (!ws && cudaMallocAsync(&ws, need, s) != cudaSuccess) return AR_ERR_CUDA;
 
+  const int grp = H / Hkv;
   const int T_pad = (T + 127) / 128 * 128;
   char* w8 = static_cast<char*>(ws);
   const size_t vb = vec_bytes(B, T, H);
@@ -349,19 +366,19 @@ int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, cons
   const int nk = (T + 127) / 128;
   const int nb = band_tiles(w, T);
   const long long ph = g_pairs_head(T, nb);
-  // heads per launch: as many as the G buffer holds for this window
-  const long long cap_tiles = (long long)g_heads_cap(B, T, H) * g_pairs_head(T, nk);
-  const int BH = B * H;
-  const int hpl_max = (int)std::min<long long>(BH, std::max<long long>(1, cap_tiles / ph));
-  const int n_groups = (BH + hpl_max - 1) / hpl_max;
-  const int hpl = (BH + n_groups - 1) / n_groups;  // equal groups
+  // K/V heads per launch: as many whole groups as the G buffer holds for this window
+  const long long cap_tiles = (long long)g_heads_cap(B, T, H, grp) * g_pairs_head(T, nk);
+  const int BKV = B * Hkv;
+  const int kpl_max = (int)std::min<long long>(BKV, std::max<long long>(1, cap_tiles / (ph * grp)));
+  const int n_groups = (BKV + kpl_max - 1) / kpl_max;
+  const int kpl = (BKV + n_groups - 1) / n_groups;  // equal launches
   CUtensorMap tg;
-  if (make_g_map(&tg, gbuf, 2 * (long long)hpl * ph * 128) != AR_OK) {
+  if (make_g_map(&tg, gbuf, 2 * (long long)kpl * grp * ph * 128) != AR_OK) {
     if (!workspace) cudaFreeAsync(ws, s);
     return AR_ERR_CUDA;
   }
-  for (int bh0 = 0; bh0 < BH; bh0 += hpl) {
-    const int n_bh = std::min(hpl, BH - bh0);
+  for (int bk0 = 0; bk0 < BKV; bk0 += kpl) {
+    const int n_bk = std::min(kpl, BKV - bk0);
     ar::BwdParams p;
     p.dk = static_cast<__nv_bfloat16*>(dk);
     p.dv = static_cast<__nv_bfloat16*>(dv);
@@ -373,11 +390,13 @@ int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, cons
     p.T = T;
     p.H = H;
     p.T_pad = T_pad;
+    p.Hkv = Hkv;
+    p.grp = grp;
     p.w = w;
     p.nk = nk;
-    p.n_units = n_bh * nk;
-    p.bh0 = bh0;
-    p.n_bh = n_bh;
+    p.n_units = n_bk * nk;
+    p.bh0 = bk0;
+    p.n_bh = n_bk;
     p.nb = nb;
     p.pairs_head = (int)ph;
     p.eps = eps;
@@ -396,11 +415,12 @@ int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, cons
     d.B = B;
     d.T = T;
     d.H = H;
+    d.grp = grp;
     d.w = w;
     d.nq = nk;
-    d.n_units = n_bh * nk;  // units of one query tile
-    d.bh0 = bh0;
-    d.n_bh = n_bh;
+    d.n_units = n_bk * grp * nk;  // units of one query tile of one query head
+    d.bh0 = bk0 * grp;            // the query heads of K/V heads bk0 .. bk0 + n_bk - 1
+    d.n_bh = n_bk * grp;
     d.nb = nb;
     d.pairs_head = (int)ph;
     d.eps = eps;
@@ -416,6 +436,13 @@ int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, cons
   cudaError_t e = cudaGetLastError();
   if (!workspace) cudaFreeAsync(ws, s);
   return e == cudaSuccess ? AR_OK : AR_ERR_CUDA;
+}
+
+int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                void* dq, void* dk, void* dv, int B, int T, int H, int D, int window, float eps, float scale,
+                void* workspace, size_t workspace_bytes, void* stream) {
+  return ar_attn_bwd_gqa(q, k, v, o, dO, lse, dq, dk, dv, B, T, H, H, D, window, eps, scale, workspace,
+                         workspace_bytes, stream);
 }
 
 int ar_attn_sync_status(void* stream) {
@@ -564,7 +591,7 @@ extern "C" int ar_attn_fwd_noalloc(const void* q, const void* k, const void* v, 
                                                               T_pad, eps, scale * 1.4426950408889634f);
     t.stop();
   }
-  const ar::FwdParams p = fwd_params(o, lse, ck, B, T, H, window, eps, scale);
+  const ar::FwdParams p = fwd_params(o, lse, ck, B, T, H, H, window, eps, scale);
   const int grid = p.n_units < sms ? p.n_units : sms;
   {
     KernelTimer t(AR_KERNEL_FWD, s);

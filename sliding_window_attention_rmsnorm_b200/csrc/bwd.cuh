@@ -1,7 +1,9 @@
 // Fused QK-RMSNorm + band-limited causal attention, backward main kernel, sm_100a.
 //
 // For one head and one tile of 128 keys j, loops over the query tiles i whose
-// band reaches those keys and accumulates (s_ij as in the forward pass):
+// band reaches those keys and accumulates (s_ij as in the forward pass; with
+// grouped K/V heads the loop runs over those query tiles of every query head
+// of the K/V head's group, so dK and dV sum the group's contributions):
 //   P_ij  = exp(s_ij - lse_i)                      recomputed from the saved lse
 //   dV_j += sum_i P_ij dO_i
 //   dP_ij = dO_i . v_j,  dS_ij = P_ij (dP_ij - delta_i),  delta_i = dO_i . o_i
@@ -40,17 +42,18 @@
 namespace ar {
 
 struct BwdParams {
-  __nv_bfloat16* dk;       // [B, T, H, 128]
-  __nv_bfloat16* dv;       // [B, T, H, 128]
-  const __nv_bfloat16* k;  // [B, T, H, 128] raw keys, for the dk epilogue
+  __nv_bfloat16* dk;       // [B, T, Hkv, 128]
+  __nv_bfloat16* dv;       // [B, T, Hkv, 128]
+  const __nv_bfloat16* k;  // [B, T, Hkv, 128] raw keys, for the dk epilogue
   const float* lse2;       // [B*H, T_pad] lse * log2(e), 0 on padding
   const float* delta;      // [B*H, T_pad] rowsum(dO * o), 0 on padding
   const float* rq;         // [B*H, T_pad] 1/rms(q_i), 0 on padding
   int B, T, H, T_pad;
+  int Hkv, grp;  // K/V heads and query heads per K/V head (H = Hkv * grp; grp = 1: multi-head)
   int w;        // left window (w >= T means full causal)
   int nk;       // key tiles per head = ceil(T / 128)
   int n_units;  // n_bh * nk
-  int bh0, n_bh;   // heads bh0 .. bh0 + n_bh - 1 (b * H + h) are processed by this launch
+  int bh0, n_bh;   // K/V heads bh0 .. bh0 + n_bh - 1 (b * Hkv + hk) are processed by this launch
   int nb;          // key tiles in one query tile's band: min(nk, floor((w + 127) / 128) + 1)
   int pairs_head;  // G tiles per head: sum over query tiles of min(qt + 1, nb)
   float eps, scale;
@@ -58,9 +61,9 @@ struct BwdParams {
   int wide_k;  // k is 32-byte aligned: key rows are read with 256-bit loads
 };
 
-// Slot of the G tile of (query tile qt, key tile kt) of the launch's head
-// number hl (0 .. n_bh - 1) in the G buffer: query tiles in order, each followed
-// by its band's key tiles, newest first.
+// Slot of the G tile of (query tile qt, key tile kt) of the launch's query head
+// number hl (0 .. grp * n_bh - 1) in the G buffer: query tiles in order, each
+// followed by its band's key tiles, newest first.
 __device__ __forceinline__ long long g_pair(int hl, int qt, int kt, int nb, int pairs_head) {
   const long long before = qt <= nb ? (long long)qt * (qt + 1) / 2
                                     : (long long)nb * (nb + 1) / 2 + (long long)(qt - nb) * nb;
@@ -88,8 +91,14 @@ constexpr uint32_t kAbort = kTmemPtr + 4;
 constexpr uint32_t kSmemBytes = kAbort + 4;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
+// A unit: K/V head h (flat bh, local hl) and key tile kt.  Its N = grp * nq
+// iterations run the nq band query tiles qlo .. qlo + nq - 1 of each query head
+// of the group in turn: iteration it is query head h * grp + it / nq, query
+// tile qlo + it % nq.
 struct Unit {
-  int hl, bh, b, h, kt, qlo, N;
+  int hl, bh, b, h, kt, qlo, nq, N;
+  __device__ int qhead(int it) const { return it / nq; }  // group member
+  __device__ int qtile(int it) const { return qlo + it % nq; }
 };
 
 __device__ __forceinline__ int unit_index(int cta, int round, int G) {
@@ -102,12 +111,13 @@ __device__ __forceinline__ Unit decode(const BwdParams& p, int u) {
   U.kt = u / p.n_bh;
   U.hl = u % p.n_bh;
   U.bh = p.bh0 + U.hl;
-  U.b = U.bh / p.H;
-  U.h = U.bh % p.H;
+  U.b = U.bh / p.Hkv;
+  U.h = U.bh % p.Hkv;
   U.qlo = U.kt;
   const long long last_q = (long long)U.kt * 128 + 127 + p.w;
   const int qhi = (int)min((long long)(p.nk - 1), last_q / 128);
-  U.N = qhi - U.qlo + 1;
+  U.nq = qhi - U.qlo + 1;
+  U.N = p.grp * U.nq;
   return U;
 }
 
@@ -216,14 +226,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         last_kv_par = uidx & 1;
         for (int it = 0; it < U.N; ++it, ++qc) {
-          const int qt = U.qlo + it;
+          const int qt = U.qtile(it), hq = U.h * p.grp + U.qhead(it);
           const int st = qc & 1, ph = (qc >> 1) & 1;
           if (!mbar_wait(bar_addr(sbase, QEMPTY + st), ph ^ 1, abort_flag)) { ok = false; break; }
           mbar_expect_tx(bar_addr(sbase, QFULL + st), 2 * kTile);
           for (int hf = 0; hf < 2; ++hf) {
-            tma_load_4d(sbase + kQ + st * kTile + hf * kHalf, &tm_q, bar_addr(sbase, QFULL + st), hf * 64, U.h,
+            tma_load_4d(sbase + kQ + st * kTile + hf * kHalf, &tm_q, bar_addr(sbase, QFULL + st), hf * 64, hq,
                         qt * 128, U.b);
-            tma_load_4d(sbase + kDO + st * kTile + hf * kHalf, &tm_do, bar_addr(sbase, QFULL + st), hf * 64, U.h,
+            tma_load_4d(sbase + kDO + st * kTile + hf * kHalf, &tm_do, bar_addr(sbase, QFULL + st), hf * 64, hq,
                         qt * 128, U.b);
           }
           last_q_par[st] = ph;
@@ -248,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
         for (int it = 0; it < U.N && ok; ++it, ++qc) {
-          const long long pair = g_pair(U.hl, U.qlo + it, U.kt, p.nb, p.pairs_head);
+          const long long pair = g_pair(U.hl * p.grp + U.qhead(it), U.qtile(it), U.kt, p.nb, p.pairs_head);
           for (int a = 0; a < 2; ++a) {
             if (!mbar_wait(bar_addr(sbase, DSREADY + a), qc & 1, abort_flag)) {
               ok = false;
@@ -392,10 +402,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive(bar_addr(sbase, KVEMPTY));  // done reading K from shared memory
         const float Cj = rk * p.scale * kLog2e;
-        const size_t vbase = (size_t)U.bh * p.T_pad;
         float dt0 = 0.f, dt1 = 0.f;
         for (int it = 0; it < U.N; ++it, ++qc) {
-          const int qt = U.qlo + it;
+          const int qt = U.qtile(it);
+          const size_t vbase = ((size_t)U.b * p.H + U.h * p.grp + U.qhead(it)) * p.T_pad;
           const int i0 = qt * 128 + 64 * a;  // first query of this half
           // per-query vectors of this half, staged through shared memory
           const int vsel = row >> 6, vq = row & 63;
@@ -481,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Unit U = decode(p, u);
         // ------------------------------------------------------------ dK, dV epilogue
         const int j = U.kt * 128 + row;
-        const size_t orow = (((size_t)U.b * p.T + (j < p.T ? j : 0)) * p.H + U.h) * 128;
+        const size_t orow = (((size_t)U.b * p.T + (j < p.T ? j : 0)) * p.Hkv + U.h) * 128;
         const bool jv = j < p.T;
         // dk = scale (acc - coef k), coef = rk^2 (acc . k) / D, with acc . k summed by
         // the compute warpgroups as sum_i G_ij S_ij; the raw key row is loaded into

@@ -35,10 +35,11 @@ struct DqParams {
   const __nv_bfloat16* q;  // [B, T, H, 128]
   __nv_bfloat16* dq;       // [B, T, H, 128]
   int B, T, H;
+  int grp;         // query heads per K/V head: k has H / grp heads (1: multi-head)
   int w;           // left window (w >= T means full causal)
   int nq;          // query tiles per head
   int n_units;     // n_bh * nq
-  int bh0, n_bh;   // heads processed by this launch (as in the backward kernel)
+  int bh0, n_bh;   // query heads bh0 .. bh0 + n_bh - 1 (b * H + h): the groups of the backward launch's K/V heads
   int nb;          // key tiles in one query tile's band (as in the backward kernel)
   int pairs_head;  // G tiles per head
   float eps, scale;
@@ -148,8 +149,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                           (int)((2 * slot + hf) * 128));
           } else {
             for (int hf = 0; hf < 2; ++hf)
-              tma_load_4d(sbase + kK + s * kTile + hf * kHalf, &tm_k, bar_addr(sbase, full + s), hf * 64, U.h,
-                          kt * 128, U.b);
+              tma_load_4d(sbase + kK + s * kTile + hf * kHalf, &tm_k, bar_addr(sbase, full + s), hf * 64,
+                          U.h / p.grp, kt * 128, U.b);
           }
           last_par[s] = ph;
         }

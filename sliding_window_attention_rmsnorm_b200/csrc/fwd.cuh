@@ -58,8 +58,9 @@ namespace ar {
 struct FwdParams {
   __nv_bfloat16* o;  // [B, T, H, 128]
   float* lse;        // [B, H, T]
-  const float* ck;   // kCkGlobal only: [B*H, T_pad] rk_j * scale * log2(e), 0 on padding
+  const float* ck;   // kCkGlobal only: [B*Hkv, T_pad] rk_j * scale * log2(e), 0 on padding
   int B, T, H, T_pad;
+  int grp;           // query heads per K/V head: k, v have H / grp heads (1: multi-head)
   int w;             // left window (w >= T means full causal)
   int nqp;           // query-tile pairs per head = ceil(T / 256)
   int n_units;       // B * H * nqp
@@ -111,6 +112,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Unit {
   int bh, b, h;
+  int hk;  // K/V head read by query head h
   int r0[2];
   bool valid[2];
   int lo[2], hi[2];
@@ -131,6 +133,7 @@ __device__ __forceinline__ Unit decode(const FwdParams& p, int u) {
   U.bh = u % BH;
   U.b = U.bh / p.H;
   U.h = U.bh % p.H;
+  U.hk = U.h / p.grp;
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     U.r0[k] = qp * 256 + 128 * k;
@@ -248,17 +251,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(bar_addr(sbase, KEMPTY + st), ph ^ 1, abort_flag)) { ok = false; break; }
           mbar_expect_tx(bar_addr(sbase, KFULL + st), kTile);
           for (int hf = 0; hf < 2; ++hf)
-            tma_load_4d(sbase + kK + st * kTile + hf * kHalf, &tm_k, bar_addr(sbase, KFULL + st), hf * 64, U.h,
+            tma_load_4d(sbase + kK + st * kTile + hf * kHalf, &tm_k, bar_addr(sbase, KFULL + st), hf * 64, U.hk,
                         n * 128, U.b);
           last_k_par[st] = ph;
           const int vs = kv % kVStages, vph = (kv / kVStages) & 1;
           if (!mbar_wait(bar_addr(sbase, VEMPTY + vs), vph ^ 1, abort_flag)) { ok = false; break; }
           mbar_expect_tx(bar_addr(sbase, VFULL + vs), kTile + (kCkGlobal ? 512 : 0));
           for (int hf = 0; hf < 2; ++hf)
-            tma_load_4d(sbase + kV + vs * kTile + hf * kHalf, &tm_v, bar_addr(sbase, VFULL + vs), hf * 64, U.h,
+            tma_load_4d(sbase + kV + vs * kTile + hf * kHalf, &tm_v, bar_addr(sbase, VFULL + vs), hf * 64, U.hk,
                         n * 128, U.b);
           if (kCkGlobal)
-            bulk_load(sbase + kCK + vs * 512, p.ck + (size_t)U.bh * p.T_pad + n * 128, 512,
+            bulk_load(sbase + kCK + vs * 512, p.ck + ((size_t)U.b * (p.H / p.grp) + U.hk) * p.T_pad + n * 128, 512,
                       bar_addr(sbase, VFULL + vs));
           last_v_par[vs] = vph;
         }

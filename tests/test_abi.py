@@ -121,3 +121,29 @@ def test_bwd_argument_errors(L):
     assert bwd_call(L, dq=P16 + 4) == -4
     assert bwd_call(L, scale=-0.5) == -5
     assert bwd_call(L, ws=P16, ws_bytes=100) == -9
+
+
+def test_grouped_kv_head_arguments(L):
+    vp = ctypes.c_void_p
+
+    def fwd_gqa(H, Hkv, k=P16):
+        return L.ar_attn_fwd_gqa(vp(P16), vp(k), vp(P16), vp(P16), vp(P16), 1, 128, H, Hkv, 128, -1, 1e-6, 0.088,
+                                 None)
+
+    def bwd_gqa(H, Hkv, ws=None, ws_bytes=0):
+        p = vp(P16)
+        return L.ar_attn_bwd_gqa(p, p, p, p, p, p, p, p, p, 1, 128, H, Hkv, 128, -1, 1e-6, 0.088, vp(ws),
+                                 ws_bytes, None)
+
+    # Hkv must divide H and lie in 1..H; checked before anything touches a device
+    for H, Hkv in ((4, 3), (4, 0), (4, 5), (6, -2)):
+        assert fwd_gqa(H, Hkv) == -2 and bwd_gqa(H, Hkv) == -2
+        assert attn.bwd_workspace_bytes(1, 128, H, 128, Hkv) == 0
+    assert fwd_gqa(4, 2, k=P16 + 8) == -4
+    assert bwd_gqa(4, 2, ws=P16, ws_bytes=100) == -9
+    # per query head as for multi-head attention: G tiles of whole groups, here all 4 query heads
+    assert attn.bwd_workspace_bytes(1, 200, 4, 128, 2) == 3 * 4 * 256 * 4 + 4 * 3 * 32768
+    assert attn.bwd_workspace_bytes(1, 200, 4, 128, 2) == attn.bwd_workspace_bytes(1, 200, 4, 128)
+    # T = 8192: 15 query heads fit in 1 GiB of G tiles; groups of 4 round that down to 12
+    assert attn.bwd_workspace_bytes(4, 8192, 8, 128, 2) == 3 * 32 * 8192 * 4 + 12 * 2080 * 32768
+    assert attn.bwd_workspace_bytes(4, 8192, 8, 128, 8) == 3 * 32 * 8192 * 4 + 15 * 2080 * 32768

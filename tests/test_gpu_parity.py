@@ -269,3 +269,42 @@ def test_16_byte_aligned_tensors_match_aligned_ones():
     assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
     for a, b in zip(g, g_ref):
         assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------------ grouped K/V heads
+def gqa_inputs(seed, B, T, H, Hkv):
+    """q, dO with H heads and k, v with Hkv heads (seeded bf16, as for every case)."""
+    xq = synth.layer_inputs(seed, 0, B, T, H, 128)
+    xk = synth.layer_inputs(seed, 1, B, T, Hkv, 128)
+    return dict(q=xq["q"], dO=xq["dO"], k=xk["k"], v=xk["v"])
+
+
+@pytest.mark.parametrize("B,T,H,Hkv,window", [(2, 300, 4, 2, 100), (1, 256, 4, 1, -1), (1, 200, 6, 3, 0),
+                                              (2, 384, 8, 2, 200)])
+def test_grouped_kv_heads(B, T, H, Hkv, window):
+    """k, v with Hkv < H heads: query head h reads K/V head h // (H // Hkv), and
+    dk, dv sum over the group; against the fp64 oracle's grouped-head path."""
+    x = gqa_inputs(18, B, T, H, Hkv)
+    g = run_gpu(x, window)
+    assert g["dk"].shape == (B, T, Hkv, 128) and g["dv"].shape == (B, T, Hkv, 128)
+    ref = run_oracle(x, window)
+    compare(g, ref, H, tag="gqa H=%d Hkv=%d w=%d" % (H, Hkv, window), edge=True)
+
+
+def test_grouped_kv_heads_equal_duplicated_heads_on_gpu():
+    """The same K/V head repeated for each query head of a group: the grouped
+    forward is bitwise the multi-head forward (same tiles, same arithmetic), and
+    the grouped dk, dv match the group sums of the multi-head ones."""
+    B, T, H, Hkv, w = 1, 256, 4, 2, 64
+    x = gqa_inputs(19, B, T, H, Hkv)
+    xd = dict(x, k=x["k"].repeat_interleave(H // Hkv, dim=2).contiguous(),
+              v=x["v"].repeat_interleave(H // Hkv, dim=2).contiguous())
+    g, gd = run_gpu(x, w), run_gpu(xd, w)
+    assert np.array_equal(g["o"], gd["o"]) and np.array_equal(g["lse"], gd["lse"])
+    for n in ("dk", "dv"):
+        summed = gd[n].astype(np.float64).reshape(B, T, Hkv, H // Hkv, 128).sum(axis=3)
+        # the grouped result is rounded to bf16 once, each summed term once more:
+        # three roundings of at most half a bf16 ulp (2^-9 relative) each
+        err = np.abs(g[n] - summed)
+        assert (err - (MAX_ABS + 2.0 ** -7 * np.abs(summed))).max() <= 0, (n, err.max())
+        assert np.linalg.norm(g[n] - summed) / np.linalg.norm(summed) <= REL_L2
