@@ -47,6 +47,9 @@ WORKLOADS = {
                    name="long-context S layer fwd+bwd, B=2 T=8192 H=4 D=128, window 4096"),
     "long_l": dict(config=4, B=2, T=8192, H=4, n_layer=1, windows=[8192],
                    name="long-context L layer fwd+bwd, B=2 T=8192 H=4 D=128, full causal"),
+    # grouped K/V heads (n_kv_head = n_head / 2): not one of the stated workloads
+    "stack8_gqa": dict(config=3, B=8, T=2048, H=4, Hkv=2, n_layer=8, pattern="SSSL",
+                       name="8-layer SSSL attention stack fwd+bwd, B=8 T=2048 H=4 Hkv=2 D=128 (windows 1024/full)"),
 }
 
 
@@ -186,11 +189,21 @@ class ClockSampler:
 _INPUT_CACHE = {}
 
 
-def _layer_inputs_cached(wl, layer):
+def layer_host_inputs(wl, layer):
+    """Seeded bf16 CPU inputs of one layer: q, dO with H heads, k, v with Hkv."""
     from sliding_window_attention_rmsnorm_b200 import synth
-    key = (wl["config"], layer)
+    H, Hkv = wl["H"], wl.get("Hkv", wl["H"])
+    if Hkv == H:
+        return synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], H, D)
+    x = synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], H, D, roles=("q", "dO"))
+    x.update(synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], Hkv, D, roles=("k", "v")))
+    return x
+
+
+def _layer_inputs_cached(wl, layer):
+    key = (wl["config"], wl.get("Hkv"), layer)
     if key not in _INPUT_CACHE:
-        _INPUT_CACHE[key] = synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], wl["H"], D)
+        _INPUT_CACHE[key] = layer_host_inputs(wl, layer)
     return _INPUT_CACHE[key]
 
 
@@ -205,8 +218,9 @@ def oracle_sample(wl, seconds, seed_layer_offset=0):
         layer = (n + seed_layer_offset) % wl["n_layer"]
         head = (7 * n + 3) % (B * H)
         b, h = divmod(head, H)
+        hk = h // (H // wl.get("Hkv", H))  # the query head's K/V head
         x = _layer_inputs_cached(wl, layer)
-        xs = {r: t[b:b + 1, :, h:h + 1].contiguous() for r, t in x.items()}
+        xs = {r: t[b:b + 1, :, (hk if r in ("k", "v") else h):][:, :, :1].contiguous() for r, t in x.items()}
         t0 = time.perf_counter()
         orc.attn_fwd(xs["q"], xs["k"], xs["v"], ws[layer])
         orc.attn_bwd(xs["q"], xs["k"], xs["v"], xs["dO"], ws[layer])
@@ -269,7 +283,7 @@ def run_ours(args, wl, rank, world, dist):
     torch.cuda.set_device(dev)
     build.build()
     B, T, H, L = wl["B"], wl["T"], wl["H"], wl["n_layer"]
-    host = [synth.layer_inputs(wl["config"], l, B, T, H, D) for l in range(L)]
+    host = [layer_host_inputs(wl, l) for l in range(L)]
     layers = [{r: t.to("cuda", non_blocking=False) for r, t in x.items()} for x in host]
     st = stack.Stack(layers, wl.get("pattern", "SSSL"), windows=wl.get("windows"))
     windows = lib_windows(wl)
@@ -390,8 +404,10 @@ def run_ours(args, wl, rank, world, dist):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl["name"], "global_batch": B * world, "seq_len": T, "heads": H,
+                       **({"kv_heads": wl["Hkv"]} if wl.get("Hkv", H) != H else {}),
                        "layers": L, "windows": windows, "parallelism": "replicas x%d" % world,
-                       "l2": "inputs larger than L2 (%.0f MB of q,k,v,dO per step)" % (4 * L * tok * D * 2 / 1e6)},
+                       "l2": "inputs larger than L2 (%.0f MB of q,k,v,dO per step)"
+                             % (sum(t.numel() * t.element_size() for x in host for t in x.values()) / 1e6)},
             "pct_of_bf16_peak": {"sustained": value / world / peaks["bf16_sustained"],
                                  "burst": value / world / peaks["bf16_burst"], "source": peaks["source"]},
             "roofline": roof,

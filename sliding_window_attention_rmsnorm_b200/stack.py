@@ -22,7 +22,8 @@ def layer_windows(n_layer: int, seq_len: int, pattern: str = "SSSL"):
 class Stack:
     """Forward and backward of every layer, enqueued back to back on one stream.
 
-    layers: list of dicts with bf16 CUDA tensors q, k, v, dO [B, T, H, 128].
+    layers: list of dicts with bf16 CUDA tensors q, dO [B, T, H, 128] and k, v
+    [B, T, Hkv, 128] (Hkv = H, or fewer for grouped K/V heads).
     Outputs (o, lse, dq, dk, dv) and scratch are allocated once and reused.
     """
 
@@ -30,15 +31,16 @@ class Stack:
         import torch
         self.layers = layers
         B, T, H, D = layers[0]["q"].shape
+        Hkv = layers[0]["k"].shape[2]
         self.windows = list(windows) if windows is not None else layer_windows(len(layers), T, pattern)
         self.eps, self.scale = eps, scale
         dev = layers[0]["q"].device
         self.out = [dict(o=torch.empty_like(L["q"]),
                          lse=torch.empty((B, H, T), dtype=torch.float32, device=dev),
-                         dq=torch.empty_like(L["q"]), dk=torch.empty_like(L["q"]),
-                         dv=torch.empty_like(L["q"])) for L in layers]
+                         dq=torch.empty_like(L["q"]), dk=torch.empty_like(L["k"]),
+                         dv=torch.empty_like(L["v"])) for L in layers]
         self.ws_fwd = torch.empty(attn.fwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device=dev)
-        self.ws_bwd = torch.empty(attn.bwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device=dev)
+        self.ws_bwd = torch.empty(attn.bwd_workspace_bytes(B, T, H, D, Hkv), dtype=torch.uint8, device=dev)
 
     def forward(self):
         for L, O, w in zip(self.layers, self.out, self.windows):

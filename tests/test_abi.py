@@ -147,3 +147,18 @@ def test_grouped_kv_head_arguments(L):
     # T = 8192: 15 query heads fit in 1 GiB of G tiles; groups of 4 round that down to 12
     assert attn.bwd_workspace_bytes(4, 8192, 8, 128, 2) == 3 * 32 * 8192 * 4 + 12 * 2080 * 32768
     assert attn.bwd_workspace_bytes(4, 8192, 8, 128, 8) == 3 * 32 * 8192 * 4 + 15 * 2080 * 32768
+
+
+def test_stack_buffers_follow_kv_heads(L):
+    """The stack driver sizes dk, dv like k, v and its backward scratch for the
+    K/V head count (built on CPU tensors: nothing is launched here)."""
+    import torch
+    from sliding_window_attention_rmsnorm_b200 import stack
+    B, T, H, D = 1, 200, 4, 128
+    for Hkv in (4, 2, 1):
+        layer = dict(q=torch.zeros(B, T, H, D, dtype=torch.bfloat16), dO=torch.zeros(B, T, H, D, dtype=torch.bfloat16),
+                     k=torch.zeros(B, T, Hkv, D, dtype=torch.bfloat16), v=torch.zeros(B, T, Hkv, D, dtype=torch.bfloat16))
+        st = stack.Stack([layer, layer], windows=[100, 200])
+        assert st.out[0]["dk"].shape == (B, T, Hkv, D) and st.out[1]["dv"].shape == (B, T, Hkv, D)
+        assert st.out[0]["dq"].shape == (B, T, H, D) and st.out[0]["lse"].shape == (B, H, T)
+        assert st.ws_bwd.numel() == attn.bwd_workspace_bytes(B, T, H, D, Hkv) > 0
