@@ -108,20 +108,16 @@ def measured_peaks():
     return dict(bf16_burst=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
 
 
-# DRAM bytes (read + write) per launch from one ncu capture of the kernel
-# (profiles/attn_kernels_layer_s.md: S layer, B=8 T=2048 H=4), valid only while the
-# kernel's sources are byte-identical to the ones captured.
-CAPTURED_TRAFFIC = {
-    "bwd": {"bytes": 167386112,
-            "sources": {"bwd.cuh": "4f1cda0699923ec45c81c71364d9c8f0aa436e52416facee433476de96112dd2",
-                        "sm100.cuh": "cea2fd62bb5f0b803ae6ea4e5190ce97adea9f5b5598bee2001819a0a7ba2e12"}},
-    "fwd": {"bytes": 52466944,
-            "sources": {"fwd.cuh": "ecbb304d05850280362d603c41d992a6d553bd89550841fb6f32b88b8a386768",
-                        "sm100.cuh": "cea2fd62bb5f0b803ae6ea4e5190ce97adea9f5b5598bee2001819a0a7ba2e12"}},
-}
+# DRAM bytes (read + write) per launch from one ncu capture of each kernel on a
+# single layer of B=8 T=2048 H=4 (window 1024, and full causal), valid only
+# while the kernel's sources are byte-identical to the ones captured.  Keyed
+# by kernel, then by (B, T, H, window).
+CAPTURED_TRAFFIC = {}
 
 
-def captured_traffic(kind):
+def captured_traffic(kind, wl, windows):
+    """Mean DRAM bytes per launch of one kernel over the workload's layers, or
+    None when a layer shape was not captured or a source changed since."""
     import hashlib
     rec = CAPTURED_TRAFFIC.get(kind)
     if rec is None:
@@ -133,7 +129,13 @@ def captured_traffic(kind):
                 return None
         except OSError:
             return None
-    return rec["bytes"]
+    per_layer = []
+    for w in windows:
+        key = (wl["B"], wl["T"], wl["H"], w if w < wl["T"] - 1 else wl["T"])
+        if key not in rec["bytes"] or wl.get("Hkv", wl["H"]) != wl["H"]:
+            return None
+        per_layer.append(rec["bytes"][key])
+    return sum(per_layer) / len(per_layer)
 
 
 # ---------------------------------------------------------------- clocks
@@ -335,19 +337,31 @@ def run_ours(args, wl, rank, world, dist):
     value = job_tflops(world, fwd_f + bwd_f, ms)
     peaks = measured_peaks()
 
-    # roofline of the dominant kernel: counted FLOPs per launch over its event-timed mean duration
-    per_kind_flops = {"fwd": fwd_f / L, "bwd": bwd_f / L}
+    # Roofline of the dominant kernel: the counted FLOPs of its own products per
+    # launch over its event-timed mean duration.  The backward's counted work is
+    # 2.5x the forward's, five products of the forward's size; the main kernel
+    # runs four of them (S, dP, dV, dK) and the dq kernel the fifth (G K).  The
+    # per-launch events cover tens of milliseconds, so the burst peak applies.
+    per_kind_flops = {"fwd": fwd_f / L, "bwd": bwd_f / L * 4 / 5, "dq": bwd_f / L / 5}
     dom = max(("fwd", "bwd"), key=lambda k: kern[k][0])
     tot_ms, n_launch = kern[dom]
     achieved = (per_kind_flops[dom] * n_launch) / (tot_ms * 1e-3) / 1e12
-    roof = {"kernel": dom + "_kernel", "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_sustained"],
-            "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"], "traffic": captured_traffic(dom),
-            "peak_kind": "bf16 sustained (%s)" % peaks["source"]}
+    roof = {"kernel": dom + "_kernel", "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_burst"],
+            "unit": "TFLOP/s", "frac": achieved / peaks["bf16_burst"],
+            "traffic": captured_traffic(dom, wl, windows),
+            "peak_kind": "bf16 burst (%s)" % peaks["source"],
+            "flops_per_launch": per_kind_flops[dom]}
     kernels = {k: {"ms_per_launch": (v[0] / v[1]) if v[1] else None, "launches": v[1],
                    "share": v[0] / max(1e-9, sum(x[0] for x in kern.values()))} for k, v in kern.items()}
-    for k in ("fwd", "bwd"):
+    for k in ("fwd", "bwd", "dq"):
         if kern[k][1]:
             kernels[k]["tflops"] = per_kind_flops[k] * kern[k][1] / (kern[k][0] * 1e-3) / 1e12
+            kernels[k]["frac_of_burst"] = kernels[k]["tflops"] / peaks["bf16_burst"]
+            kernels[k]["traffic"] = captured_traffic(k, wl, windows)
+    if kern["bwd"][1] and kern["dq"][1]:  # the whole backward's products over both kernels' time
+        t = (kern["bwd"][0] + kern["dq"][0]) * 1e-3
+        kernels["bwd+dq"] = {"tflops": bwd_f * kern["bwd"][1] / L / t / 1e12}
+        kernels["bwd+dq"]["frac_of_burst"] = kernels["bwd+dq"]["tflops"] / peaks["bf16_burst"]
     # memory-bound helpers: algorithmic bytes per launch
     tok = B * T * H
     # the dq kernel reads one 32 KB G tile per (query tile, key tile) pair of the band

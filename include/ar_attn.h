@@ -32,7 +32,7 @@
  *     abort crosses the ABI.  Argument errors are detected before any work is
  *     enqueued.  A device-side wait that gives up (AR_ERR_TIMEOUT) is reported
  *     by ar_attn_sync_status().
- *   - Workspace (ar_attn_bwd; the forward needs none): if `workspace` is NULL
+ *   - Workspace (ar_attn_bwd only; the forward needs none): if `workspace` is NULL
  *     the library allocates it stream-ordered (cudaMallocAsync / cudaFreeAsync
  *     on `stream`); otherwise it must hold at least the bytes returned by
  *     ar_attn_bwd_workspace_bytes() and be 256-byte aligned.  It is scratch:
@@ -62,20 +62,22 @@ enum {
   AR_ERR_LAYOUT = -11      /* a kernel found its shared memory misaligned and did not run (sync_status) */
 };
 
-/* Bytes of scratch ar_attn_fwd needs: always 0.  The fused forward kernel
- * derives the per-key norm factors from each K tile it loads, so it needs no
- * scratch; the workspace arguments of ar_attn_fwd are accepted and ignored. */
-size_t ar_attn_fwd_workspace_bytes(int B, int T, int H, int D);
-
 /* Forward pass.  Inputs q, k, v; outputs o [B,T,H,D] bf16 and lse [B,H,T] fp32
- * (lse is what ar_attn_bwd needs).  One fused kernel on `stream`; allocates
- * nothing.  `workspace` and `workspace_bytes` are ignored (may be NULL / 0). */
+ * (lse is what ar_attn_bwd needs).  The operation is the one at the top of
+ * this file: norm(q), norm(k) as in the "autoresearch" README (gitee), section
+ * 7.3 "CausalSelfAttention", then the windowed causal attention of its sections
+ * 5.2.1-5.2.2 (FlashAttention-3, window_size = (window, 0)).  One fused kernel
+ * on `stream`; allocates nothing and needs no scratch (the per-key norm
+ * factors are derived from each K tile inside the kernel).
+ * lse may be NULL: the kernel then does not store it.  That is the
+ * forward-only use (the README's section 9.4 "evaluate_bpb" runs the model
+ * without gradients), and o is identical either way. */
 int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
-                int B, int T, int H, int D, int window, float eps, float scale,
-                void* workspace, size_t workspace_bytes, void* stream);
+                int B, int T, int H, int D, int window, float eps, float scale, void* stream);
 
-/* Bytes of scratch ar_attn_bwd needs: three fp32 per-(b, h, t) vectors (rounded
- * up to whole 128-token tiles) plus a buffer of bf16 128x128 tiles G^T, one per
+/* Bytes of scratch ar_attn_bwd needs (the pages do not describe the backward's
+ * storage; this is this library's layout): three fp32 per-(b, h, t) vectors
+ * (rounded up to whole 128-token tiles) plus a buffer of bf16 128x128 tiles G^T, one per
  * (query tile, key tile) pair of the causal band of a group of heads: for
  * nq = ceil(T/128), nq(nq+1)/2 tiles of 32 KB per head, for as many heads as
  * fit in 1 GiB (at least one, at most B*H); larger problems are processed in
@@ -83,8 +85,14 @@ int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
  * sizes. */
 size_t ar_attn_bwd_workspace_bytes(int B, int T, int H, int D);
 
-/* Backward pass.  Inputs q, k, v, the forward's o and lse, and the upstream
- * gradient dO; outputs dq, dk, dv [B,T,H,D] bf16 (overwritten, not added to).
+/* Backward pass: the exact gradient of ar_attn_fwd's o with respect to q, k
+ * and v, through the attention and through both RMSNorms.  The pages' training
+ * loop runs a forward and a backward pass every step ("autoresearch" README
+ * (gitee), section 5.1, the outline of train.py's training loop), through
+ * FlashAttention-3's backward (section 5.2.1); the gradient itself is the
+ * standard softmax-attention one, with delta = rowsum(dO * o).  Inputs q, k,
+ * v, the forward's o and lse, and the upstream gradient dO; outputs dq, dk, dv
+ * [B,T,H,D] bf16 (overwritten, not added to).
  * window, eps and scale must be the forward's.  Launches, on `stream`: the
  * pre-pass (delta = rowsum(dO * o), 1/rms(q), lse * log2 e), then per head
  * group the fused backward kernel (dk, dv, and the bf16 tiles G = dS rq rk
@@ -116,20 +124,37 @@ int ar_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, 
 
 /* Synchronises `stream`, then reads and clears this device's status word.
  * Returns AR_OK, AR_ERR_TIMEOUT if a kernel abandoned a wait since the last
- * call, or AR_ERR_CUDA if the synchronisation itself failed. */
+ * call, AR_ERR_LAYOUT if a kernel refused to run, or AR_ERR_CUDA if the
+ * synchronisation itself failed.  The pages' own failure handling is at the
+ * level of whole runs (the "autoresearch" README (gitee), section 6.3: a run
+ * over its time budget is killed and logged as a crash); this is the library's
+ * counterpart for one call: no kernel waits forever. */
 int ar_attn_sync_status(void* stream);
+
+/* Limit, in nanoseconds, of every device-side wait inside the kernels launched
+ * after this call (process-wide; 0 restores the default of 2 s).  A kernel
+ * whose wait runs out abandons its work, leaves its outputs unspecified and
+ * sets AR_ERR_TIMEOUT for ar_attn_sync_status; the waits that let copies and
+ * tensor-core work in flight finish before a CTA exits keep the default limit.
+ * Meant for failure-detection tests; a limit far below a kernel's run time
+ * makes every call time out.  Returns AR_OK. */
+int ar_attn_set_wait_limit_ns(unsigned long long ns);
 
 /* Static, human-readable text for a status code (never NULL). */
 const char* ar_attn_strerror(int status);
 
 /* Window of layer `layer` in a stack of n_layer layers following `pattern`
  * (characters 'S' and 'L', case-insensitive; layer l uses pattern[l mod len]):
- * 'L' -> seq_len, 'S' -> seq_len / 2, and the last layer always seq_len.
+ * 'L' -> seq_len, 'S' -> seq_len / 2, and the last layer always seq_len
+ * ("autoresearch" README (gitee), section 5.2.2, the "SSSL" window pattern;
+ * web3.okx.com review, paragraph on the window pattern).
  * Returns a negative AR_ERR_* code on invalid arguments. */
 int ar_attn_layer_window(int layer, int n_layer, int seq_len, const char* pattern);
 
 /* Number of visible (query, key) pairs of one head: sum_i (min(i, w) + 1),
- * w = window as above.  Used to count the FLOPs the attention really does. */
+ * w = window as above.  Used to count the FLOPs the attention really does
+ * (the pages count attention work per visible key: the xyutech.top run log's
+ * FLOPs-per-token figure). */
 long long ar_attn_unmasked_pairs(int T, int window);
 
 /* Kernel timing for measurement.  Kernel kinds, in launch order: */
@@ -154,12 +179,11 @@ int ar_attn_timing_enable(int on);
 int ar_attn_timing_read(double* ms, long long* count);
 
 /* Forward pass that allocates nothing, for callers that cannot call
- * cudaMalloc: code running inside a CUDA-graph capture that must not allocate,
- * plug-ins whose host application owns the device allocator, or real-time loops
- * that forbid allocation after start-up.  It computes what ar_attn_fwd computes
- * (same arguments minus the workspace) in two launches: a pre-pass writes the
+ * cudaMalloc: plug-ins whose host application owns the device allocator, or
+ * real-time loops that forbid allocation after start-up.  It computes what
+ * ar_attn_fwd computes (same arguments) in two launches: a pre-pass writes the
  * per-key norm factors into a fixed array compiled into the library, and the
- * forward kernel reads them from there.  (ar_attn_fwd itself now derives the
+ * forward kernel reads them from there.  (ar_attn_fwd itself derives the
  * factors inside its kernel and allocates nothing either; this entry point
  * keeps the two-launch form and its contract.)
  * There is no counterpart to this entry point on the reference pages.

@@ -41,11 +41,9 @@ def lib():
                           % LIB_PATH)
         L = ctypes.CDLL(LIB_PATH)
         vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
-        L.ar_attn_fwd_workspace_bytes.argtypes = [i, i, i, i]
-        L.ar_attn_fwd_workspace_bytes.restype = sz
         L.ar_attn_bwd_workspace_bytes.argtypes = [i, i, i, i]
         L.ar_attn_bwd_workspace_bytes.restype = sz
-        L.ar_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, vp, sz, vp]
+        L.ar_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, vp]
         L.ar_attn_fwd.restype = i
         L.ar_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, f, vp, sz, vp]
         L.ar_attn_bwd.restype = i
@@ -67,6 +65,10 @@ def lib():
         L.ar_attn_bwd_gqa_workspace_bytes.restype = sz
         L.ar_attn_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, vp, sz, vp]
         L.ar_attn_bwd_gqa.restype = i
+        L.ar_attn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+        L.ar_attn_set_wait_limit_ns.restype = i
+        L.ar_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, vp]
+        L.ar_attn_fwd_noalloc.restype = i
         _lib = L
     return _lib
 
@@ -111,39 +113,54 @@ def default_scale(D: int) -> float:
     return 1.0 / math.sqrt(D)
 
 
-def fwd_workspace_bytes(B, T, H, D) -> int:
-    return int(lib().ar_attn_fwd_workspace_bytes(B, T, H, D))
-
-
 def bwd_workspace_bytes(B, T, H, D, Hkv=None) -> int:
     if Hkv is None or Hkv == H:
         return int(lib().ar_attn_bwd_workspace_bytes(B, T, H, D))
     return int(lib().ar_attn_bwd_gqa_workspace_bytes(B, T, H, Hkv, D))
 
 
-def fwd(q, k, v, window: int, eps: float = 1e-6, scale=None, out=None, lse=None, workspace=None):
+def _check_out(t, like, name):
+    """A caller-supplied output must match the tensor it is shaped after."""
+    if not (t.is_cuda and t.dtype == like.dtype and t.is_contiguous() and tuple(t.shape) == tuple(like.shape)
+            and t.device == like.device):
+        raise ValueError("%s must be a contiguous %s CUDA tensor of shape %s" % (name, like.dtype, tuple(like.shape)))
+
+
+def _check_lse(t, B, H, T, device):
+    if not (t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and tuple(t.shape) == (B, H, T)
+            and t.device == device):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, H, T]")
+
+
+def fwd(q, k, v, window: int, eps: float = 1e-6, scale=None, out=None, lse=None, need_lse: bool = True):
     """o, lse = attention(norm(q), norm(k), v) over the band 0 <= i - j <= window.
 
     q: bf16 CUDA tensor [B, T, H, 128]; k, v: [B, T, Hkv, 128] with Hkv
     dividing H (Hkv < H: grouped K/V heads, query head h reads K/V head
     h // (H // Hkv)).  Returns o (bf16, like q) and lse (fp32 [B, H, T]).
+    need_lse=False is the forward-only use (no backward follows): the kernel
+    does not store lse and None is returned in its place; o is unchanged.
     Enqueued on torch's current stream.
     """
     Hkv = _check_qkv(q, k, v)
     B, T, H, D = q.shape
     if scale is None:
         scale = default_scale(D)
+    if out is not None:
+        _check_out(out, q, "out")
     o = torch.empty_like(q) if out is None else out
-    lse_t = torch.empty((B, H, T), dtype=torch.float32, device=q.device) if lse is None else lse
+    if need_lse:
+        lse_t = torch.empty((B, H, T), dtype=torch.float32, device=q.device) if lse is None else lse
+        _check_lse(lse_t, B, H, T, q.device)
+    else:
+        lse_t = None
     if Hkv != H:
         st = lib().ar_attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, T, H, Hkv, D, int(window),
                                    float(eps), float(scale), _stream())
         _check(st, "ar_attn_fwd_gqa")
         return o, lse_t
-    if workspace is None:
-        workspace = torch.empty(max(fwd_workspace_bytes(B, T, H, D), 1), dtype=torch.uint8, device=q.device)
     st = lib().ar_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, T, H, D, int(window),
-                           float(eps), float(scale), _ptr(workspace), workspace.numel(), _stream())
+                           float(eps), float(scale), _stream())
     _check(st, "ar_attn_fwd")
     return o, lse_t
 
@@ -158,10 +175,12 @@ def bwd(q, k, v, o, dO, lse, window: int, eps: float = 1e-6, scale=None, dq=None
     Hkv = _check_qkv(q, k, v)
     _check_inputs(q, o, dO)
     B, T, H, D = q.shape
-    if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, H, T)):
-        raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, H, T]")
+    _check_lse(lse, B, H, T, q.device)
     if scale is None:
         scale = default_scale(D)
+    for t, like, name in ((dq, q, "dq"), (dk, k, "dk"), (dv, v, "dv")):
+        if t is not None:
+            _check_out(t, like, name)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -183,6 +202,13 @@ def bwd(q, k, v, o, dO, lse, window: int, eps: float = 1e-6, scale=None, dq=None
 def sync_status():
     """Synchronise the current stream and raise if a kernel gave up a wait."""
     _check(lib().ar_attn_sync_status(_stream()), "ar_attn_sync_status")
+
+
+def set_wait_limit_ns(ns: int = 0):
+    """Limit of every device-side wait in kernels launched from now on (0: the
+    default, 2 s).  A kernel whose wait runs out abandons its work and
+    sync_status() raises AR_ERR_TIMEOUT; for failure-detection tests."""
+    _check(lib().ar_attn_set_wait_limit_ns(int(ns)), "ar_attn_set_wait_limit_ns")
 
 
 def unmasked_pairs(T: int, window: int) -> int:
@@ -211,8 +237,8 @@ NOALLOC_MAX_KEYS = 1 << 20
 def fwd_noalloc(q, k, v, window: int, eps: float = 1e-6, scale=None, out=None, lse=None):
     """The forward through ar_attn_fwd_noalloc: no workspace is allocated.
 
-    For callers that must not allocate device memory (inside a graph capture,
-    under a host-owned allocator).  Scratch is the library's built-in array, so
+    For callers that must not allocate device memory (a host application that
+    owns the allocator).  Scratch is the library's built-in array, so
     B * H * ceil(T/128)*128 must not exceed NOALLOC_MAX_KEYS, and calls that
     can overlap on the GPU must be serialised by the caller.  The outputs o and
     lse may be passed in (out, lse) so that nothing at all is allocated here.
@@ -221,13 +247,12 @@ def fwd_noalloc(q, k, v, window: int, eps: float = 1e-6, scale=None, out=None, l
     B, T, H, D = q.shape
     if scale is None:
         scale = default_scale(D)
+    if out is not None:
+        _check_out(out, q, "out")
     o = torch.empty_like(q) if out is None else out
     lse_t = torch.empty((B, H, T), dtype=torch.float32, device=q.device) if lse is None else lse
-    L = lib()
-    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
-    L.ar_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, vp]
-    L.ar_attn_fwd_noalloc.restype = i
-    st = L.ar_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, T, H, D, int(window),
+    _check_lse(lse_t, B, H, T, q.device)
+    st = lib().ar_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, T, H, D, int(window),
                                float(eps), float(scale), _stream())
     _check(st, "ar_attn_fwd_noalloc")
     return o, lse_t

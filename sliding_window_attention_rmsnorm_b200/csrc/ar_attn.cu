@@ -11,6 +11,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -33,6 +34,8 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+// Limit of every device-side wait in the kernels launched from now on.
+std::atomic<unsigned long long> g_wait_ns{ar::kWaitLimitNs};
 
 // Checks the current device once: compute capability 10.0, kernel attributes.
 using FwdKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, ar::FwdParams);
@@ -70,9 +73,10 @@ int device_setup(int* sms_out) {
       d.status = AR_ERR_CUDA;
     }
     if (d.status == AR_OK) {
-      // The kernels move registers between warpgroups with setmaxnreg; the split
-      // is sized for exactly 168 registers per thread at launch, so refuse any
-      // other build rather than launch a kernel whose register raise cannot be met.
+      // The forward moves registers between warpgroups with setmaxnreg; its split
+      // is sized for exactly ar::fwd::kLaunchRegs registers per thread at launch,
+      // so refuse any other build rather than launch a kernel whose register raise
+      // cannot be met.  The backward kernel is checked for its own budget.
       if (!fwd_regs_ok(ar::fwd::fwd_kernel<true, false>) || !fwd_regs_ok(ar::fwd::fwd_kernel<false, false>) ||
           !fwd_regs_ok(ar::fwd::fwd_kernel<true, true>) || !fwd_regs_ok(ar::fwd::fwd_kernel<false, true>))
         d.status = AR_ERR_CUDA;
@@ -155,6 +159,7 @@ ar::FwdParams fwd_params(void* o, float* lse, const float* ck, int B, int T, int
   p.bound = scale * 128.0f * 1.4426950408889634f;
   p.cscale = scale * 1.4426950408889634f;
   p.wide = aligned(o, 32);
+  p.wait_ns = g_wait_ns.load();
   return p;
 }
 
@@ -275,11 +280,6 @@ int prep_grid(long long rows, int sms) {
 
 extern "C" {
 
-size_t ar_attn_fwd_workspace_bytes(int B, int T, int H, int D) {
-  (void)B, (void)T, (void)H, (void)D;
-  return 0;  // the forward kernel derives the per-key norm factors itself
-}
-
 size_t ar_attn_bwd_gqa_workspace_bytes(int B, int T, int H, int Hkv, int D) {
   if (check_shape(B, T, H, D) != AR_OK || check_kv_heads(H, Hkv) != AR_OK) return 0;
   return 3 * vec_bytes(B, T, H) + g_heads_cap(B, T, H, H / Hkv) * g_head_bytes(T, (T + 127) / 128);
@@ -289,7 +289,7 @@ size_t ar_attn_bwd_workspace_bytes(int B, int T, int H, int D) { return ar_attn_
 
 int ar_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T, int H, int Hkv,
                     int D, int window, float eps, float scale, void* stream) {
-  if (!q || !k || !v || !o || !lse) return AR_ERR_NULL;
+  if (!q || !k || !v || !o) return AR_ERR_NULL;  // lse may be NULL: not stored
   int st = check_shape(B, T, H, D);
   if (st != AR_OK) return st;
   if ((st = check_kv_heads(H, Hkv)) != AR_OK) return st;
@@ -315,8 +315,7 @@ int ar_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float*
 }
 
 int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T, int H, int D,
-                int window, float eps, float scale, void* workspace, size_t workspace_bytes, void* stream) {
-  (void)workspace, (void)workspace_bytes;  // no scratch needed: see ar_attn_fwd_workspace_bytes
+                int window, float eps, float scale, void* stream) {
   return ar_attn_fwd_gqa(q, k, v, o, lse, B, T, H, H, D, window, eps, scale, stream);
 }
 
@@ -403,6 +402,7 @@ int ar_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, 
     p.scale = scale;
     p.wide = aligned(dk, 32) && aligned(dv, 32);
     p.wide_k = aligned(k, 32);
+    p.wait_ns = g_wait_ns.load();
     {
       KernelTimer t(AR_KERNEL_BWD, s);
       ar::bwd::bwd_kernel<<<std::min(p.n_units, sms), ar::bwd::kThreads, ar::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo,
@@ -427,6 +427,7 @@ int ar_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, 
     d.scale = scale;
     d.wide = aligned(dq, 32);
     d.wide_q = aligned(q, 32);
+    d.wait_ns = p.wait_ns;
     {
       KernelTimer t(AR_KERNEL_DQ, s);
       ar::dqk::dq_kernel<<<std::min(d.n_units, sms), ar::dqk::kThreads, ar::dqk::kSmemBytes, s>>>(tg, tk, d);
@@ -484,6 +485,11 @@ int ar_attn_layer_window(int layer, int n_layer, int seq_len, const char* patter
   if (c == 'L') return seq_len;
   if (c == 'S') return seq_len / 2;
   return AR_ERR_ARG;
+}
+
+int ar_attn_set_wait_limit_ns(unsigned long long ns) {
+  g_wait_ns.store(ns == 0 ? ar::kWaitLimitNs : ns);
+  return AR_OK;
 }
 
 int ar_attn_timing_enable(int on) {
@@ -567,7 +573,7 @@ int noalloc_scratch(float** out) {
 
 extern "C" int ar_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T,
                                    int H, int D, int window, float eps, float scale, void* stream) {
-  if (!q || !k || !v || !o || !lse) return AR_ERR_NULL;
+  if (!q || !k || !v || !o) return AR_ERR_NULL;  // lse may be NULL: not stored
   int st = check_shape(B, T, H, D);
   if (st != AR_OK) return st;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))

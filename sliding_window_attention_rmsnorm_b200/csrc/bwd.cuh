@@ -59,6 +59,7 @@ struct BwdParams {
   float eps, scale;
   int wide;    // dk and dv are 32-byte aligned: rows are written with 256-bit stores
   int wide_k;  // k is 32-byte aligned: key rows are read with 256-bit loads
+  unsigned long long wait_ns;  // limit of a device-side wait (kWaitLimitNs unless set otherwise)
 };
 
 // Slot of the G tile of (query tile qt, key tile kt) of the launch's query head
@@ -218,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = unit_index(cta, r, G);
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
-        if (uidx > 0 && !mbar_wait(bar_addr(sbase, KVEMPTY), (uidx - 1) & 1, abort_flag)) break;
+        if (uidx > 0 && !mbar_wait(bar_addr(sbase, KVEMPTY), (uidx - 1) & 1, abort_flag, p.wait_ns)) break;
         mbar_expect_tx(bar_addr(sbase, KVFULL), 2 * kTile);
         for (int hf = 0; hf < 2; ++hf) {
           tma_load_4d(sbase + kK + hf * kHalf, &tm_k, bar_addr(sbase, KVFULL), hf * 64, U.h, U.kt * 128, U.b);
@@ -228,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int it = 0; it < U.N; ++it, ++qc) {
           const int qt = U.qtile(it), hq = U.h * p.grp + U.qhead(it);
           const int st = qc & 1, ph = (qc >> 1) & 1;
-          if (!mbar_wait(bar_addr(sbase, QEMPTY + st), ph ^ 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(bar_addr(sbase, QEMPTY + st), ph ^ 1, abort_flag, p.wait_ns)) { ok = false; break; }
           mbar_expect_tx(bar_addr(sbase, QFULL + st), 2 * kTile);
           for (int hf = 0; hf < 2; ++hf) {
             tma_load_4d(sbase + kQ + st * kTile + hf * kHalf, &tm_q, bar_addr(sbase, QFULL + st), hf * 64, hq,
@@ -240,11 +241,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++uidx;
       }
-      if (*abort_flag) {
-        volatile int never = 0;
-        if (last_kv_par >= 0) mbar_wait(bar_addr(sbase, KVFULL), last_kv_par, &never);
+      {
+        // Every exit, normal or aborted: the copies still in flight land before
+        // the CTA's shared memory goes away (on the normal path they have landed).
+        if (last_kv_par >= 0) mbar_drain(bar_addr(sbase, KVFULL), last_kv_par);
         for (int s = 0; s < 2; ++s)
-          if (last_q_par[s] >= 0) mbar_wait(bar_addr(sbase, QFULL + s), last_q_par[s], &never);
+          if (last_q_par[s] >= 0) mbar_drain(bar_addr(sbase, QFULL + s), last_q_par[s]);
       }
     } else if (warp == 14 && lane == 0) {
       // ---------------------------------------------------------- G^T stores
@@ -260,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int it = 0; it < U.N && ok; ++it, ++qc) {
           const long long pair = g_pair(U.hl * p.grp + U.qhead(it), U.qtile(it), U.kt, p.nb, p.pairs_head);
           for (int a = 0; a < 2; ++a) {
-            if (!mbar_wait(bar_addr(sbase, DSREADY + a), qc & 1, abort_flag)) {
+            if (!mbar_wait(bar_addr(sbase, DSREADY + a), qc & 1, abort_flag, p.wait_ns)) {
               ok = false;
               break;
             }
@@ -315,10 +317,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = unit_index(cta, r, G);
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
-        if (!mbar_wait(bar_addr(sbase, KVFULL), uidx & 1, abort_flag)) break;
+        if (!mbar_wait(bar_addr(sbase, KVFULL), uidx & 1, abort_flag, p.wait_ns)) break;
         {  // prologue: S and dP of both halves of the first tile
           const int st = qc & 1, ph = (qc >> 1) & 1;
-          if (!mbar_wait(bar_addr(sbase, QFULL + st), ph, abort_flag)) break;
+          if (!mbar_wait(bar_addr(sbase, QFULL + st), ph, abort_flag, p.wait_ns)) break;
 #pragma unroll
           for (int a = 0; a < 2; ++a) {
             tc_fence_after();
@@ -337,15 +339,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool has_next = it + 1 < U.N;
 #pragma unroll
           for (int a = 0; a < 2; ++a) {
-            if (!mbar_wait(bar_addr(sbase, DSREADY + a), q & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(bar_addr(sbase, DSREADY + a), q & 1, abort_flag, p.wait_ns)) { ok = false; break; }
             if (it == 0 && a == 0 && uidx > 0 &&
-                !mbar_wait(bar_addr(sbase, ACCFREE), (uidx - 1) & 1, abort_flag)) { ok = false; break; }
+                !mbar_wait(bar_addr(sbase, ACCFREE), (uidx - 1) & 1, abort_flag, p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             issue_grad(a, st, it == 0 && a == 0);
             mma_commit(bar_addr(sbase, DSFREE + a));
             if (a == 1) mma_commit(bar_addr(sbase, QEMPTY + st));
             if (has_next) {
-              if (a == 0 && !mbar_wait(bar_addr(sbase, QFULL + st1), ph1, abort_flag)) { ok = false; break; }
+              if (a == 0 && !mbar_wait(bar_addr(sbase, QFULL + st1), ph1, abort_flag, p.wait_ns)) { ok = false; break; }
               tc_fence_after();
               issue_dp(a, st1);
               issue_s(a, st1);
@@ -360,8 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++uidx;
       }
       mma_commit(bar_addr(sbase, FINAL));
-      volatile int never = 0;
-      mbar_wait(bar_addr(sbase, FINAL), 0, &never);
+      mbar_drain(bar_addr(sbase, FINAL), 0);
     }
   } else {
     if (warp < 8) {
@@ -381,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
         const int j = U.kt * 128 + row;
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, KVFULL), uidx & 1, abort_flag))) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, KVFULL), uidx & 1, abort_flag, p.wait_ns))) break;
         float rk;
         {
           float ss[4] = {0.f, 0.f, 0.f, 0.f};
@@ -412,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float v0 = vsel == 0 ? p.lse2[vbase + i0 + vq] : p.rq[vbase + i0 + vq];
           const float v1 = vsel == 0 ? p.delta[vbase + i0 + vq] : 0.f;
           if (qc > 0 &&
-              !__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VECEMPTY + a), (qc - 1) & 1, abort_flag))) {
+              !__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VECEMPTY + a), (qc - 1) & 1, abort_flag, p.wait_ns))) {
             ok = false;
             break;
           }
@@ -423,16 +424,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             sts_f32(vaddr + 512 + 4 * vq, v0);
           }
           mbar_arrive(bar_addr(sbase, VECFULL + a));
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VECFULL + a), qc & 1, abort_flag))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VECFULL + a), qc & 1, abort_flag, p.wait_ns))) {
             ok = false;
             break;
           }
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, SFULL + a), qc & 1, abort_flag))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, SFULL + a), qc & 1, abort_flag, p.wait_ns))) {
             ok = false;
             break;
           }
           if (qc > 0 &&
-              !__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DSFREE + a), (qc - 1) & 1, abort_flag))) {
+              !__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DSFREE + a), (qc - 1) & 1, abort_flag, p.wait_ns))) {
             ok = false;
             break;
           }
@@ -464,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // DSREADY (so the epilogue's wait for the final products covers it) and
             // once the epilogue has taken the previous unit's (DOTFREE)
             if (uidx > 0 &&
-                !__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DOTFREE), (uidx - 1) & 1, abort_flag))) {
+                !__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DOTFREE), (uidx - 1) & 1, abort_flag, p.wait_ns))) {
               ok = false;
               break;
             }
@@ -510,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DKDVDONE), uidx & 1, abort_flag))) break;
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DKDVDONE), uidx & 1, abort_flag, p.wait_ns))) break;
           tc_fence_after();
           const float coef = lds_f32(sbase + kDot + 4 * row) + lds_f32(sbase + kDot + 4 * (128 + row));
           mbar_arrive(bar_addr(sbase, DOTFREE));

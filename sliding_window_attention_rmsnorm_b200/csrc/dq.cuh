@@ -45,6 +45,7 @@ struct DqParams {
   float eps, scale;
   int wide;        // dq is 32-byte aligned: rows are written with 256-bit stores
   int wide_q;      // q is 32-byte aligned: query rows are read with 256-bit loads
+  unsigned long long wait_ns;  // limit of a device-side wait (kWaitLimitNs unless set otherwise)
 };
 
 namespace dqk {
@@ -137,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Unit U = decode(p, u);
         for (int kt = U.hi; kt >= U.lo; --kt, ++c) {
           const int s = c % nst, ph = (c / nst) & 1;
-          if (!mbar_wait(bar_addr(sbase, empty + s), ph ^ 1, abort_flag)) {
+          if (!mbar_wait(bar_addr(sbase, empty + s), ph ^ 1, abort_flag, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -155,10 +156,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           last_par[s] = ph;
         }
       }
-      if (*abort_flag) {
-        volatile int never = 0;
+      {
+        // Every exit, normal or aborted: the copies still in flight land before
+        // the CTA's shared memory goes away (on the normal path they have landed).
         for (int s = 0; s < nst; ++s)
-          if (last_par[s] >= 0) mbar_wait(bar_addr(sbase, full + s), last_par[s], &never);
+          if (last_par[s] >= 0) mbar_drain(bar_addr(sbase, full + s), last_par[s]);
       }
     }
   } else if (warp == 5) {
@@ -174,12 +176,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
         const int ab = uidx % kAcc;
-        if (uidx >= kAcc && !mbar_wait(bar_addr(sbase, ACCFREE + ab), (uidx / kAcc - 1) & 1, abort_flag)) break;
+        if (uidx >= kAcc && !mbar_wait(bar_addr(sbase, ACCFREE + ab), (uidx / kAcc - 1) & 1, abort_flag, p.wait_ns)) break;
         for (int kt = U.hi; kt >= U.lo; --kt, ++ck, ++cg) {
           const int ks = ck % kKStages, kph = (ck / kKStages) & 1;
           const int gs = cg % kGStages, gph = (cg / kGStages) & 1;
-          if (!mbar_wait(bar_addr(sbase, KFULL + ks), kph, abort_flag) ||
-              !mbar_wait(bar_addr(sbase, GFULL + gs), gph, abort_flag)) {
+          if (!mbar_wait(bar_addr(sbase, KFULL + ks), kph, abort_flag, p.wait_ns) ||
+              !mbar_wait(bar_addr(sbase, GFULL + gs), gph, abort_flag, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -196,8 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++uidx;
       }
       mma_commit(bar_addr(sbase, FINAL));
-      volatile int never = 0;
-      mbar_wait(bar_addr(sbase, FINAL), 0, &never);
+      mbar_drain(bar_addr(sbase, FINAL), 0);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -229,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, ACCFULL + ab), (uidx / kAcc) & 1, abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, ACCFULL + ab), (uidx / kAcc) & 1, abort_flag, p.wait_ns))) {
           ok = false;
           break;
         }

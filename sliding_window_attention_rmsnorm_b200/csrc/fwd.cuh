@@ -57,7 +57,7 @@ namespace ar {
 
 struct FwdParams {
   __nv_bfloat16* o;  // [B, T, H, 128]
-  float* lse;        // [B, H, T]
+  float* lse;        // [B, H, T], or NULL: not stored (forward-only use)
   const float* ck;   // kCkGlobal only: [B*Hkv, T_pad] rk_j * scale * log2(e), 0 on padding
   int B, T, H, T_pad;
   int grp;           // query heads per K/V head: k, v have H / grp heads (1: multi-head)
@@ -68,6 +68,7 @@ struct FwdParams {
   float bound;       // scale * D * log2(e): the largest |logit| in log2 units
   float cscale;      // scale * log2(e)
   int wide;          // o is 32-byte aligned: rows are written with 256-bit stores
+  unsigned long long wait_ns;  // limit of a device-side wait (kWaitLimitNs unless set otherwise)
 };
 
 namespace fwd {
@@ -89,9 +90,6 @@ constexpr int kKStages = 3, kVStages = 2;
 // issued after both softmax warpgroups finished tile n - kKStages - 1.
 constexpr int kCkSlots = kKStages + 1;
 constexpr uint32_t kQ = 0, kK = 2 * kTile, kV = kK + kKStages * kTile, kCK = kV + kVStages * kTile;
-// Of every 4 pairs of softmax exponentials, this many are computed on the FMA
-// pipe (exp2_fma2) and the rest on the MUFU unit.
-constexpr int kEmuPairsOf4 = 0;
 // Largest logit bound (log2 units) for which the fixed softmax offset is used:
 // p >= 2^-64 stays a normal number in fp32 and bf16.
 constexpr float kFixedBoundMax = 32.0f;
@@ -204,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int it = 0; it < U.N; ++it, ++kv) {
           const int n = U.hi_u - it;
           const int st = kv % kKStages, ph = (kv / kKStages) & 1;
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, KFULL + st), ph, abort_flag))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, KFULL + st), ph, abort_flag, p.wait_ns))) {
             ok = false;
             break;
           }
@@ -237,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = unit_index(cta, r, G);
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
-        if (uidx > 0 && !mbar_wait(bar_addr(sbase, QEMPTY), (uidx - 1) & 1, abort_flag)) break;
+        if (uidx > 0 && !mbar_wait(bar_addr(sbase, QEMPTY), (uidx - 1) & 1, abort_flag, p.wait_ns)) break;
         mbar_expect_tx(bar_addr(sbase, QFULL), kTile * (U.valid[1] ? 2 : 1));
         for (int k = 0; k < 2; ++k)
           if (U.valid[k])
@@ -248,14 +246,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int it = 0; it < U.N; ++it, ++kv) {
           const int n = U.hi_u - it;
           const int st = kv % kKStages, ph = (kv / kKStages) & 1;
-          if (!mbar_wait(bar_addr(sbase, KEMPTY + st), ph ^ 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(bar_addr(sbase, KEMPTY + st), ph ^ 1, abort_flag, p.wait_ns)) { ok = false; break; }
           mbar_expect_tx(bar_addr(sbase, KFULL + st), kTile);
           for (int hf = 0; hf < 2; ++hf)
             tma_load_4d(sbase + kK + st * kTile + hf * kHalf, &tm_k, bar_addr(sbase, KFULL + st), hf * 64, U.hk,
                         n * 128, U.b);
           last_k_par[st] = ph;
           const int vs = kv % kVStages, vph = (kv / kVStages) & 1;
-          if (!mbar_wait(bar_addr(sbase, VEMPTY + vs), vph ^ 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(bar_addr(sbase, VEMPTY + vs), vph ^ 1, abort_flag, p.wait_ns)) { ok = false; break; }
           mbar_expect_tx(bar_addr(sbase, VFULL + vs), kTile + (kCkGlobal ? 512 : 0));
           for (int hf = 0; hf < 2; ++hf)
             tma_load_4d(sbase + kV + vs * kTile + hf * kHalf, &tm_v, bar_addr(sbase, VFULL + vs), hf * 64, U.hk,
@@ -267,14 +265,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++uidx;
       }
-      if (*abort_flag) {
-        // Let copies still in flight land before the CTA's shared memory goes away.
-        volatile int never = 0;
+      {
+        // Every exit, normal or aborted: the copies still in flight land before
+        // the CTA's shared memory goes away (on the normal path they have landed).
         for (int s = 0; s < kKStages; ++s)
-          if (last_k_par[s] >= 0) mbar_wait(bar_addr(sbase, KFULL + s), last_k_par[s], &never);
+          if (last_k_par[s] >= 0) mbar_drain(bar_addr(sbase, KFULL + s), last_k_par[s]);
         for (int s = 0; s < kVStages; ++s)
-          if (last_v_par[s] >= 0) mbar_wait(bar_addr(sbase, VFULL + s), last_v_par[s], &never);
-        if (last_q_par >= 0) mbar_wait(bar_addr(sbase, QFULL), last_q_par, &never);
+          if (last_v_par[s] >= 0) mbar_drain(bar_addr(sbase, VFULL + s), last_v_par[s]);
+        if (last_q_par >= 0) mbar_drain(bar_addr(sbase, QFULL), last_q_par);
       }
     } else if (warp == 9 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
@@ -305,10 +303,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = unit_index(cta, r, G);
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
-        if (!mbar_wait(bar_addr(sbase, QFULL), uidx & 1, abort_flag)) break;
+        if (!mbar_wait(bar_addr(sbase, QFULL), uidx & 1, abort_flag, p.wait_ns)) break;
         {
           const int st = kv % kKStages, ph = (kv / kKStages) & 1;
-          if (!mbar_wait(bar_addr(sbase, KFULL + st), ph, abort_flag)) break;
+          if (!mbar_wait(bar_addr(sbase, KFULL + st), ph, abort_flag, p.wait_ns)) break;
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 2; ++k)
@@ -328,14 +326,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int vsn = kvn % kVStages, vphn = (kvn / kVStages) & 1;
           const int stx = kvx % kKStages, phx = (kvx / kKStages) & 1;
           const bool has_next = it + 1 < U.N;
-          if (!mbar_wait(bar_addr(sbase, VFULL + vsn), vphn, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(bar_addr(sbase, VFULL + vsn), vphn, abort_flag, p.wait_ns)) { ok = false; break; }
           bool k_next_ready = false;
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
             if (U.in(k, n)) {
               if (first_pv[k] && ounits[k] > 0 &&
-                  !mbar_wait(bar_addr(sbase, OFREE + k), (ounits[k] - 1) & 1, abort_flag)) { ok = false; break; }
-              if (!mbar_wait(bar_addr(sbase, PFULL + k), pcount[k] & 1, abort_flag)) { ok = false; break; }
+                  !mbar_wait(bar_addr(sbase, OFREE + k), (ounits[k] - 1) & 1, abort_flag, p.wait_ns)) { ok = false; break; }
+              if (!mbar_wait(bar_addr(sbase, PFULL + k), pcount[k] & 1, abort_flag, p.wait_ns)) { ok = false; break; }
               ++pcount[k];
               tc_fence_after();
               issue_pv(k, vsn, !first_pv[k]);
@@ -344,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (k == 1) mma_commit(bar_addr(sbase, VEMPTY + vsn));
             if (has_next && U.in(k, n - 1)) {
               if (!k_next_ready) {
-                if (!mbar_wait(bar_addr(sbase, KFULL + stx), phx, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(bar_addr(sbase, KFULL + stx), phx, abort_flag, p.wait_ns)) { ok = false; break; }
                 k_next_ready = true;
               }
               tc_fence_after();
@@ -367,8 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Drain: every MMA issued by this thread completes before TMEM is freed.
       mma_commit(bar_addr(sbase, FINAL));
-      volatile int never = 0;
-      mbar_wait(bar_addr(sbase, FINAL), 0, &never);
+      mbar_drain(bar_addr(sbase, FINAL), 0);
     }
   } else {
     regs_inc<kRegsHigh>();
@@ -397,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++uidx;
         continue;
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, QFULL), uidx & 1, abort_flag))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, QFULL), uidx & 1, abort_flag, p.wait_ns))) break;
       const int i = r0k + row;
       // rq_i from this thread's own Q row in shared memory.
       float rq;
@@ -431,11 +428,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kSlots = kCkGlobal ? kVStages : kCkSlots;
         const int vsn = kvn % kSlots, vphn = (kvn / kSlots) & 1;
         if (!__all_sync(0xffffffffu,
-                        mbar_wait(bar_addr(sbase, (kCkGlobal ? VFULL : CKFULL) + vsn), vphn, abort_flag))) {
+                        mbar_wait(bar_addr(sbase, (kCkGlobal ? VFULL : CKFULL) + vsn), vphn, abort_flag, p.wait_ns))) {
           ok = false;
           break;
         }
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, SFULL + k), scount & 1, abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, SFULL + k), scount & 1, abort_flag, p.wait_ns))) {
           ok = false;
           break;
         }
@@ -473,14 +470,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
-                  float t0, t1, p0, p1;
+                  float t0, t1;
                   ffma2(t0, t1, x[2 * h2], x[2 * h2 + 1], rq, rq, negb, negb);
-                  if (((2 * j4 + h2) & 3) < kEmuPairsOf4) {
-                    exp2_fma2(t0, t1, p0, p1);  // FMA pipe
-                  } else {
-                    p0 = ex2(t0);  // MUFU
-                    p1 = ex2(t1);
-                  }
+                  const float p0 = ex2(t0), p1 = ex2(t1);
                   fadd2(l0, l1, p0, p1);
                   const uint32_t pp = pack_bf16(p0, p1);
                   add_bf16x2_f32(lr0, lr1, pp);
@@ -570,15 +562,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            float t0, t1, p0, p1;
+            float t0, t1;
             ffma2(t0, t1, __uint_as_float(s[32 * c + 2 * e]), __uint_as_float(s[32 * c + 2 * e + 1]), rq, rq, negm,
                   negm);
-            if ((e & 3) < kEmuPairsOf4) {
-              exp2_fma2(t0, t1, p0, p1);  // FMA pipe
-            } else {
-              p0 = ex2(t0);  // MUFU
-              p1 = ex2(t1);
-            }
+            const float p0 = ex2(t0), p1 = ex2(t1);
             fadd2(l0, l1, p0, p1);
             pk[e] = pack_bf16(p0, p1);
           }
@@ -590,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, ODONE + k), ecount & 1, abort_flag))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, ODONE + k), ecount & 1, abort_flag, p.wait_ns))) break;
       ++ecount;
       tc_fence_after();
       const float l = l0 + l1;
@@ -616,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(bar_addr(sbase, OFREE + k));
-      if (iv) p.lse[(size_t)U.bh * p.T + i] = ((kFixed ? p.bound : m) + log2f(l)) * kLn2;
+      if (iv && p.lse) p.lse[(size_t)U.bh * p.T + i] = ((kFixed ? p.bound : m) + log2f(l)) * kLn2;
       kv += U.N;
       ++uidx;
     }

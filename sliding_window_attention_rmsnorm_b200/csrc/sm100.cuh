@@ -15,7 +15,10 @@ namespace ar {
 enum : int { DEV_TIMEOUT = 1, DEV_LAYOUT = 2 };
 __device__ int g_status = 0;
 
-// A wait gives up after this many nanoseconds of %globaltimer.
+// Default limit of a device-side wait, in nanoseconds of %globaltimer.  Every
+// kernel takes its limit as a parameter (the library passes this value unless
+// ar_attn_set_wait_limit_ns chose another); the waits that drain copies and
+// tensor-core work still in flight before a CTA exits always use this one.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ unsigned long long globaltimer() {
@@ -67,21 +70,30 @@ __device__ __forceinline__ bool mbar_try_sleep(uint32_t bar, uint32_t parity, ui
       : "memory");
   return ok != 0;
 }
-// Wait for the phase of `parity` to complete.  Bounded: after kWaitLimitNs it
+// Wait for the phase of `parity` to complete.  Bounded: after limit_ns it
 // records DEV_TIMEOUT, raises the CTA's abort flag and returns false.  A wait
 // also returns false when another role of the CTA has aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit_ns) {
   if (mbar_try(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
+  const uint32_t hint = limit_ns < 20000ull ? (uint32_t)limit_ns : 20000u;
   for (;;) {
-    if (mbar_try_sleep(bar, parity, 20000u)) return true;
+    if (mbar_try_sleep(bar, parity, hint)) return true;
     if (*abort_flag) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       atomicOr(&g_status, DEV_TIMEOUT);
       *abort_flag = 1;
       return false;
     }
   }
+}
+// Wait, with the default limit, for work this thread itself started (a copy,
+// a batch of tensor-core operations) before the CTA may exit.  Used on every
+// exit path, normal or aborted, so that nothing is left in flight.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+  volatile int never = 0;
+  mbar_wait(bar, parity, &never, kWaitLimitNs);
 }
 
 // ------------------------------------------------------------------ TMA / bulk copies
@@ -299,31 +311,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-
-// 2^t for two arguments on the FMA pipe instead of the MUFU unit (whose ex2
-// throughput, 16 per clock per SM, is the softmax bottleneck).  Cody-Waite
-// style: n = round(t) via the 1.5*2^23 rounding constant, f = t - n in
-// [-1/2, 1/2], 2^f by a degree-3 polynomial fitted here for minimax relative
-// error (7.5e-5 over the interval), and 2^n added to the exponent field.
-// t is clamped to [-126, 2^22); t = -inf gives 2^-126.
-__device__ __forceinline__ void exp2_fma2(float t0, float t1, float& p0, float& p1) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  t0 = fmaxf(t0, -126.0f);
-  t1 = fmaxf(t1, -126.0f);
-  uint64_t r, n, f, p;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2pack(t0, t1)), "l"(f2pack(kRound, kRound)));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(n) : "l"(r), "l"(f2pack(kRound, kRound)));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f) : "l"(f2pack(t0, t1)), "l"(n));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(f2pack(5.517166853e-02f, 5.517166853e-02f)), "l"(f),
-      "l"(f2pack(2.426111400e-01f, 2.426111400e-01f)));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(f2pack(6.932609677e-01f, 6.932609677e-01f)));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(f2pack(9.999280572e-01f, 9.999280572e-01f)));
-  float q0, q1, r0, r1;
-  f2unpack(p, q0, q1);
-  f2unpack(r, r0, r1);
-  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(r0) << 23));
-  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(r1) << 23));
 }
 
 // ------------------------------------------------------------------ math helpers

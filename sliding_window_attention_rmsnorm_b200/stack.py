@@ -39,13 +39,11 @@ class Stack:
                          lse=torch.empty((B, H, T), dtype=torch.float32, device=dev),
                          dq=torch.empty_like(L["q"]), dk=torch.empty_like(L["k"]),
                          dv=torch.empty_like(L["v"])) for L in layers]
-        self.ws_fwd = torch.empty(attn.fwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device=dev)
         self.ws_bwd = torch.empty(attn.bwd_workspace_bytes(B, T, H, D, Hkv), dtype=torch.uint8, device=dev)
 
     def forward(self):
         for L, O, w in zip(self.layers, self.out, self.windows):
-            attn.fwd(L["q"], L["k"], L["v"], w, self.eps, self.scale, out=O["o"], lse=O["lse"],
-                     workspace=self.ws_fwd)
+            attn.fwd(L["q"], L["k"], L["v"], w, self.eps, self.scale, out=O["o"], lse=O["lse"])
 
     def backward(self):
         for L, O, w in zip(reversed(self.layers), reversed(self.out), reversed(self.windows)):

@@ -69,9 +69,8 @@ def test_unmasked_pairs_matches_oracle(L):
 
 def test_workspace_sizes(L):
     B, T, H, D = 8, 2048, 4, 128
-    # the forward kernel derives the per-key norm factors itself: no scratch
-    assert attn.fwd_workspace_bytes(B, T, H, D) == 0
-    assert attn.fwd_workspace_bytes(1, 200, 1, 128) == 0
+    # the forward needs no scratch: it has no workspace argument at all
+    assert not hasattr(L, "ar_attn_fwd_workspace_bytes")
     # three per-token fp32 vectors + one 32 KB G tile per (query tile, key tile)
     # pair of the full causal band, nq (nq + 1) / 2 per head (nq = 16 here)
     assert attn.bwd_workspace_bytes(B, T, H, D) == 3 * B * H * T * 4 + B * H * 136 * 32768
@@ -88,10 +87,9 @@ P16 = 1 << 20  # a 16-byte aligned placeholder address; never dereferenced
 
 
 def fwd_call(L, q=P16, k=P16, v=P16, o=P16, lse=P16, B=1, T=128, H=1, D=128, window=-1, eps=1e-6,
-             scale=0.088, ws=None, ws_bytes=0):
+             scale=0.088):
     vp = ctypes.c_void_p
-    return L.ar_attn_fwd(vp(q), vp(k), vp(v), vp(o), vp(lse), B, T, H, D, window, eps, scale, vp(ws),
-                         ws_bytes, None)
+    return L.ar_attn_fwd(vp(q), vp(k), vp(v), vp(o), vp(lse), B, T, H, D, window, eps, scale, None)
 
 
 def bwd_call(L, ptr=P16, dq=P16, B=1, T=128, H=1, D=128, eps=1e-6, scale=0.088, ws=None, ws_bytes=0):
@@ -102,7 +100,11 @@ def bwd_call(L, ptr=P16, dq=P16, B=1, T=128, H=1, D=128, eps=1e-6, scale=0.088, 
 
 def test_fwd_argument_errors(L):
     assert fwd_call(L, q=0) == -1
-    assert fwd_call(L, lse=0) == -1
+    assert fwd_call(L, o=0) == -1
+    # lse may be NULL (the forward-only use): validation goes on to the next check
+    assert fwd_call(L, lse=0, B=0) == -2
+    assert fwd_call(L, lse=0, k=P16 + 8) == -4
+    assert fwd_call(L, lse=P16 + 2) == -4
     assert fwd_call(L, B=0) == -2
     assert fwd_call(L, T=-3) == -2
     assert fwd_call(L, H=0) == -2
@@ -162,3 +164,24 @@ def test_stack_buffers_follow_kv_heads(L):
         assert st.out[0]["dk"].shape == (B, T, Hkv, D) and st.out[1]["dv"].shape == (B, T, Hkv, D)
         assert st.out[0]["dq"].shape == (B, T, H, D) and st.out[0]["lse"].shape == (B, H, T)
         assert st.ws_bwd.numel() == attn.bwd_workspace_bytes(B, T, H, D, Hkv) > 0
+
+
+def test_wait_limit_setter(L):
+    """Host-side only: the setter accepts any limit and 0 restores the default."""
+    assert L.ar_attn_set_wait_limit_ns(ctypes.c_ulonglong(1)) == 0
+    assert L.ar_attn_set_wait_limit_ns(ctypes.c_ulonglong(0)) == 0
+    attn.set_wait_limit_ns(0)
+
+
+def test_binding_rejects_mismatched_outputs():
+    """Caller-supplied outputs are checked against the tensors they are shaped
+    after before anything reaches the library (CPU tensors: rejected as not on
+    a CUDA device, whatever else is wrong)."""
+    import torch
+    q = torch.zeros(1, 4, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        attn._check_out(torch.zeros(1, 4, 1, 128, dtype=torch.bfloat16), q, "dq")
+    with pytest.raises(ValueError):
+        attn._check_out(q.float(), q, "out")
+    with pytest.raises(ValueError):
+        attn._check_lse(torch.zeros(1, 2, 4), 1, 2, 4, q.device)

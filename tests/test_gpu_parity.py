@@ -15,6 +15,7 @@ import numpy as np
 import pytest
 import torch
 
+import kernel_model
 from oracle import oracle as orc
 from oracle.stack import layer_windows as oracle_windows
 from sliding_window_attention_rmsnorm_b200 import attn, build, stack, synth
@@ -29,14 +30,54 @@ EPS = 1e-6
 # precision model) add up to about one bf16 ulp of the result on top of the
 # output's own rounding, so |err| <= 2e-2 + 2^-8 |ref| elementwise.
 ULP_SLACK = 2.0 ** -8
+# The same cases are compared with tests/kernel_model.py, which recomputes the
+# kernels' sequence of bf16 roundings in fp64 (its CPU tests show it equals
+# the oracle without them).  Elementwise the GPU cannot match it exactly: a
+# rounding of one P or G value that lands on the other side (about one value
+# in a thousand, from fp32 against fp64 arithmetic before the rounding) moves a
+# short row's output by a few ulps.  In aggregate it must:
+#   ||gpu - model|| <= 2^-8 ||model||          (one ulp, in relative L2)
+#   ||gpu - oracle|| <= 1.2 ||model - oracle|| + 2e-6 sqrt(n)
+# i.e. the GPU's error is the error the bf16 roundings explain, and no more.
+MODEL_L2, MODEL_ERR_RATIO, MODEL_FLOOR = 2.0 ** -8, 1.2, 2e-6
 
 
-@pytest.fixture(scope="module", autouse=True)
-def _lib():
-    if not torch.cuda.is_available():
-        pytest.skip("no CUDA device")
-    build.build()
-    attn.lib()
+def model_misfit(gpu, x, window, eps=EPS, scale=None, names=("o", "lse", "dq", "dk", "dv"), ref=None):
+    """Per tensor: (relative L2 distance of the GPU from the kernel-arithmetic
+    model, and ||gpu - oracle|| / (||model - oracle|| + floor) when the oracle
+    result `ref` is given).  The model's backward is fed the GPU's own o and
+    lse, so that a rounding of o that went the other way on the GPU (which
+    moves delta = dO . o) is not counted against the backward.  For lse the
+    first number is the largest absolute difference."""
+    mo, mlse = kernel_model.forward(x["q"], x["k"], x["v"], window, eps, scale)
+    model = dict(o=mo, lse=mlse)
+    if any(n in names for n in ("dq", "dk", "dv")):
+        mdq, mdk, mdv = kernel_model.backward(x["q"], x["k"], x["v"], gpu["o"], x["dO"], gpu["lse"], window, eps,
+                                              scale)
+        model.update(dq=mdq, dk=mdk, dv=mdv)
+    out = {}
+    for n in names:
+        a, m = gpu[n].astype(np.float64), model[n]
+        if n == "lse":
+            out[n] = (float(np.abs(a - m).max()), 0.0)
+            continue
+        nm = np.linalg.norm(m)
+        rel = float(np.linalg.norm(a - m) / nm) if nm > 0 else float(np.abs(a).max())
+        ratio = 0.0
+        if ref is not None:
+            r = ref[n]
+            ratio = float(np.linalg.norm(a - r) / (MODEL_ERR_RATIO * np.linalg.norm(m - r) + MODEL_FLOOR * math.sqrt(r.size)))
+        out[n] = (rel, ratio)
+    return out
+
+
+def check_model(gpu, x, window, eps=EPS, scale=None, tag="", ref=None):
+    for n, (rel, ratio) in model_misfit(gpu, x, window, eps, scale, ref=ref).items():
+        if n == "lse":
+            assert rel <= 1e-5, (tag, n, "lse off the kernel-arithmetic model by", rel)
+            continue
+        assert rel <= MODEL_L2, (tag, n, "rel l2 against the kernel-arithmetic model", rel)
+        assert ratio <= 1.0, (tag, n, "error beyond what the bf16 roundings explain", ratio)
 
 
 def run_gpu(x, window, eps=EPS, scale=None, D=128):
@@ -101,26 +142,40 @@ def test_small_config_whole(window):
 def test_ragged_and_windows(T, window):
     B, H = 2, 3
     x = synth.layer_inputs(7, T, B, T, H, 128)
-    compare(run_gpu(x, window), run_oracle(x, window), H, tag="T=%d w=%d" % (T, window), edge=True)
+    g, ref = run_gpu(x, window), run_oracle(x, window)
+    compare(g, ref, H, tag="T=%d w=%d" % (T, window), edge=True)
+    check_model(g, x, window, tag="T=%d w=%d" % (T, window), ref=ref)
 
 
 def test_peaked_logits():
     """Keys close to their queries push logits towards the +-sqrt(D) bound and
-    saturate the softmax.  dq and dk then nearly vanish (|dq| ~ 5e-3), and their
-    absolute error is set by delta = rowsum(dO * o) taken from the bf16 output
-    o; they are held to the absolute bound only, o and dv also to relative L2."""
+    saturate the softmax.  dq and dk then nearly vanish (|dq| ~ 5e-3) and their
+    error against the oracle is dominated by delta = rowsum(dO * o) taken from
+    the bf16 output o (FlashAttention's convention): the kernel-arithmetic
+    model shows a relative L2 error of about 0.34 from that rounding alone.  So
+    dq and dk are held to the oracle by the absolute bound, and to the model
+    (which reproduces that error) by the one-ulp bound at their own scale; an
+    all-zero dq or dk would miss the latter by far, as checked here."""
     B, T, H = 1, 384, 2
     x = synth.layer_inputs(9, 0, B, T, H, 128)
     x["k"] = synth.peaked_keys(x["q"], 9999)
     for w in (64, -1):
-        compare(run_gpu(x, w), run_oracle(x, w), H, tag="peaked w=%d" % w, edge=True, rel_for=("o", "dv"))
+        g, ref = run_gpu(x, w), run_oracle(x, w)
+        compare(g, ref, H, tag="peaked w=%d" % w, edge=True, rel_for=("o", "dv"))
+        check_model(g, x, w, tag="peaked w=%d" % w, ref=ref)
+        for n in ("dq", "dk"):
+            zero = dict(g, **{n: np.zeros_like(g[n])})
+            rel, _ = model_misfit(zero, x, w, names=(n,))[n]
+            assert rel == 1.0 > MODEL_L2, (n, "a zero gradient must fail the model check")
 
 
 def test_other_eps_and_scale():
     B, T, H = 1, 256, 2
     x = synth.layer_inputs(11, 0, B, T, H, 128)
     for eps, scale in ((0.0, 0.05), (1e-2, 0.2)):
-        compare(run_gpu(x, 100, eps, scale), run_oracle(x, 100, eps, scale), H, tag="eps=%g" % eps, edge=True)
+        g, ref = run_gpu(x, 100, eps, scale), run_oracle(x, 100, eps, scale)
+        compare(g, ref, H, tag="eps=%g" % eps, edge=True)
+        check_model(g, x, 100, eps, scale, tag="eps=%g" % eps, ref=ref)
 
 
 def test_running_max_forward():
@@ -138,6 +193,9 @@ def test_running_max_forward():
         attn.sync_status()
         ro, rl = orc.attn_fwd(x["q"], x["k"], x["v"], w, EPS, 0.2)
         o = o.float().cpu().numpy().astype(np.float64)
+        mis = model_misfit(dict(o=o, lse=lse.cpu().numpy()), x, w, EPS, 0.2, names=("o", "lse"),
+                           ref=dict(o=ro, lse=rl))
+        assert mis["o"][0] <= MODEL_L2 and mis["o"][1] <= 1.0 and mis["lse"][0] <= 1e-5, (w, peaked, mis)
         err = np.abs(o - ro)
         assert (err - (MAX_ABS + ULP_SLACK * np.abs(ro))).max() <= 0, (w, peaked, err.max())
         assert np.linalg.norm(o - ro) / np.linalg.norm(ro) <= REL_L2, (w, peaked)
@@ -178,14 +236,77 @@ def test_stack_of_eight_layers_sampled():
         compare(gpu, run_oracle(xc, st.windows[l], heads=head), H, head, tag="stack layer %d" % l)
 
 
-def test_twelve_layer_stack_shape_sampled():
-    """Depth-12 stack shape (H=6): layer 0 (S) and layer 11 (forced L) on one head each."""
-    B, T, H = 8, 2048, 6
-    ws = oracle_windows(12, T, "SSSL")
-    for l in (0, 11):
-        x = synth.layer_inputs(5, l, B, T, H, 128)
-        head = [7 * l % (B * H)]
-        compare(run_gpu(x, ws[l]), run_oracle(x, ws[l], heads=head), H, head, tag="cfg5 layer %d" % l)
+def test_twelve_layer_stack_sampled():
+    """The 12-layer SSSL stack of the depth-12 model (B=8, T=2048, H=6; layer 11
+    forced global), run through the stack driver as the benchmark runs it (one
+    backward workspace reused by every layer), every layer checked on one head."""
+    B, T, H, n_layer = 8, 2048, 6, 12
+    layers = [{r: t.cuda() for r, t in synth.layer_inputs(5, l, B, T, H, 128).items()} for l in range(n_layer)]
+    st = stack.Stack(layers, "SSSL", EPS)
+    assert st.windows == oracle_windows(n_layer, T, "SSSL")
+    st.step()
+    attn.sync_status()
+    for l in range(n_layer):
+        head = [(7 * l + 5) % (B * H)]
+        xc = {r: t.cpu() for r, t in layers[l].items()}
+        gpu = {n: t.float().cpu().numpy() for n, t in st.out[l].items()}
+        compare(gpu, run_oracle(xc, st.windows[l], heads=head), H, head, tag="cfg5 layer %d" % l)
+
+
+@pytest.mark.parametrize("Hkv", [8, 4])
+def test_backward_in_several_head_groups(Hkv):
+    """B=2, T=8192, H=8, full causal: the G tiles of all 16 query heads (68 MB
+    each) exceed the 1 GiB buffer, so the backward runs as two launches of the
+    main and dq kernels over disjoint head groups (the second with a nonzero
+    first head).  One head from each launch is compared with the oracle; with
+    grouped K/V heads (Hkv=4) the two launches hold whole groups."""
+    B, T, H, w = 2, 8192, 8, -1
+    assert attn.bwd_workspace_bytes(B, T, H, 128, Hkv) < B * H * 2080 * 32768  # really split
+    if Hkv == H:
+        x = synth.layer_inputs(6, 0, B, T, H, 128)
+        heads = [3, B * H - 3]  # first launch: heads 0-7; second: 8-15
+    else:
+        x = gqa_inputs(24, B, T, H, Hkv)
+        heads = [1, B * Hkv - 2]  # K/V heads; the oracle also computes their groups' query heads
+    g = run_gpu(x, w)
+    grp = H // Hkv
+    qheads = [hk // Hkv * H + (hk % Hkv) * grp + m for hk in heads for m in range(grp)]
+    o, lse = orc.attn_fwd(x["q"], x["k"], x["v"], w, EPS, heads=qheads)
+    rg = orc.attn_bwd(x["q"], x["k"], x["v"], x["dO"], w, EPS, heads=heads)  # K/V heads and their groups
+    ref = dict(o=o, lse=lse, dq=rg["dq"], dk=rg["dk"], dv=rg["dv"])
+    for n in ("o", "lse", "dq"):
+        compare_one(g[n], ref[n], n, H, qheads, tag="groups Hkv=%d" % Hkv)
+    for n in ("dk", "dv"):
+        compare_one(g[n], ref[n], n, Hkv, heads, tag="groups Hkv=%d" % Hkv)
+
+
+def compare_one(a, b, n, nh, heads, tag=""):
+    """The spec bar on one tensor restricted to the listed flat heads."""
+    a = select(a, n, nh, heads).astype(np.float64)
+    b = select(b, n, nh, heads)
+    err = np.abs(a - b)
+    if n == "lse":
+        assert err.max() <= LSE_ABS, (tag, n, err.max())
+        return
+    assert err.max() <= MAX_ABS, (tag, n, "max abs", err.max())
+    assert np.linalg.norm(a - b) / np.linalg.norm(b) <= REL_L2, (tag, n)
+
+
+def test_forward_without_lse():
+    """The forward-only use: lse not requested, o bitwise the same."""
+    B, T, H, w = 2, 640, 3, 200
+    x = synth.layer_inputs(25, 0, B, T, H, 128)
+    q, k, v = (x[r].cuda() for r in ("q", "k", "v"))
+    o, lse = attn.fwd(q, k, v, w)
+    o2, none = attn.fwd(q, k, v, w, need_lse=False)
+    attn.sync_status()
+    assert none is None and torch.equal(o, o2)
+    kv = gqa_inputs(25, B, T, 4, 2)
+    q4, k2, v2 = (kv[r].cuda() for r in ("q", "k", "v"))
+    o4, _ = attn.fwd(q4, k2, v2, w)
+    o4b, _ = attn.fwd(q4, k2, v2, w, need_lse=False)
+    attn.sync_status()
+    assert torch.equal(o4, o4b)
 
 
 # ------------------------------------------------------------------ closed forms on the GPU
@@ -289,6 +410,7 @@ def test_grouped_kv_heads(B, T, H, Hkv, window):
     assert g["dk"].shape == (B, T, Hkv, 128) and g["dv"].shape == (B, T, Hkv, 128)
     ref = run_oracle(x, window)
     compare(g, ref, H, tag="gqa H=%d Hkv=%d w=%d" % (H, Hkv, window), edge=True)
+    check_model(g, x, window, tag="gqa H=%d Hkv=%d w=%d" % (H, Hkv, window), ref=ref)
 
 
 def test_grouped_kv_heads_equal_duplicated_heads_on_gpu():
@@ -302,9 +424,14 @@ def test_grouped_kv_heads_equal_duplicated_heads_on_gpu():
     g, gd = run_gpu(x, w), run_gpu(xd, w)
     assert np.array_equal(g["o"], gd["o"]) and np.array_equal(g["lse"], gd["lse"])
     for n in ("dk", "dv"):
-        summed = gd[n].astype(np.float64).reshape(B, T, Hkv, H // Hkv, 128).sum(axis=3)
-        # the grouped result is rounded to bf16 once, each summed term once more:
-        # three roundings of at most half a bf16 ulp (2^-9 relative) each
+        terms = gd[n].astype(np.float64).reshape(B, T, Hkv, H // Hkv, 128)
+        summed = terms.sum(axis=3)
+        # each summed term was rounded to bf16 on its own (half an ulp, 2^-9 of
+        # that term) and the grouped result once (2^-9 of the sum); when the
+        # terms cancel, their roundings can exceed 2^-9 of the sum, so the bound
+        # counts them by their absolute values, and by twice that for the
+        # bf16 P and G operands (which are rounded per term as well)
+        bound = MAX_ABS + 2.0 ** -8 * np.abs(terms).sum(axis=3) + 2.0 ** -9 * np.abs(summed)
         err = np.abs(g[n] - summed)
-        assert (err - (MAX_ABS + 2.0 ** -7 * np.abs(summed))).max() <= 0, (n, err.max())
+        assert (err - bound).max() <= 0, (n, err.max())
         assert np.linalg.norm(g[n] - summed) / np.linalg.norm(summed) <= REL_L2
