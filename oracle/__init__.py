@@ -9,5 +9,7 @@ Contents:
   attn_oracle.c  plain C fp64 forward/backward (the definitions, written out)
   oracle.py      ctypes loader and numpy/torch marshalling
   stack.py       the per-layer window pattern ("SSSL", last layer global)
+  rope_ve.py     rotary position embedding of q, k and the value-embedding gate
+                 on v (the steps just before the core), on top of the above
   build.py       compiles attn_oracle.c with gcc/OpenMP
 """
