@@ -47,6 +47,11 @@ WORKLOADS = {
                    name="long-context S layer fwd+bwd, B=2 T=8192 H=4 D=128, window 4096"),
     "long_l": dict(config=4, B=2, T=8192, H=4, n_layer=1, windows=[8192],
                    name="long-context L layer fwd+bwd, B=2 T=8192 H=4 D=128, full causal"),
+    # the stack with the steps before the core fused in: RoPE on every layer, the
+    # value embedding on every other layer (the last included); not a stated workload
+    "stack8_rope": dict(config=3, B=8, T=2048, H=4, n_layer=8, pattern="SSSL", rope=True,
+                        name="8-layer SSSL attention stack fwd+bwd with fused RoPE and value embeddings, "
+                             "B=8 T=2048 H=4 D=128 (windows 1024/full)"),
     # grouped K/V heads (n_kv_head = n_head / 2): not one of the stated workloads
     "stack8_gqa": dict(config=3, B=8, T=2048, H=4, Hkv=2, n_layer=8, pattern="SSSL",
                        name="8-layer SSSL attention stack fwd+bwd, B=8 T=2048 H=4 Hkv=2 D=128 (windows 1024/full)"),
@@ -192,13 +197,17 @@ _INPUT_CACHE = {}
 
 
 def layer_host_inputs(wl, layer):
-    """Seeded bf16 CPU inputs of one layer: q, dO with H heads, k, v with Hkv."""
+    """Seeded bf16 CPU inputs of one layer: q, dO with H heads, k, v with Hkv
+    (and ve, g on the value-embedding layers of a RoPE workload)."""
     from sliding_window_attention_rmsnorm_b200 import synth
     H, Hkv = wl["H"], wl.get("Hkv", wl["H"])
     if Hkv == H:
-        return synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], H, D)
-    x = synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], H, D, roles=("q", "dO"))
-    x.update(synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], Hkv, D, roles=("k", "v")))
+        x = synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], H, D)
+    else:
+        x = synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], H, D, roles=("q", "dO"))
+        x.update(synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], Hkv, D, roles=("k", "v")))
+    if wl.get("rope") and layer % 2 == (wl["n_layer"] - 1) % 2:
+        x["ve"], x["g"] = synth.value_embedding(wl["config"], layer, wl["B"], wl["T"], Hkv, D)
     return x
 
 
@@ -222,10 +231,17 @@ def oracle_sample(wl, seconds, seed_layer_offset=0):
         b, h = divmod(head, H)
         hk = h // (H // wl.get("Hkv", H))  # the query head's K/V head
         x = _layer_inputs_cached(wl, layer)
-        xs = {r: t[b:b + 1, :, (hk if r in ("k", "v") else h):][:, :, :1].contiguous() for r, t in x.items()}
+        xs = {r: t[b:b + 1, :, (hk if r in ("k", "v", "ve", "g") else h):][:, :, :1].contiguous()
+              for r, t in x.items()}
         t0 = time.perf_counter()
-        orc.attn_fwd(xs["q"], xs["k"], xs["v"], ws[layer])
-        orc.attn_bwd(xs["q"], xs["k"], xs["v"], xs["dO"], ws[layer])
+        if wl.get("rope"):
+            from oracle import rope_ve
+            cs, sn = rope_ve.rope_tables(T, D)
+            rope_ve.attn_fwd(xs["q"], xs["k"], xs["v"], cs, sn, ws[layer], ve=xs.get("ve"), g=xs.get("g"))
+            rope_ve.attn_bwd(xs["q"], xs["k"], xs["v"], xs["dO"], cs, sn, ws[layer], ve=xs.get("ve"), g=xs.get("g"))
+        else:
+            orc.attn_fwd(xs["q"], xs["k"], xs["v"], ws[layer])
+            orc.attn_bwd(xs["q"], xs["k"], xs["v"], xs["dO"], ws[layer])
         t_total += time.perf_counter() - t0
         flops += pairs(T, ws[layer]) * FWD_FLOPS_PER_PAIR * (1 + BWD_FACTOR)
         heads_done.append((layer, head))
@@ -287,7 +303,8 @@ def run_ours(args, wl, rank, world, dist):
     B, T, H, L = wl["B"], wl["T"], wl["H"], wl["n_layer"]
     host = [layer_host_inputs(wl, l) for l in range(L)]
     layers = [{r: t.to("cuda", non_blocking=False) for r, t in x.items()} for x in host]
-    st = stack.Stack(layers, wl.get("pattern", "SSSL"), windows=wl.get("windows"))
+    rope = attn.rope_tables(T, D) if wl.get("rope") else None
+    st = stack.Stack(layers, wl.get("pattern", "SSSL"), windows=wl.get("windows"), rope=rope)
     windows = lib_windows(wl)
     fwd_f, bwd_f = step_flops(wl, windows)
 

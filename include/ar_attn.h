@@ -122,6 +122,43 @@ int ar_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, 
                     int B, int T, int H, int Hkv, int D, int window, float eps, float scale,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* The forward with the two steps the pages run just before the core fused
+ * into its tile loads ("autoresearch" README (gitee), section 7.4: rotary
+ * position embedding of q and k; section 5.2.3: the value embedding mixed
+ * into v on the layers that have one).  q, k, v are the unrotated, unmixed
+ * tensors; the kernel rotates each Q and K tile and mixes each V tile in shared
+ * memory, so nothing rotated or mixed is ever written.
+ *   rope_cos, rope_sin: bf16 [rope_rows, D/2] (rope_rows >= T), row t holding
+ *     position t's cos and sin; row t of q and k becomes
+ *     (x1 cos_t + x2 sin_t, -x1 sin_t + x2 cos_t) with x1, x2 its two halves.
+ *   ve, ve_gate: both NULL (no value embedding), or ve bf16 [B, T, Hkv, D] and
+ *     the gate logits g bf16 [B, T, Hkv]: v becomes v + 2 sigmoid(g) ve.
+ * Everything else (layouts, lse optional, grouped K/V heads, errors) is as for
+ * ar_attn_fwd_gqa.  AR_ERR_NULL if a table is NULL or only one of ve, ve_gate
+ * is; AR_ERR_SHAPE if rope_rows < T; tables and ve 16-byte aligned. */
+int ar_attn_fwd_rope(const void* q, const void* k, const void* v, void* o, float* lse, const void* rope_cos,
+                     const void* rope_sin, int rope_rows, const void* ve, const void* ve_gate, int B, int T,
+                     int H, int Hkv, int D, int window, float eps, float scale, void* stream);
+
+/* Backward of ar_attn_fwd_rope: the gradients with respect to the unrotated,
+ * unmixed q, k, v, and (with the value embedding) to ve and the gate logits g.
+ * Arguments as for ar_attn_bwd_gqa plus the tables and ve, ve_gate of the
+ * forward, and the outputs dve bf16 [B, T, Hkv, D] and dgate fp32 [B, T, Hkv]
+ * (all four of ve, ve_gate, dve, dgate NULL without a value embedding).
+ * A pre-pass writes the rotated q, k and the mixed v into the workspace (the
+ * same bf16 values the forward formed in its tiles); the backward kernels run
+ * on them and finish the chain rule in their epilogues: dq = R^T dq_rot and
+ * dk = R^T dk_rot with R^T the transposed rotation of the row's position
+ * (dx1 = d1 cos - d2 sin, dx2 = d1 sin + d2 cos), dv = dv_mix,
+ * dve = 2 sigmoid(g) dv_mix and dgate = (dv_mix . ve) 2 sigmoid(g) (1 - sigmoid(g)).
+ * The workspace must hold ar_attn_bwd_rope_workspace_bytes(..., ve != NULL)
+ * bytes (NULL: allocated stream-ordered, as for ar_attn_bwd). */
+size_t ar_attn_bwd_rope_workspace_bytes(int B, int T, int H, int Hkv, int D, int with_ve);
+int ar_attn_bwd_rope(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                     const void* rope_cos, const void* rope_sin, int rope_rows, const void* ve, const void* ve_gate,
+                     void* dq, void* dk, void* dv, void* dve, float* dgate, int B, int T, int H, int Hkv, int D,
+                     int window, float eps, float scale, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears this device's status word.
  * Returns AR_OK, AR_ERR_TIMEOUT if a kernel abandoned a wait since the last
  * call, AR_ERR_LAYOUT if a kernel refused to run, or AR_ERR_CUDA if the
@@ -164,11 +201,12 @@ enum {
   AR_KERNEL_BWD_PREP = 2, /* delta, 1/rms(q), lse * log2(e) (memory-bound) */
   AR_KERNEL_BWD = 3,      /* fused backward attention: dk, dv, G tiles (tensor-core bound) */
   AR_KERNEL_DQ = 4,       /* dq = G K with the q-side RMSNorm backward (reads the G tiles) */
-  AR_KERNEL_KINDS = 5
+  AR_KERNEL_ROPE_PREP = 5, /* rotated q, k and mixed v for the RoPE backward (memory-bound) */
+  AR_KERNEL_KINDS = 6
 };
 
 /* on != 0: clear the record and, until called with on == 0, bracket every
- * kernel that ar_attn_fwd, ar_attn_fwd_noalloc and ar_attn_bwd launch with CUDA events on the call's
+ * kernel that the forward and backward entry points launch with CUDA events on the call's
  * stream (a few microseconds of host time per kernel).  on == 0 stops
  * recording and keeps what was recorded for ar_attn_timing_read.  Returns AR_OK. */
 int ar_attn_timing_enable(int on);

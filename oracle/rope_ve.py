@@ -86,20 +86,41 @@ def mix_value(v, ve, g):
     return _f64(v) + 2.0 * _sigmoid(_f64(g))[..., None] * _f64(ve)
 
 
-def attn_fwd(q, k, v, cos, sin, window, eps=1e-6, scale=None, ve=None, g=None, heads=None):
-    """Forward of the attention core with RoPE on q, k (and the value embedding
-    on v when ve, g are given); returns (o, lse)."""
+def bf16_round(x):
+    """fp64 values rounded to the nearest bf16 value (ties to even)."""
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)
+    quantum = np.ldexp(1.0, e - 8)  # bf16 keeps 8 significant bits
+    return np.round(x / quantum) * quantum
+
+
+def _operands(q, k, v, cos, sin, ve, g, round_operands):
     qr, kr = rope(q, cos, sin), rope(k, cos, sin)
     vm = mix_value(v, ve, g) if ve is not None else _f64(v)
+    if round_operands is not None:
+        qr, kr = round_operands(qr), round_operands(kr)
+        if ve is not None:
+            vm = round_operands(vm)
+    return qr, kr, vm
+
+
+def attn_fwd(q, k, v, cos, sin, window, eps=1e-6, scale=None, ve=None, g=None, heads=None, round_operands=None):
+    """Forward of the attention core with RoPE on q, k (and the value embedding
+    on v when ve, g are given); returns (o, lse).  round_operands: None (exact),
+    or a function applied to the rotated q, k and the mixed v before the core,
+    e.g. bf16_round: in the pages' model those are bf16 tensors (the rotation
+    and the gate run under bf16 autocast)."""
+    qr, kr, vm = _operands(q, k, v, cos, sin, ve, g, round_operands)
     return _attn.attn_fwd(qr, kr, vm, window, eps, scale, heads=heads)
 
 
-def attn_bwd(q, k, v, dO, cos, sin, window, eps=1e-6, scale=None, ve=None, g=None, heads=None):
+def attn_bwd(q, k, v, dO, cos, sin, window, eps=1e-6, scale=None, ve=None, g=None, heads=None,
+             round_operands=None):
     """Backward of attn_fwd above: dict(dq, dk, dv[, dve, dg]) in fp64 (dg is the
     gradient with respect to the gate logits g).  heads: K/V heads, as for
-    oracle.attn_bwd."""
-    qr, kr = rope(q, cos, sin), rope(k, cos, sin)
-    vm = mix_value(v, ve, g) if ve is not None else _f64(v)
+    oracle.attn_bwd; round_operands as for attn_fwd (the chain rule through the
+    rotation and the gate stays exact)."""
+    qr, kr, vm = _operands(q, k, v, cos, sin, ve, g, round_operands)
     r = _attn.attn_bwd(qr, kr, vm, dO, window, eps, scale, heads=heads)
     out = dict(dq=rope_transposed(r["dq"], cos, sin), dk=rope_transposed(r["dk"], cos, sin), dv=r["dv"])
     if ve is not None:

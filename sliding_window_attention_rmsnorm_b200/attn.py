@@ -65,6 +65,13 @@ def lib():
         L.ar_attn_bwd_gqa_workspace_bytes.restype = sz
         L.ar_attn_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, vp, sz, vp]
         L.ar_attn_bwd_gqa.restype = i
+        L.ar_attn_fwd_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, i, i, i, i, f, f, vp]
+        L.ar_attn_fwd_rope.restype = i
+        L.ar_attn_bwd_rope_workspace_bytes.argtypes = [i, i, i, i, i, i]
+        L.ar_attn_bwd_rope_workspace_bytes.restype = sz
+        L.ar_attn_bwd_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp,
+                                       i, i, i, i, i, i, f, f, vp, sz, vp]
+        L.ar_attn_bwd_rope.restype = i
         L.ar_attn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
         L.ar_attn_set_wait_limit_ns.restype = i
         L.ar_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, vp]
@@ -204,6 +211,106 @@ def sync_status():
     _check(lib().ar_attn_sync_status(_stream()), "ar_attn_sync_status")
 
 
+def _check_rope(cos, sin, T):
+    if not (cos.is_cuda and sin.is_cuda and cos.dtype == torch.bfloat16 and sin.dtype == torch.bfloat16
+            and cos.is_contiguous() and sin.is_contiguous() and cos.dim() == 2 and cos.shape == sin.shape
+            and cos.shape[1] == 64 and cos.shape[0] >= T):
+        raise ValueError("cos, sin must be contiguous bf16 CUDA tensors [rows >= T, 64]")
+
+
+def _check_ve(ve, gate, k):
+    if (ve is None) != (gate is None):
+        raise ValueError("ve and ve_gate go together")
+    if ve is None:
+        return
+    _check_out(ve, k, "ve")
+    B, T, Hkv, _ = k.shape
+    if not (gate.is_cuda and gate.dtype == torch.bfloat16 and gate.is_contiguous()
+            and tuple(gate.shape) == (B, T, Hkv)):
+        raise ValueError("ve_gate must be a contiguous bf16 CUDA tensor [B, T, Hkv]")
+
+
+def rope_tables(T: int, D: int = 128, base: float = 10000.0, device="cuda"):
+    """cos, sin [T, D/2] bf16 as the pages' model precomputes them (angles
+    t / base^(2c/D) in fp32, rounded to bf16); built once per model, outside
+    the attention core."""
+    c = torch.arange(0, D, 2, dtype=torch.float32)
+    inv = 1.0 / (base ** (c / D))
+    ang = torch.outer(torch.arange(T, dtype=torch.float32), inv)
+    return ang.cos().to(torch.bfloat16).to(device), ang.sin().to(torch.bfloat16).to(device)
+
+
+def fwd_rope(q, k, v, cos, sin, window: int, eps: float = 1e-6, scale=None, ve=None, ve_gate=None, out=None,
+             lse=None, need_lse: bool = True):
+    """The forward with the steps before the core fused into it: q and k rotated
+    by RoPE (cos, sin: bf16 [rows >= T, 64], row t = position t) and, when ve
+    ([B, T, Hkv, 128]) and ve_gate (the gate logits g, [B, T, Hkv]) are given,
+    v replaced by v + 2 sigmoid(g) ve.  q, k, v are the unrotated, unmixed
+    tensors; nothing rotated or mixed is written."""
+    Hkv = _check_qkv(q, k, v)
+    B, T, H, D = q.shape
+    _check_rope(cos, sin, T)
+    _check_ve(ve, ve_gate, k)
+    if scale is None:
+        scale = default_scale(D)
+    if out is not None:
+        _check_out(out, q, "out")
+    o = torch.empty_like(q) if out is None else out
+    lse_t = None
+    if need_lse:
+        lse_t = torch.empty((B, H, T), dtype=torch.float32, device=q.device) if lse is None else lse
+        _check_lse(lse_t, B, H, T, q.device)
+    st = lib().ar_attn_fwd_rope(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), _ptr(cos), _ptr(sin),
+                                int(cos.shape[0]), _ptr(ve), _ptr(ve_gate), B, T, H, Hkv, D, int(window),
+                                float(eps), float(scale), _stream())
+    _check(st, "ar_attn_fwd_rope")
+    return o, lse_t
+
+
+def bwd_rope_workspace_bytes(B, T, H, D, Hkv=None, with_ve=False) -> int:
+    return int(lib().ar_attn_bwd_rope_workspace_bytes(B, T, H, Hkv or H, D, 1 if with_ve else 0))
+
+
+def bwd_rope(q, k, v, o, dO, lse, cos, sin, window: int, eps: float = 1e-6, scale=None, ve=None, ve_gate=None,
+             dq=None, dk=None, dv=None, dve=None, dgate=None, workspace=None):
+    """Backward of fwd_rope: (dq, dk, dv) for the unrotated, unmixed q, k, v,
+    plus (dve, dgate) when the forward mixed in a value embedding (dgate: the
+    gradient of the gate logits, fp32 [B, T, Hkv])."""
+    Hkv = _check_qkv(q, k, v)
+    _check_inputs(q, o, dO)
+    B, T, H, D = q.shape
+    _check_lse(lse, B, H, T, q.device)
+    _check_rope(cos, sin, T)
+    _check_ve(ve, ve_gate, k)
+    if scale is None:
+        scale = default_scale(D)
+    for t, like, name in ((dq, q, "dq"), (dk, k, "dk"), (dv, v, "dv"), (dve, k, "dve")):
+        if t is not None:
+            _check_out(t, like, name)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    with_ve = ve is not None
+    if with_ve:
+        dve = torch.empty_like(k) if dve is None else dve
+        if dgate is None:
+            dgate = torch.empty((B, T, Hkv), dtype=torch.float32, device=q.device)
+        elif not (dgate.is_cuda and dgate.dtype == torch.float32 and dgate.is_contiguous()
+                  and tuple(dgate.shape) == (B, T, Hkv)):
+            raise ValueError("dgate must be a contiguous fp32 CUDA tensor [B, T, Hkv]")
+    else:
+        dve = dgate = None
+    if workspace is None:
+        workspace = torch.empty(bwd_rope_workspace_bytes(B, T, H, D, Hkv, with_ve), dtype=torch.uint8,
+                                device=q.device)
+    st = lib().ar_attn_bwd_rope(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(cos), _ptr(sin),
+                                int(cos.shape[0]), _ptr(ve), _ptr(ve_gate), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dve),
+                                _ptr(dgate), B, T, H, Hkv, D, int(window), float(eps), float(scale), _ptr(workspace),
+                                workspace.numel(), _stream())
+    _check(st, "ar_attn_bwd_rope")
+    return (dq, dk, dv, dve, dgate) if with_ve else (dq, dk, dv)
+
+
 def set_wait_limit_ns(ns: int = 0):
     """Limit of every device-side wait in kernels launched from now on (0: the
     default, 2 s).  A kernel whose wait runs out abandons its work and
@@ -215,7 +322,7 @@ def unmasked_pairs(T: int, window: int) -> int:
     return int(lib().ar_attn_unmasked_pairs(int(T), int(window)))
 
 
-KERNELS = ("fwd_prep", "fwd", "bwd_prep", "bwd", "dq")
+KERNELS = ("fwd_prep", "fwd", "bwd_prep", "bwd", "dq", "rope_prep")
 
 
 def timing_enable(on: bool = True):

@@ -30,6 +30,7 @@ struct DeviceInfo {
   bool ready = false;
   int status = AR_OK;  // AR_OK or AR_ERR_DEVICE / AR_ERR_CUDA
   int sms = 0;
+  int prep_blocks = 1;  // resident 256-thread blocks of the delta pre-pass per SM
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -46,8 +47,12 @@ bool fwd_regs_ok(FwdKernel f) {
   cudaFuncAttributes a;
   return cudaFuncGetAttributes(&a, f) == cudaSuccess && a.numRegs == ar::fwd::kLaunchRegs;
 }
+using BwdKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, ar::BwdParams);
+cudaError_t bwd_attr(BwdKernel f) {
+  return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, ar::bwd::kSmemBytes);
+}
 
-int device_setup(int* sms_out) {
+int device_setup(int* sms_out, int* prep_blocks_out = nullptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return AR_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return AR_ERR_DEVICE;
@@ -66,9 +71,15 @@ int device_setup(int* sms_out) {
                fwd_attr(ar::fwd::fwd_kernel<false, false>) != cudaSuccess ||
                fwd_attr(ar::fwd::fwd_kernel<true, true>) != cudaSuccess ||
                fwd_attr(ar::fwd::fwd_kernel<false, true>) != cudaSuccess ||
-               cudaFuncSetAttribute(ar::bwd::bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    ar::bwd::kSmemBytes) != cudaSuccess ||
-               cudaFuncSetAttribute(ar::dqk::dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+               fwd_attr(ar::fwd::fwd_kernel<true, false, 1>) != cudaSuccess ||
+               fwd_attr(ar::fwd::fwd_kernel<false, false, 1>) != cudaSuccess ||
+               fwd_attr(ar::fwd::fwd_kernel<true, false, 3>) != cudaSuccess ||
+               fwd_attr(ar::fwd::fwd_kernel<false, false, 3>) != cudaSuccess ||
+               bwd_attr(ar::bwd::bwd_kernel<0>) != cudaSuccess || bwd_attr(ar::bwd::bwd_kernel<1>) != cudaSuccess ||
+               bwd_attr(ar::bwd::bwd_kernel<3>) != cudaSuccess ||
+               cudaFuncSetAttribute(ar::dqk::dq_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    ar::dqk::kSmemBytes) != cudaSuccess ||
+               cudaFuncSetAttribute(ar::dqk::dq_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     ar::dqk::kSmemBytes) != cudaSuccess) {
       d.status = AR_ERR_CUDA;
     }
@@ -78,12 +89,19 @@ int device_setup(int* sms_out) {
       // so refuse any other build rather than launch a kernel whose register raise
       // cannot be met.  The backward kernel is checked for its own budget.
       if (!fwd_regs_ok(ar::fwd::fwd_kernel<true, false>) || !fwd_regs_ok(ar::fwd::fwd_kernel<false, false>) ||
-          !fwd_regs_ok(ar::fwd::fwd_kernel<true, true>) || !fwd_regs_ok(ar::fwd::fwd_kernel<false, true>))
+          !fwd_regs_ok(ar::fwd::fwd_kernel<true, true>) || !fwd_regs_ok(ar::fwd::fwd_kernel<false, true>) ||
+          !fwd_regs_ok(ar::fwd::fwd_kernel<true, false, 1>) || !fwd_regs_ok(ar::fwd::fwd_kernel<false, false, 1>) ||
+          !fwd_regs_ok(ar::fwd::fwd_kernel<true, false, 3>) || !fwd_regs_ok(ar::fwd::fwd_kernel<false, false, 3>))
         d.status = AR_ERR_CUDA;
-      cudaFuncAttributes ba;
-      if (cudaFuncGetAttributes(&ba, ar::bwd::bwd_kernel) != cudaSuccess || ba.numRegs != ar::bwd::kLaunchRegs)
-        d.status = AR_ERR_CUDA;
+      for (BwdKernel f : {ar::bwd::bwd_kernel<0>, ar::bwd::bwd_kernel<1>, ar::bwd::bwd_kernel<3>}) {
+        cudaFuncAttributes ba;
+        if (cudaFuncGetAttributes(&ba, f) != cudaSuccess || ba.numRegs != ar::bwd::kLaunchRegs) d.status = AR_ERR_CUDA;
+      }
     }
+    if (d.status == AR_OK &&
+        (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.prep_blocks, ar::bwd_prep_kernel, 256, 0) != cudaSuccess ||
+         d.prep_blocks < 1))
+      d.status = AR_ERR_CUDA;
     if (!g_encode && d.status == AR_OK) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
@@ -100,6 +118,7 @@ int device_setup(int* sms_out) {
     return d.status;
   }
   *sms_out = d.sms;
+  if (prep_blocks_out) *prep_blocks_out = d.prep_blocks;
   return AR_OK;
 }
 
@@ -145,6 +164,8 @@ ar::FwdParams fwd_params(void* o, float* lse, const float* ck, int B, int T, int
                          float eps, float scale) {
   ar::FwdParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
+  p.rcos = p.rsin = p.ve = p.vg = nullptr;
+  p.wide_ve = 0;
   p.lse = lse;
   p.ck = ck;
   p.B = B;
@@ -165,12 +186,21 @@ ar::FwdParams fwd_params(void* o, float* lse, const float* ck, int B, int T, int
 
 // The forward with the fixed softmax offset when the logit bound allows it
 // (see fwd.cuh), else the running-max forward; key factors computed in the
-// kernel, or (ck_global) read from p.ck.
+// kernel, or (ck_global) read from p.ck; pro: the prologue fusion (1: RoPE,
+// 3: RoPE and the value embedding).
 void launch_fwd(int grid, cudaStream_t s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                const ar::FwdParams& p, bool ck_global) {
+                const ar::FwdParams& p, bool ck_global, int pro = 0) {
   using namespace ar::fwd;
   const bool fixed = p.bound <= kFixedBoundMax;
-  if (fixed && !ck_global)
+  if (pro == 1 && fixed)
+    fwd_kernel<true, false, 1><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
+  else if (pro == 1)
+    fwd_kernel<false, false, 1><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
+  else if (pro == 3 && fixed)
+    fwd_kernel<true, false, 3><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
+  else if (pro == 3)
+    fwd_kernel<false, false, 3><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
+  else if (fixed && !ck_global)
     fwd_kernel<true, false><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
   else if (!fixed && !ck_global)
     fwd_kernel<false, false><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
@@ -276,6 +306,16 @@ int prep_grid(long long rows, int sms) {
   return (int)blocks;
 }
 
+// The delta pre-pass: 32 rows per 256-thread block and iteration, as many
+// blocks as are resident on the GPU at once, looping over the rows.
+int bwd_prep_grid(long long rows, int sms, int per_sm) {
+  long long blocks = (rows + 31) / 32;
+  const long long cap = (long long)sms * per_sm;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return (int)blocks;
+}
+
 }  // namespace
 
 extern "C" {
@@ -314,32 +354,71 @@ int ar_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float*
   return cudaGetLastError() == cudaSuccess ? AR_OK : AR_ERR_CUDA;
 }
 
+int ar_attn_fwd_rope(const void* q, const void* k, const void* v, void* o, float* lse, const void* rope_cos,
+                     const void* rope_sin, int rope_rows, const void* ve, const void* ve_gate, int B, int T, int H,
+                     int Hkv, int D, int window, float eps, float scale, void* stream) {
+  if (!q || !k || !v || !o || !rope_cos || !rope_sin) return AR_ERR_NULL;  // lse may be NULL: not stored
+  if ((ve == nullptr) != (ve_gate == nullptr)) return AR_ERR_NULL;
+  int st = check_shape(B, T, H, D);
+  if (st != AR_OK) return st;
+  if ((st = check_kv_heads(H, Hkv)) != AR_OK) return st;
+  if (rope_rows < T) return AR_ERR_SHAPE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(rope_cos, 16) || !aligned(rope_sin, 16) || !aligned(ve, 16) || !aligned(ve_gate, 2))
+    return AR_ERR_ALIGN;
+  if ((st = check_args(eps, scale)) != AR_OK) return st;
+  int sms = 0;
+  if ((st = device_setup(&sms)) != AR_OK) return st;
+
+  CUtensorMap tq, tk, tv;
+  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, Hkv) != AR_OK ||
+      make_map(&tv, v, B, T, Hkv) != AR_OK)
+    return AR_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ar::FwdParams p = fwd_params(o, lse, nullptr, B, T, H, Hkv, window, eps, scale);
+  p.rcos = static_cast<const __nv_bfloat16*>(rope_cos);
+  p.rsin = static_cast<const __nv_bfloat16*>(rope_sin);
+  p.ve = static_cast<const __nv_bfloat16*>(ve);
+  p.vg = static_cast<const __nv_bfloat16*>(ve_gate);
+  p.wide_ve = ve != nullptr && aligned(ve, 32);
+  const int grid = p.n_units < sms ? p.n_units : sms;
+  {
+    KernelTimer t(AR_KERNEL_FWD, s);
+    launch_fwd(grid, s, tq, tk, tv, p, false, ve ? 3 : 1);
+    t.stop();
+  }
+  return cudaGetLastError() == cudaSuccess ? AR_OK : AR_ERR_CUDA;
+}
+
 int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T, int H, int D,
                 int window, float eps, float scale, void* stream) {
   return ar_attn_fwd_gqa(q, k, v, o, lse, B, T, H, H, D, window, eps, scale, stream);
 }
 
-int ar_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
-                    void* dq, void* dk, void* dv, int B, int T, int H, int Hkv, int D, int window, float eps,
-                    float scale, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return AR_ERR_NULL;
-  int st = check_shape(B, T, H, D);
-  if (st != AR_OK) return st;
-  if ((st = check_kv_heads(H, Hkv)) != AR_OK) return st;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
-      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
-    return AR_ERR_ALIGN;
-  if ((st = check_args(eps, scale)) != AR_OK) return st;
-  const size_t need = ar_attn_bwd_gqa_workspace_bytes(B, T, H, Hkv, D);
-  if (workspace && workspace_bytes < need) return AR_ERR_WORKSPACE;
-  if (workspace && !aligned(workspace, 256)) return AR_ERR_ALIGN;
-  int sms = 0;
-  if ((st = device_setup(&sms)) != AR_OK) return st;
+}  // extern "C"
 
-  CUtensorMap tq, tk, tv, tdo;
-  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, Hkv) != AR_OK ||
-      make_map(&tv, v, B, T, Hkv) != AR_OK || make_map(&tdo, dO, B, T, H) != AR_OK)
-    return AR_ERR_CUDA;
+namespace {
+
+// The RoPE / value-embedding arguments of the backward (NULL pointers: off).
+struct RopeArgs {
+  const __nv_bfloat16 *rcos = nullptr, *rsin = nullptr, *ve = nullptr, *vg = nullptr;
+  __nv_bfloat16* dve = nullptr;
+  float* dg = nullptr;
+};
+
+// Extra workspace of the RoPE path: the rotated q and k and (with a value
+// embedding) the mixed v, bf16, after the G buffer.
+size_t rope_bytes(int B, int T, int H, int Hkv, bool with_ve) {
+  const size_t kvb = round_up((size_t)B * T * Hkv * kD * 2, 256);
+  return round_up((size_t)B * T * H * kD * 2, 256) + kvb * (with_ve ? 2 : 1);
+}
+
+int bwd_run(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
+            void* dk, void* dv, int B, int T, int H, int Hkv, int window, float eps, float scale, void* workspace,
+            size_t need, void* stream, const RopeArgs* ra) {
+  int sms = 0, prep_blocks = 1;
+  int st = device_setup(&sms, &prep_blocks);
+  if (st != AR_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   void* ws = workspace;
   if (!ws && cudaMallocAsync(&ws, need, s) != cudaSuccess) return AR_ERR_CUDA;
@@ -353,12 +432,39 @@ int ar_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, 
   float* rq = reinterpret_cast<float*>(w8 + 2 * vb);
   char* gbuf = w8 + 3 * vb;
   const long long rows = (long long)B * T * H;
+  const int pro = ra ? (ra->ve ? 3 : 1) : 0;
+
+  // the operands the backward kernels read: q, k, v themselves, or (RoPE path)
+  // the rotated q, k and mixed v the pre-pass writes after the G buffer
+  const void *qx = q, *kx = k, *vx = v;
+  if (ra) {
+    char* r8 = gbuf + g_heads_cap(B, T, H, grp) * g_head_bytes(T, (T + 127) / 128);
+    __nv_bfloat16* qr = reinterpret_cast<__nv_bfloat16*>(r8);
+    __nv_bfloat16* kr = reinterpret_cast<__nv_bfloat16*>(r8 + round_up((size_t)B * T * H * kD * 2, 256));
+    __nv_bfloat16* vm = kr + round_up((size_t)B * T * Hkv * kD * 2, 256) / 2;
+    const long long prows = rows + (long long)B * T * Hkv * (ra->ve ? 2 : 1);
+    KernelTimer t(AR_KERNEL_ROPE_PREP, s);
+    ar::rope_ve_prep_kernel<<<bwd_prep_grid(prows, sms, prep_blocks), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), ra->ve, ra->vg, ra->rcos, ra->rsin, qr, kr, vm, B, T, H, Hkv);
+    t.stop();
+    qx = qr;
+    kx = kr;
+    if (ra->ve) vx = vm;
+  }
+  CUtensorMap tq, tk, tv, tdo;
+  if (make_map(&tq, qx, B, T, H) != AR_OK || make_map(&tk, kx, B, T, Hkv) != AR_OK ||
+      make_map(&tv, vx, B, T, Hkv) != AR_OK || make_map(&tdo, dO, B, T, H) != AR_OK) {
+    if (!workspace) cudaFreeAsync(ws, s);
+    return AR_ERR_CUDA;
+  }
 
   {
     KernelTimer t(AR_KERNEL_BWD_PREP, s);
-    ar::bwd_prep_kernel<<<prep_grid(rows, sms), 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(o),
-        static_cast<const __nv_bfloat16*>(dO), lse, lse2, delta, rq, B, T, H, T_pad, eps);
+    ar::bwd_prep_kernel<<<bwd_prep_grid(rows, sms, prep_blocks), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(qx), static_cast<const __nv_bfloat16*>(o),
+        static_cast<const __nv_bfloat16*>(dO), lse, lse2, delta, rq, B, T, H, T_pad, eps,
+        aligned(qx, 32) && aligned(o, 32) && aligned(dO, 32));
     t.stop();
   }
   const int w = effective_window(window, T);
@@ -381,10 +487,16 @@ int ar_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, 
     ar::BwdParams p;
     p.dk = static_cast<__nv_bfloat16*>(dk);
     p.dv = static_cast<__nv_bfloat16*>(dv);
-    p.k = static_cast<const __nv_bfloat16*>(k);
+    p.k = static_cast<const __nv_bfloat16*>(kx);
     p.lse2 = lse2;
     p.delta = delta;
     p.rq = rq;
+    p.rcos = ra ? ra->rcos : nullptr;
+    p.rsin = ra ? ra->rsin : nullptr;
+    p.ve = ra ? ra->ve : nullptr;
+    p.vg = ra ? ra->vg : nullptr;
+    p.dve = ra ? ra->dve : nullptr;
+    p.dg = ra ? ra->dg : nullptr;
     p.B = B;
     p.T = T;
     p.H = H;
@@ -400,17 +512,25 @@ int ar_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, 
     p.pairs_head = (int)ph;
     p.eps = eps;
     p.scale = scale;
-    p.wide = aligned(dk, 32) && aligned(dv, 32);
-    p.wide_k = aligned(k, 32);
+    p.wide = aligned(dk, 32) && aligned(dv, 32) && (p.dve == nullptr || aligned(p.dve, 32));
+    p.wide_k = aligned(kx, 32);
+    p.wide_ve = p.ve != nullptr && aligned(p.ve, 32);
     p.wait_ns = g_wait_ns.load();
     {
       KernelTimer t(AR_KERNEL_BWD, s);
-      ar::bwd::bwd_kernel<<<std::min(p.n_units, sms), ar::bwd::kThreads, ar::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo,
-                                                                                                 tg, p);
+      const int grid = std::min(p.n_units, sms);
+      if (pro == 0)
+        ar::bwd::bwd_kernel<0><<<grid, ar::bwd::kThreads, ar::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo, tg, p);
+      else if (pro == 1)
+        ar::bwd::bwd_kernel<1><<<grid, ar::bwd::kThreads, ar::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo, tg, p);
+      else
+        ar::bwd::bwd_kernel<3><<<grid, ar::bwd::kThreads, ar::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo, tg, p);
       t.stop();
     }
     ar::DqParams d;
-    d.q = static_cast<const __nv_bfloat16*>(q);
+    d.q = static_cast<const __nv_bfloat16*>(qx);
+    d.rcos = p.rcos;
+    d.rsin = p.rsin;
     d.dq = static_cast<__nv_bfloat16*>(dq);
     d.B = B;
     d.T = T;
@@ -426,17 +546,78 @@ int ar_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, 
     d.eps = eps;
     d.scale = scale;
     d.wide = aligned(dq, 32);
-    d.wide_q = aligned(q, 32);
+    d.wide_q = aligned(qx, 32);
     d.wait_ns = p.wait_ns;
     {
       KernelTimer t(AR_KERNEL_DQ, s);
-      ar::dqk::dq_kernel<<<std::min(d.n_units, sms), ar::dqk::kThreads, ar::dqk::kSmemBytes, s>>>(tg, tk, d);
+      const int grid = std::min(d.n_units, sms);
+      if (ra)
+        ar::dqk::dq_kernel<true><<<grid, ar::dqk::kThreads, ar::dqk::kSmemBytes, s>>>(tg, tk, d);
+      else
+        ar::dqk::dq_kernel<false><<<grid, ar::dqk::kThreads, ar::dqk::kSmemBytes, s>>>(tg, tk, d);
       t.stop();
     }
   }
   cudaError_t e = cudaGetLastError();
   if (!workspace) cudaFreeAsync(ws, s);
   return e == cudaSuccess ? AR_OK : AR_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ar_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                    void* dq, void* dk, void* dv, int B, int T, int H, int Hkv, int D, int window, float eps,
+                    float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return AR_ERR_NULL;
+  int st = check_shape(B, T, H, D);
+  if (st != AR_OK) return st;
+  if ((st = check_kv_heads(H, Hkv)) != AR_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
+    return AR_ERR_ALIGN;
+  if ((st = check_args(eps, scale)) != AR_OK) return st;
+  const size_t need = ar_attn_bwd_gqa_workspace_bytes(B, T, H, Hkv, D);
+  if (workspace && workspace_bytes < need) return AR_ERR_WORKSPACE;
+  if (workspace && !aligned(workspace, 256)) return AR_ERR_ALIGN;
+  return bwd_run(q, k, v, o, dO, lse, dq, dk, dv, B, T, H, Hkv, window, eps, scale, workspace, need, stream, nullptr);
+}
+
+size_t ar_attn_bwd_rope_workspace_bytes(int B, int T, int H, int Hkv, int D, int with_ve) {
+  const size_t base = ar_attn_bwd_gqa_workspace_bytes(B, T, H, Hkv, D);
+  return base ? base + rope_bytes(B, T, H, Hkv, with_ve != 0) : 0;
+}
+
+int ar_attn_bwd_rope(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                     const void* rope_cos, const void* rope_sin, int rope_rows, const void* ve, const void* ve_gate,
+                     void* dq, void* dk, void* dv, void* dve, float* dgate, int B, int T, int H, int Hkv, int D,
+                     int window, float eps, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !rope_cos || !rope_sin) return AR_ERR_NULL;
+  const bool with_ve = ve != nullptr;
+  if (with_ve && (!ve_gate || !dve || !dgate)) return AR_ERR_NULL;
+  if (!with_ve && (ve_gate || dve || dgate)) return AR_ERR_NULL;
+  int st = check_shape(B, T, H, D);
+  if (st != AR_OK) return st;
+  if ((st = check_kv_heads(H, Hkv)) != AR_OK) return st;
+  if (rope_rows < T) return AR_ERR_SHAPE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(rope_cos, 16) ||
+      !aligned(rope_sin, 16) || !aligned(ve, 16) || !aligned(ve_gate, 2) || !aligned(dve, 16) ||
+      !aligned(dgate, 4))
+    return AR_ERR_ALIGN;
+  if ((st = check_args(eps, scale)) != AR_OK) return st;
+  const size_t need = ar_attn_bwd_rope_workspace_bytes(B, T, H, Hkv, D, with_ve);
+  if (workspace && workspace_bytes < need) return AR_ERR_WORKSPACE;
+  if (workspace && !aligned(workspace, 256)) return AR_ERR_ALIGN;
+  RopeArgs ra;
+  ra.rcos = static_cast<const __nv_bfloat16*>(rope_cos);
+  ra.rsin = static_cast<const __nv_bfloat16*>(rope_sin);
+  ra.ve = static_cast<const __nv_bfloat16*>(ve);
+  ra.vg = static_cast<const __nv_bfloat16*>(ve_gate);
+  ra.dve = static_cast<__nv_bfloat16*>(dve);
+  ra.dg = dgate;
+  return bwd_run(q, k, v, o, dO, lse, dq, dk, dv, B, T, H, Hkv, window, eps, scale, workspace, need, stream, &ra);
 }
 
 int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
@@ -507,8 +688,8 @@ int ar_attn_timing_enable(int on) {
 
 int ar_attn_timing_read(double* ms, long long* count) {
   std::lock_guard<std::mutex> lock(g_timing.mu);
-  double acc[AR_KERNEL_KINDS] = {0, 0, 0, 0, 0};
-  long long n[AR_KERNEL_KINDS] = {0, 0, 0, 0, 0};
+  double acc[AR_KERNEL_KINDS] = {};
+  long long n[AR_KERNEL_KINDS] = {};
   int st = AR_OK;
   for (auto& r : g_timing.recs) {
     float t = 0.f;

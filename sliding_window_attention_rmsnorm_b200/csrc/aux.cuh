@@ -3,6 +3,7 @@
 //
 //   fwd_prep  : ck[bh, t] = rk_t * scale * log2(e), rk_t = 1/sqrt(mean_d k_td^2 + eps)
 //   bwd_prep  : delta[bh, t] = sum_d dO_td o_td  (FlashAttention's backward pre-pass),
+//               read 8 lanes to a row with 256-bit loads,
 //               rq[bh, t]    = 1/sqrt(mean_d q_td^2 + eps),
 //               lse2[bh, t]  = lse[bh, t] * log2(e)
 // The [B*H, T_pad] vectors are zero on the padding t >= T so that every tile
@@ -71,27 +72,50 @@ __global__ void fwd_prep_kernel(const __nv_bfloat16* __restrict__ k, float* __re
   }
 }
 
+// c += sum over the 8 bf16 pairs of a and b of a_k * b_k (products exact in
+// f32, one rounding per fma; the bf16 halves are read directly).
+__device__ __forceinline__ void dot_bf16x8_f32(float& c0, float& c1, const uint4& a, const uint4& b) {
+  const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    asm("{\n .reg .b16 al, ah, bl, bh;\n mov.b32 {al, ah}, %2;\n mov.b32 {bl, bh}, %3;\n"
+        " fma.rn.f32.bf16 %0, al, bl, %0;\n fma.rn.f32.bf16 %1, ah, bh, %1;\n}"
+        : "+f"(c0), "+f"(c1)
+        : "r"(wa[e]), "r"(wb[e]));
+}
+
+// One row (one token of one head, 128 elements) per 8 lanes, 32 bytes of each
+// of q, o and dO per lane: 256-bit loads when the tensors are 32-byte aligned.
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ o,
                                 const __nv_bfloat16* __restrict__ dO, const float* __restrict__ lse,
                                 float* __restrict__ lse2, float* __restrict__ delta, float* __restrict__ rq, int B,
-                                int T, int H, int T_pad, float eps) {
+                                int T, int H, int T_pad, float eps, int wide) {
   const long long rows = (long long)B * T * H;
-  const int sub = threadIdx.x & 15;
-  const long long gstride = (long long)gridDim.x * (blockDim.x / 16);
+  const int sub = threadIdx.x & 7;
+  const long long gstride = (long long)gridDim.x * (blockDim.x / 8);
   const float kLog2e = 1.4426950408889634f;
-  for (long long r = (long long)blockIdx.x * (blockDim.x / 16) + threadIdx.x / 16; r < rows; r += gstride) {
-    float fq[8], fo[8], fd[8];
-    unpack8(__ldg(reinterpret_cast<const uint4*>(q + r * 128) + sub), fq);
-    unpack8(__ldg(reinterpret_cast<const uint4*>(o + r * 128) + sub), fo);
-    unpack8(__ldg(reinterpret_cast<const uint4*>(dO + r * 128) + sub), fd);
-    float ss = 0.f, dl = 0.f;
+  for (long long r = (long long)blockIdx.x * (blockDim.x / 8) + threadIdx.x / 8; r < rows; r += gstride) {
+    uint4 q0, q1, o0, o1, d0, d1;
+    ldg32B(q + r * 128 + sub * 16, q0, q1, wide);
+    ldg32B(o + r * 128 + sub * 16, o0, o1, wide);
+    ldg32B(dO + r * 128 + sub * 16, d0, d1, wide);
+    float s0 = 0.f, s1 = 0.f, t0 = 0.f, t1 = 0.f;
+    fma_sq_bf16x2_f32(s0, s1, q0.x);
+    fma_sq_bf16x2_f32(s0, s1, q0.y);
+    fma_sq_bf16x2_f32(s0, s1, q0.z);
+    fma_sq_bf16x2_f32(s0, s1, q0.w);
+    fma_sq_bf16x2_f32(s0, s1, q1.x);
+    fma_sq_bf16x2_f32(s0, s1, q1.y);
+    fma_sq_bf16x2_f32(s0, s1, q1.z);
+    fma_sq_bf16x2_f32(s0, s1, q1.w);
+    dot_bf16x8_f32(t0, t1, o0, d0);
+    dot_bf16x8_f32(t0, t1, o1, d1);
+    float ss = s0 + s1, dl = t0 + t1;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      ss = fmaf(fq[e], fq[e], ss);
-      dl = fmaf(fo[e], fd[e], dl);
+    for (int m = 4; m > 0; m >>= 1) {
+      ss += __shfl_xor_sync(0xffffffffu, ss, m);
+      dl += __shfl_xor_sync(0xffffffffu, dl, m);
     }
-    ss = half_warp_sum(ss);
-    dl = half_warp_sum(dl);
     if (sub == 0) {
       int b, t, h;
       split_row(r, T, H, b, t, h);
@@ -108,6 +132,60 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_
     delta[bh * T_pad + t] = 0.f;
     rq[bh * T_pad + t] = 0.f;
     lse2[bh * T_pad + t] = 0.f;
+  }
+}
+
+// The backward's pre-pass of the RoPE / value-embedding path: the rotated q
+// and k and the mixed v that the forward formed in its tiles, written out for
+// the backward kernels (the same arithmetic, so the same bf16 values).  Rows
+// [0, nq) are q rows [B, T, H], then nk k rows and nk v rows [B, T, Hkv]; one
+// row per 8 lanes.  RoPE: lane l rotates features 8l .. 8l+7 with their
+// partners 64 + 8l ..; value embedding (only when ve is given): lane l mixes
+// features 16l .. 16l+15.
+__global__ void rope_ve_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                                    const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ ve,
+                                    const __nv_bfloat16* __restrict__ vg, const __nv_bfloat16* __restrict__ rcos,
+                                    const __nv_bfloat16* __restrict__ rsin, __nv_bfloat16* __restrict__ qr,
+                                    __nv_bfloat16* __restrict__ kr, __nv_bfloat16* __restrict__ vm, int B, int T,
+                                    int H, int Hkv) {
+  const long long nq = (long long)B * T * H, nk = (long long)B * T * Hkv, rows = nq + nk + (ve ? nk : 0);
+  const int sub = threadIdx.x & 7;
+  const long long gstride = (long long)gridDim.x * (blockDim.x / 8);
+  for (long long r = (long long)blockIdx.x * (blockDim.x / 8) + threadIdx.x / 8; r < rows; r += gstride) {
+    if (r < nq + nk) {
+      const bool isq = r < nq;
+      const long long rr = isq ? r : r - nq;
+      const int t = (int)((rr / (isq ? H : Hkv)) % T);
+      const __nv_bfloat16* src = (isq ? q : k) + rr * 128;
+      __nv_bfloat16* dst = (isq ? qr : kr) + rr * 128;
+      const uint4 x1 = __ldg(reinterpret_cast<const uint4*>(src + 8 * sub));
+      const uint4 x2 = __ldg(reinterpret_cast<const uint4*>(src + 64 + 8 * sub));
+      const uint4 c = __ldg(reinterpret_cast<const uint4*>(rcos + (size_t)t * 64 + 8 * sub));
+      const uint4 sn = __ldg(reinterpret_cast<const uint4*>(rsin + (size_t)t * 64 + 8 * sub));
+      uint4 y1, y2;
+      rope_word(x1.x, x2.x, c.x, sn.x, y1.x, y2.x);
+      rope_word(x1.y, x2.y, c.y, sn.y, y1.y, y2.y);
+      rope_word(x1.z, x2.z, c.z, sn.z, y1.z, y2.z);
+      rope_word(x1.w, x2.w, c.w, sn.w, y1.w, y2.w);
+      *reinterpret_cast<uint4*>(dst + 8 * sub) = y1;
+      *reinterpret_cast<uint4*>(dst + 64 + 8 * sub) = y2;
+    } else {
+      const long long rr = r - nq - nk;
+      const uint4* src = reinterpret_cast<const uint4*>(v + rr * 128 + 16 * sub);
+      uint4* dst = reinterpret_cast<uint4*>(vm + rr * 128 + 16 * sub);
+      uint4 a = __ldg(src), b = __ldg(src + 1);
+      if (ve) {
+        const float gate = ve_gate(vg[rr]);
+        const uint4* e = reinterpret_cast<const uint4*>(ve + rr * 128 + 16 * sub);
+        const uint4 ea = __ldg(e), eb = __ldg(e + 1);
+        a = make_uint4(ve_mix_word(a.x, ea.x, gate), ve_mix_word(a.y, ea.y, gate), ve_mix_word(a.z, ea.z, gate),
+                       ve_mix_word(a.w, ea.w, gate));
+        b = make_uint4(ve_mix_word(b.x, eb.x, gate), ve_mix_word(b.y, eb.y, gate), ve_mix_word(b.z, eb.z, gate),
+                       ve_mix_word(b.w, eb.w, gate));
+      }
+      dst[0] = a;
+      dst[1] = b;
+    }
   }
 }
 

@@ -36,6 +36,14 @@
 // dP_0 | dP_1 (64 each) | dV (128) | dK (128).
 // Shared memory: K, V, Q[2], dO[2], G^T (all 128x128 bf16, 128-byte swizzled,
 // G^T half a = query columns 64a..64a+63), plus per-half query vectors.
+//
+// With the RoPE / value-embedding prologue (kPro != 0) the tensor maps and p.k
+// point at the rotated q, k and the mixed v that the pre-pass wrote (the same
+// bf16 values the forward formed in its tiles), and the epilogue finishes the
+// chain rule: dk = R_j^T dk_rot (the transposed rotation of the key's position:
+// dk1 = d1 cos - d2 sin, dk2 = d1 sin + d2 cos for the halves d1, d2), and for
+// the value embedding v_mix = v + gate ve, gate = 2 sigmoid(g): dv = dv_mix,
+// dve = gate dv_mix, dg = (dv_mix . ve) gate (1 - gate / 2).
 #pragma once
 #include "sm100.cuh"
 
@@ -48,6 +56,12 @@ struct BwdParams {
   const float* lse2;       // [B*H, T_pad] lse * log2(e), 0 on padding
   const float* delta;      // [B*H, T_pad] rowsum(dO * o), 0 on padding
   const float* rq;         // [B*H, T_pad] 1/rms(q_i), 0 on padding
+  const __nv_bfloat16* rcos;  // kPro & 1: rotary tables [>= T, 64], row t = position t
+  const __nv_bfloat16* rsin;
+  const __nv_bfloat16* ve;    // kPro & 2: value embedding [B, T, Hkv, 128] and gate logits [B, T, Hkv]
+  const __nv_bfloat16* vg;
+  __nv_bfloat16* dve;         // kPro & 2: outputs [B, T, Hkv, 128] and [B, T, Hkv]
+  float* dg;
   int B, T, H, T_pad;
   int Hkv, grp;  // K/V heads and query heads per K/V head (H = Hkv * grp; grp = 1: multi-head)
   int w;        // left window (w >= T means full causal)
@@ -59,6 +73,7 @@ struct BwdParams {
   float eps, scale;
   int wide;    // dk and dv are 32-byte aligned: rows are written with 256-bit stores
   int wide_k;  // k is 32-byte aligned: key rows are read with 256-bit loads
+  int wide_ve;  // ve is 32-byte aligned
   unsigned long long wait_ns;  // limit of a device-side wait (kWaitLimitNs unless set otherwise)
 };
 
@@ -163,10 +178,12 @@ __device__ __forceinline__ void grad_chunk(const uint32_t (&sv)[32], const uint3
   }
 }
 
+template <int kPro>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                const __grid_constant__ CUtensorMap tm_g, const BwdParams p) {
+  constexpr bool kRope = (kPro & 1) != 0, kVe = (kPro & 2) != 0;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
@@ -497,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // dk = scale (acc - coef k), coef = rk^2 (acc . k) / D, with acc . k summed by
         // the compute warpgroups as sum_i G_ij S_ij; the raw key row is loaded into
         // registers before the wait, so its latency is hidden by the unit's products
-        {
+        if constexpr (!kRope) {
           uint4 kv[16];
           {
             const uint4* krow = reinterpret_cast<const uint4*>(p.k + orow);
@@ -537,19 +554,104 @@ __global__ void __launch_bounds__(kThreads, 1)
               stg32B(p.dk + orow + 32 * c + 16, pk + 8, p.wide);
             }
           }
-        }
+        } else {
+          // dk_rot = scale (acc - coef k_rot), then dk = R_j^T dk_rot: features
+          // 16c .. 16c+15 with their partners 64 + 16c .., the rotated key row and
+          // the table entries read as needed (L2)
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DKDVDONE), uidx & 1, abort_flag, p.wait_ns))) break;
+          tc_fence_after();
+          const float coef = lds_f32(sbase + kDot + 4 * row) + lds_f32(sbase + kDot + 4 * (128 + row));
+          mbar_arrive(bar_addr(sbase, DOTFREE));
+          const __nv_bfloat16* cr = p.rcos + (size_t)(jv ? j : 0) * 64;
+          const __nv_bfloat16* sr = p.rsin + (size_t)(jv ? j : 0) * 64;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t x[32];
-          tmem_ld32(tDV + 32 * c, x);
-          tmem_wait_ld();
-          uint32_t pk[16];
+          for (int c = 0; c < 4; ++c) {
+            uint32_t xl[16], xh[16];
+            tmem_ld16(tDK + 16 * c, xl);
+            tmem_ld16(tDK + 64 + 16 * c, xh);
+            uint4 kl[2], kh[2], cc[2], sc[2];
+            if (jv) {
+              ldg32B(p.k + orow + 16 * c, kl[0], kl[1], p.wide_k);
+              ldg32B(p.k + orow + 64 + 16 * c, kh[0], kh[1], p.wide_k);
+              cc[0] = __ldg(reinterpret_cast<const uint4*>(cr + 16 * c));
+              cc[1] = __ldg(reinterpret_cast<const uint4*>(cr + 16 * c + 8));
+              sc[0] = __ldg(reinterpret_cast<const uint4*>(sr + 16 * c));
+              sc[1] = __ldg(reinterpret_cast<const uint4*>(sr + 16 * c + 8));
+            } else {
+              kl[0] = kl[1] = kh[0] = kh[1] = cc[0] = cc[1] = sc[0] = sc[1] = make_uint4(0, 0, 0, 0);
+            }
+            tmem_wait_ld();
+            uint32_t pl[8], ph[8];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]));
-          if (jv) {
-            stg32B(p.dv + orow + 32 * c, pk, p.wide);
-            stg32B(p.dv + orow + 32 * c + 16, pk + 8, p.wide);
+            for (int e = 0; e < 8; ++e) {
+              const uint4& a = kl[e >> 2];
+              const uint4& b = kh[e >> 2];
+              const uint4& cv = cc[e >> 2];
+              const uint4& sv = sc[e >> 2];
+              const uint32_t kw1 = (&a.x)[e & 3], kw2 = (&b.x)[e & 3], cw = (&cv.x)[e & 3], sw = (&sv.x)[e & 3];
+              const float d10 = p.scale * (__uint_as_float(xl[2 * e]) - coef * bf16lo(kw1));
+              const float d11 = p.scale * (__uint_as_float(xl[2 * e + 1]) - coef * bf16hi(kw1));
+              const float d20 = p.scale * (__uint_as_float(xh[2 * e]) - coef * bf16lo(kw2));
+              const float d21 = p.scale * (__uint_as_float(xh[2 * e + 1]) - coef * bf16hi(kw2));
+              const float c0 = bf16lo(cw), c1 = bf16hi(cw), s0 = bf16lo(sw), s1 = bf16hi(sw);
+              pl[e] = pack_bf16(fmaf(d10, c0, -(d20 * s0)), fmaf(d11, c1, -(d21 * s1)));
+              ph[e] = pack_bf16(fmaf(d10, s0, d20 * c0), fmaf(d11, s1, d21 * c1));
+            }
+            if (jv) {
+              stg32B(p.dk + orow + 16 * c, pl, p.wide);
+              stg32B(p.dk + orow + 64 + 16 * c, ph, p.wide);
+            }
           }
+        }
+        if constexpr (!kVe) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t x[32];
+            tmem_ld32(tDV + 32 * c, x);
+            tmem_wait_ld();
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]));
+            if (jv) {
+              stg32B(p.dv + orow + 32 * c, pk, p.wide);
+              stg32B(p.dv + orow + 32 * c + 16, pk + 8, p.wide);
+            }
+          }
+        } else {
+          // dv = dv_mix, dve = gate dv_mix, dg = (dv_mix . ve) gate (1 - gate / 2)
+          const size_t tok = ((size_t)U.b * p.T + (jv ? j : 0)) * p.Hkv + U.h;
+          const float gate = jv ? ve_gate(p.vg[tok]) : 0.f;
+          float dot0 = 0.f, dot1 = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t x[32];
+            tmem_ld32(tDV + 32 * c, x);
+            uint4 ev[4];
+            if (jv) {
+              ldg32B(p.ve + orow + 32 * c, ev[0], ev[1], p.wide_ve);
+              ldg32B(p.ve + orow + 32 * c + 16, ev[2], ev[3], p.wide_ve);
+            } else {
+              ev[0] = ev[1] = ev[2] = ev[3] = make_uint4(0, 0, 0, 0);
+            }
+            tmem_wait_ld();
+            uint32_t pk[16], pe[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float x0 = __uint_as_float(x[2 * e]), x1 = __uint_as_float(x[2 * e + 1]);
+              const uint32_t ew = (&ev[e >> 2].x)[e & 3];
+              pk[e] = pack_bf16(x0, x1);
+              pe[e] = pack_bf16(gate * x0, gate * x1);
+              dot0 = fmaf(x0, bf16lo(ew), dot0);
+              dot1 = fmaf(x1, bf16hi(ew), dot1);
+            }
+            if (jv) {
+              stg32B(p.dv + orow + 32 * c, pk, p.wide);
+              stg32B(p.dv + orow + 32 * c + 16, pk + 8, p.wide);
+              stg32B(p.dve + orow + 32 * c, pe, p.wide);
+              stg32B(p.dve + orow + 32 * c + 16, pe + 8, p.wide);
+            }
+          }
+          if (jv) p.dg[tok] = (dot0 + dot1) * gate * (1.0f - 0.5f * gate);
         }
         tc_fence_before();
         mbar_arrive(bar_addr(sbase, ACCFREE));

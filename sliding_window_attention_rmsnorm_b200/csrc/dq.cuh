@@ -21,6 +21,10 @@
 //   warp 4     TMA producer of the G tiles (two 64-query halves each; 4 stages)
 //   warp 5     MMA issuer
 //   warp 6     TMA producer of the K tiles (3 stages)
+// With the RoPE prologue (kRope) the K tiles and p.q are the rotated k and q
+// the backward's pre-pass wrote, and the epilogue ends with the transposed
+// rotation of the query's position: dq = R_i^T dq_rot (dq1 = d1 cos - d2 sin,
+// dq2 = d1 sin + d2 cos for the halves d1, d2).
 // TMEM (512 columns): four 128-column accumulators, one per unit in flight, so
 // the epilogues of short units overlap the next units' products.  The product
 // is acc (M = 128 queries, N = 128 features, K = 16 keys per step) with A = G
@@ -33,6 +37,8 @@ namespace ar {
 
 struct DqParams {
   const __nv_bfloat16* q;  // [B, T, H, 128]
+  const __nv_bfloat16* rcos;  // kRope: rotary tables [>= T, 64], row t = position t
+  const __nv_bfloat16* rsin;
   __nv_bfloat16* dq;       // [B, T, H, 128]
   int B, T, H;
   int grp;         // query heads per K/V head: k has H / grp heads (1: multi-head)
@@ -95,6 +101,7 @@ __device__ __forceinline__ long long g_slot(const DqParams& p, int hl, int qt, i
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t sbase, int i) { return sbase + kBar + 8u * i; }
 
+template <bool kRope>
 __global__ void __launch_bounds__(kThreads, 1)
     dq_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_k, const DqParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -256,27 +263,67 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const float coef = dot * (1.0f / 128.0f) / (ss * (1.0f / 128.0f) + p.eps);
-        // pass 2: dq = scale (acc - coef q)
+        if constexpr (!kRope) {
+          // pass 2: dq = scale (acc - coef q)
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t x[32];
-          tmem_ld32(tA + 32 * cc, x);
-          tmem_wait_ld();
-          uint32_t pk[16];
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t x[32];
+            tmem_ld32(tA + 32 * cc, x);
+            tmem_wait_ld();
+            uint32_t pk[16];
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const uint4 v = qv[4 * cc + q4];
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const uint4 v = qv[4 * cc + q4];
+              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float g0 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e]) - coef * bf16lo(w4[e]));
-              const float g1 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e + 1]) - coef * bf16hi(w4[e]));
-              pk[4 * q4 + e] = pack_bf16(g0, g1);
+              for (int e = 0; e < 4; ++e) {
+                const float g0 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e]) - coef * bf16lo(w4[e]));
+                const float g1 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e + 1]) - coef * bf16hi(w4[e]));
+                pk[4 * q4 + e] = pack_bf16(g0, g1);
+              }
+            }
+            if (iv) {
+              stg32B(p.dq + orow + 32 * cc, pk, p.wide);
+              stg32B(p.dq + orow + 32 * cc + 16, pk + 8, p.wide);
             }
           }
-          if (iv) {
-            stg32B(p.dq + orow + 32 * cc, pk, p.wide);
-            stg32B(p.dq + orow + 32 * cc + 16, pk + 8, p.wide);
+        } else {
+          // pass 2: dq_rot = scale (acc - coef q_rot), then dq = R_i^T dq_rot, for
+          // features 16c .. 16c+15 with their partners 64 + 16c ..
+          const __nv_bfloat16* cr = p.rcos + (size_t)(iv ? i : 0) * 64;
+          const __nv_bfloat16* sr = p.rsin + (size_t)(iv ? i : 0) * 64;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {  // unrolled: qv is indexed by c
+            uint32_t xl[16], xh[16];
+            tmem_ld16(tA + 16 * c, xl);
+            tmem_ld16(tA + 64 + 16 * c, xh);
+            uint4 cv[2], sv[2];
+            if (iv) {
+              cv[0] = __ldg(reinterpret_cast<const uint4*>(cr + 16 * c));
+              cv[1] = __ldg(reinterpret_cast<const uint4*>(cr + 16 * c + 8));
+              sv[0] = __ldg(reinterpret_cast<const uint4*>(sr + 16 * c));
+              sv[1] = __ldg(reinterpret_cast<const uint4*>(sr + 16 * c + 8));
+            } else {
+              cv[0] = cv[1] = sv[0] = sv[1] = make_uint4(0, 0, 0, 0);
+            }
+            tmem_wait_ld();
+            uint32_t pl[8], ph[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const uint32_t q1 = (&qv[2 * c + (e >> 2)].x)[e & 3], q2 = (&qv[8 + 2 * c + (e >> 2)].x)[e & 3];
+              const uint32_t cw = (&cv[e >> 2].x)[e & 3], sw = (&sv[e >> 2].x)[e & 3];
+              const float d10 = p.scale * (__uint_as_float(xl[2 * e]) - coef * bf16lo(q1));
+              const float d11 = p.scale * (__uint_as_float(xl[2 * e + 1]) - coef * bf16hi(q1));
+              const float d20 = p.scale * (__uint_as_float(xh[2 * e]) - coef * bf16lo(q2));
+              const float d21 = p.scale * (__uint_as_float(xh[2 * e + 1]) - coef * bf16hi(q2));
+              const float c0 = bf16lo(cw), c1 = bf16hi(cw), s0 = bf16lo(sw), s1 = bf16hi(sw);
+              pl[e] = pack_bf16(fmaf(d10, c0, -(d20 * s0)), fmaf(d11, c1, -(d21 * s1)));
+              ph[e] = pack_bf16(fmaf(d10, s0, d20 * c0), fmaf(d11, s1, d21 * c1));
+            }
+            if (iv) {
+              stg32B(p.dq + orow + 16 * c, pl, p.wide);
+              stg32B(p.dq + orow + 64 + 16 * c, ph, p.wide);
+            }
           }
         }
       }

@@ -340,6 +340,26 @@ __device__ __forceinline__ void fma_sq_bf16x2_f32(float& c0, float& c1, uint32_t
       : "r"(u));
 }
 
+// ------------------------------------------------------------------ RoPE / value embedding
+// The arithmetic of the two steps before the attention core, shared by the
+// forward's in-tile prologue and the backward's pre-pass so that both produce
+// the same bf16 values.
+// y1 = x1 c + x2 s, y2 = x2 c - x1 s for the bf16 pairs of one word of each
+// half of a row (x1: features d, x2: features d + 64; c, s: the table entries).
+__device__ __forceinline__ void rope_word(uint32_t x1, uint32_t x2, uint32_t c, uint32_t s, uint32_t& y1,
+                                          uint32_t& y2) {
+  const float a0 = bf16lo(x1), a1 = bf16hi(x1), b0 = bf16lo(x2), b1 = bf16hi(x2);
+  const float c0 = bf16lo(c), c1 = bf16hi(c), s0 = bf16lo(s), s1 = bf16hi(s);
+  y1 = pack_bf16(fmaf(a0, c0, b0 * s0), fmaf(a1, c1, b1 * s1));
+  y2 = pack_bf16(fmaf(b0, c0, -(a0 * s0)), fmaf(b1, c1, -(a1 * s1)));
+}
+// The value-embedding gate 2 sigmoid(g) of a bf16 gate logit.
+__device__ __forceinline__ float ve_gate(__nv_bfloat16 g) { return 2.0f / (1.0f + __expf(-__bfloat162float(g))); }
+// v + gate * ve for the bf16 pairs of one word.
+__device__ __forceinline__ uint32_t ve_mix_word(uint32_t v, uint32_t e, float gate) {
+  return pack_bf16(fmaf(gate, bf16lo(e), bf16lo(v)), fmaf(gate, bf16hi(e), bf16hi(v)));
+}
+
 // 32 bytes (w[0..7]) to global memory at dst: one 256-bit store when `wide`
 // (dst 32-byte aligned), else two 128-bit stores (dst 16-byte aligned).  A warp
 // whose lanes each write a different row touches one 32-byte sector per lane

@@ -8,11 +8,13 @@ rounded to bf16, so every consumer sees the same bits.  The pages train on
 tokenised web text; the core itself only ever sees q, k, v and dO, whose
 statistics after the QK norm are what matters, hence Gaussian stand-ins.
 
-Seed of one tensor: 1000 * config + 10 * layer + {q: 0, k: 1, v: 2, dO: 3}.
+Seed of one tensor: 1000 * config + 10 * layer + {q: 0, k: 1, v: 2, dO: 3, ve: 4,
+g: 5}; ve is a value embedding [B, T, Hkv, D] and g the gate logits [B, T, Hkv]
+of the layers that mix one in (N(0,1) like the rest).
 """
 import torch
 
-_ROLE = {"q": 0, "k": 1, "v": 2, "dO": 3}
+_ROLE = {"q": 0, "k": 1, "v": 2, "dO": 3, "ve": 4, "g": 5}
 
 
 def seed_of(config: int, layer: int, role: str) -> int:
@@ -37,3 +39,9 @@ def peaked_keys(q: torch.Tensor, seed: int, noise: float = 0.1) -> torch.Tensor:
     towards their bound; a stress input, bf16."""
     n = normal_bf16(tuple(q.shape), seed).float()
     return (q.float() + noise * n).to(torch.bfloat16)
+
+
+def value_embedding(config: int, layer: int, B: int, T: int, Hkv: int, D: int):
+    """(ve [B, T, Hkv, D], g [B, T, Hkv]) bf16 CPU tensors, seeded like the rest."""
+    return (normal_bf16((B, T, Hkv, D), seed_of(config, layer, "ve")),
+            normal_bf16((B, T, Hkv), seed_of(config, layer, "g")))

@@ -157,3 +157,29 @@ def test_gate_limits():
     # gate 2 sigmoid(0) = 1 with ve = -v cancels the values: o = 0
     o_zero, _ = rope_ve.attn_fwd(q, k, v, cos, sin, w, ve=-v, g=np.zeros((B, T, H)))
     np.testing.assert_allclose(o_zero, 0.0, atol=1e-13)
+
+
+def test_bf16_round_matches_torch():
+    x = rand(5000, 40) * np.exp(rand(5000, 41) * 5)
+    x32 = x.astype(np.float32).astype(np.float64)
+    ref = torch.tensor(x32, dtype=torch.float32).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(rope_ve.bf16_round(x32), ref)
+
+
+def test_rounded_operands_only_change_the_operands():
+    """With round_operands the core sees the rounded rotated q, k (and mixed v):
+    identity rounding gives the exact result, and the forward on rounded
+    operands is the plain oracle on those operands."""
+    from oracle import oracle as orc
+    B, T, H, D, w = 1, 30, 2, 16, 7
+    q, k, v, ve = (rand((B, T, H, D), 50 + i) for i in range(4))
+    g = rand((B, T, H), 55)
+    cos, sin = rope_ve.rope_tables(T, D)
+    o1, l1 = rope_ve.attn_fwd(q, k, v, cos, sin, w, ve=ve, g=g, round_operands=lambda a: a)
+    o2, l2 = rope_ve.attn_fwd(q, k, v, cos, sin, w, ve=ve, g=g)
+    np.testing.assert_array_equal(o1, o2)
+    r = rope_ve.bf16_round
+    o3, _ = rope_ve.attn_fwd(q, k, v, cos, sin, w, ve=ve, g=g, round_operands=r)
+    o4, _ = orc.attn_fwd(r(rope_ve.rope(q, cos, sin)), r(rope_ve.rope(k, cos, sin)), r(rope_ve.mix_value(v, ve, g)), w)
+    np.testing.assert_array_equal(o3, o4)
+    assert np.abs(o3 - o2).max() > 0
