@@ -52,6 +52,9 @@ WORKLOADS = {
     "stack8_rope": dict(config=3, B=8, T=2048, H=4, n_layer=8, pattern="SSSL", rope=True,
                         name="8-layer SSSL attention stack fwd+bwd with fused RoPE and value embeddings, "
                              "B=8 T=2048 H=4 D=128 (windows 1024/full)"),
+    "layer_s_rope": dict(config=2, B=8, T=2048, H=4, n_layer=1, windows=[1024], rope=True,
+                         name="single S layer fwd+bwd with fused RoPE and value embedding, B=8 T=2048 H=4 D=128, "
+                              "window 1024"),
     # grouped K/V heads (n_kv_head = n_head / 2): not one of the stated workloads
     "stack8_gqa": dict(config=3, B=8, T=2048, H=4, Hkv=2, n_layer=8, pattern="SSSL",
                        name="8-layer SSSL attention stack fwd+bwd, B=8 T=2048 H=4 Hkv=2 D=128 (windows 1024/full)"),
@@ -394,20 +397,44 @@ def run_ours(args, wl, rank, world, dist):
             kernels[k]["gbs"] = by * kern[k][1] / (kern[k][0] * 1e-3) / 1e9
             kernels[k]["hbm_frac"] = kernels[k]["gbs"] / peaks["hbm"]
 
-    # end to end: inputs from pinned host memory, results back to host, all inside the timed region
+    # End to end: inputs from pinned host memory, results back to host, all inside
+    # the timed region.  The copies run on their own streams, layer by layer: the
+    # inputs of layer l+1 cross while layer l's forward runs, each layer's o as
+    # soon as the forwards are done, and each layer's gradients while the next
+    # (lower) layer's backward runs; the step ends when its last result is on the host.
     e2e = None
     if not args.no_e2e:
         pinned = [{r: t.pin_memory() for r, t in x.items()} for x in host]
+        out_names = [[n for n in ("o", "dq", "dk", "dv", "dve", "dg") if n in st.out[l]] for l in range(L)]
         outs_h = [{n: torch.empty(st.out[l][n].shape, dtype=st.out[l][n].dtype, pin_memory=True)
-                   for n in ("o", "dq", "dk", "dv")} for l in range(L)]
+                   for n in out_names[l]} for l in range(L)]
+        h2d_stream, d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
+
         def e2e_step():
+            h2d_stream.wait_stream(stream)  # the previous step is done with the device buffers
+            ev_in = []
+            with torch.cuda.stream(h2d_stream):
+                for l in range(L):
+                    for r, t in pinned[l].items():
+                        layers[l][r].copy_(t, non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(h2d_stream)
+                    ev_in.append(ev)
             for l in range(L):
-                for r in ("q", "k", "v", "dO"):
-                    layers[l][r].copy_(pinned[l][r], non_blocking=True)
-            st.step()
-            for l in range(L):
-                for n in ("o", "dq", "dk", "dv"):
-                    outs_h[l][n].copy_(st.out[l][n], non_blocking=True)
+                stream.wait_event(ev_in[l])
+                st.forward_layer(l)
+            d2h_stream.wait_stream(stream)
+            with torch.cuda.stream(d2h_stream):
+                for l in range(L):
+                    outs_h[l]["o"].copy_(st.out[l]["o"], non_blocking=True)
+            for l in reversed(range(L)):
+                st.backward_layer(l)
+                d2h_stream.wait_stream(stream)
+                with torch.cuda.stream(d2h_stream):
+                    for n in out_names[l]:
+                        if n != "o":
+                            outs_h[l][n].copy_(st.out[l][n], non_blocking=True)
+            stream.wait_stream(d2h_stream)
         e2e_step()
         torch.cuda.synchronize()
         barrier()

@@ -122,23 +122,30 @@ int ar_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, 
                     int B, int T, int H, int Hkv, int D, int window, float eps, float scale,
                     void* workspace, size_t workspace_bytes, void* stream);
 
-/* The forward with the two steps the pages run just before the core fused
- * into its tile loads ("autoresearch" README (gitee), section 7.4: rotary
- * position embedding of q and k; section 5.2.3: the value embedding mixed
- * into v on the layers that have one).  q, k, v are the unrotated, unmixed
- * tensors; the kernel rotates each Q and K tile and mixes each V tile in shared
- * memory, so nothing rotated or mixed is ever written.
+/* The forward with the two steps the pages run just before the core
+ * ("autoresearch" README (gitee), section 7.4: rotary position embedding of q
+ * and k; section 5.2.3: the value embedding mixed into v on the layers that
+ * have one), on the unrotated, unmixed q, k, v.  Q tiles are rotated inside the
+ * forward kernel as they land in shared memory; the rotated k and the mixed v
+ * are written once into the workspace by a pre-pass (a K or V tile is read by
+ * every query-tile unit whose band covers it, so rotating it in each tile
+ * costs more than one pass over k and v), and the kernel reads them from there.
  *   rope_cos, rope_sin: bf16 [rope_rows, D/2] (rope_rows >= T), row t holding
  *     position t's cos and sin; row t of q and k becomes
  *     (x1 cos_t + x2 sin_t, -x1 sin_t + x2 cos_t) with x1, x2 its two halves.
  *   ve, ve_gate: both NULL (no value embedding), or ve bf16 [B, T, Hkv, D] and
  *     the gate logits g bf16 [B, T, Hkv]: v becomes v + 2 sigmoid(g) ve.
- * Everything else (layouts, lse optional, grouped K/V heads, errors) is as for
- * ar_attn_fwd_gqa.  AR_ERR_NULL if a table is NULL or only one of ve, ve_gate
- * is; AR_ERR_SHAPE if rope_rows < T; tables and ve 16-byte aligned. */
+ *   workspace: at least ar_attn_fwd_rope_workspace_bytes(B, T, Hkv, D, ve != NULL)
+ *     bytes, 256-byte aligned (NULL: allocated stream-ordered on `stream`).
+ * The rotated and mixed values are rounded to bf16 once, as the pages hold
+ * them.  Everything else (layouts, lse optional, grouped K/V heads, errors) is
+ * as for ar_attn_fwd_gqa.  AR_ERR_NULL if a table is NULL or only one of ve,
+ * ve_gate is; AR_ERR_SHAPE if rope_rows < T; tables and ve 16-byte aligned. */
+size_t ar_attn_fwd_rope_workspace_bytes(int B, int T, int Hkv, int D, int with_ve);
 int ar_attn_fwd_rope(const void* q, const void* k, const void* v, void* o, float* lse, const void* rope_cos,
                      const void* rope_sin, int rope_rows, const void* ve, const void* ve_gate, int B, int T,
-                     int H, int Hkv, int D, int window, float eps, float scale, void* stream);
+                     int H, int Hkv, int D, int window, float eps, float scale, void* workspace,
+                     size_t workspace_bytes, void* stream);
 
 /* Backward of ar_attn_fwd_rope: the gradients with respect to the unrotated,
  * unmixed q, k, v, and (with the value embedding) to ve and the gate logits g.
@@ -201,7 +208,7 @@ enum {
   AR_KERNEL_BWD_PREP = 2, /* delta, 1/rms(q), lse * log2(e) (memory-bound) */
   AR_KERNEL_BWD = 3,      /* fused backward attention: dk, dv, G tiles (tensor-core bound) */
   AR_KERNEL_DQ = 4,       /* dq = G K with the q-side RMSNorm backward (reads the G tiles) */
-  AR_KERNEL_ROPE_PREP = 5, /* rotated q, k and mixed v for the RoPE backward (memory-bound) */
+  AR_KERNEL_ROPE_PREP = 5, /* rotated k (and q) and mixed v of the RoPE path (memory-bound) */
   AR_KERNEL_KINDS = 6
 };
 

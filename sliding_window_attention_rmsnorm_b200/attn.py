@@ -65,7 +65,9 @@ def lib():
         L.ar_attn_bwd_gqa_workspace_bytes.restype = sz
         L.ar_attn_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, vp, sz, vp]
         L.ar_attn_bwd_gqa.restype = i
-        L.ar_attn_fwd_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, i, i, i, i, f, f, vp]
+        L.ar_attn_fwd_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, i, i, i, i, f, f, vp, sz, vp]
+        L.ar_attn_fwd_rope_workspace_bytes.argtypes = [i, i, i, i, i]
+        L.ar_attn_fwd_rope_workspace_bytes.restype = sz
         L.ar_attn_fwd_rope.restype = i
         L.ar_attn_bwd_rope_workspace_bytes.argtypes = [i, i, i, i, i, i]
         L.ar_attn_bwd_rope_workspace_bytes.restype = sz
@@ -240,13 +242,17 @@ def rope_tables(T: int, D: int = 128, base: float = 10000.0, device="cuda"):
     return ang.cos().to(torch.bfloat16).to(device), ang.sin().to(torch.bfloat16).to(device)
 
 
+def fwd_rope_workspace_bytes(B, T, Hkv, D, with_ve=False) -> int:
+    return int(lib().ar_attn_fwd_rope_workspace_bytes(B, T, Hkv, D, 1 if with_ve else 0))
+
+
 def fwd_rope(q, k, v, cos, sin, window: int, eps: float = 1e-6, scale=None, ve=None, ve_gate=None, out=None,
-             lse=None, need_lse: bool = True):
-    """The forward with the steps before the core fused into it: q and k rotated
-    by RoPE (cos, sin: bf16 [rows >= T, 64], row t = position t) and, when ve
-    ([B, T, Hkv, 128]) and ve_gate (the gate logits g, [B, T, Hkv]) are given,
-    v replaced by v + 2 sigmoid(g) ve.  q, k, v are the unrotated, unmixed
-    tensors; nothing rotated or mixed is written."""
+             lse=None, need_lse: bool = True, workspace=None):
+    """The forward with the steps before the core: q and k rotated by RoPE (cos,
+    sin: bf16 [rows >= T, 64], row t = position t) and, when ve ([B, T, Hkv,
+    128]) and ve_gate (the gate logits g, [B, T, Hkv]) are given, v replaced by
+    v + 2 sigmoid(g) ve.  q, k, v are the unrotated, unmixed tensors; Q is
+    rotated inside the kernel, k and v in one pre-pass into the workspace."""
     Hkv = _check_qkv(q, k, v)
     B, T, H, D = q.shape
     _check_rope(cos, sin, T)
@@ -260,9 +266,12 @@ def fwd_rope(q, k, v, cos, sin, window: int, eps: float = 1e-6, scale=None, ve=N
     if need_lse:
         lse_t = torch.empty((B, H, T), dtype=torch.float32, device=q.device) if lse is None else lse
         _check_lse(lse_t, B, H, T, q.device)
+    if workspace is None:
+        workspace = torch.empty(fwd_rope_workspace_bytes(B, T, Hkv, D, ve is not None), dtype=torch.uint8,
+                                device=q.device)
     st = lib().ar_attn_fwd_rope(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), _ptr(cos), _ptr(sin),
                                 int(cos.shape[0]), _ptr(ve), _ptr(ve_gate), B, T, H, Hkv, D, int(window),
-                                float(eps), float(scale), _stream())
+                                float(eps), float(scale), _ptr(workspace), workspace.numel(), _stream())
     _check(st, "ar_attn_fwd_rope")
     return o, lse_t
 

@@ -71,10 +71,8 @@ int device_setup(int* sms_out, int* prep_blocks_out = nullptr) {
                fwd_attr(ar::fwd::fwd_kernel<false, false>) != cudaSuccess ||
                fwd_attr(ar::fwd::fwd_kernel<true, true>) != cudaSuccess ||
                fwd_attr(ar::fwd::fwd_kernel<false, true>) != cudaSuccess ||
-               fwd_attr(ar::fwd::fwd_kernel<true, false, 1>) != cudaSuccess ||
-               fwd_attr(ar::fwd::fwd_kernel<false, false, 1>) != cudaSuccess ||
-               fwd_attr(ar::fwd::fwd_kernel<true, false, 3>) != cudaSuccess ||
-               fwd_attr(ar::fwd::fwd_kernel<false, false, 3>) != cudaSuccess ||
+               fwd_attr(ar::fwd::fwd_kernel<true, false, true>) != cudaSuccess ||
+               fwd_attr(ar::fwd::fwd_kernel<false, false, true>) != cudaSuccess ||
                bwd_attr(ar::bwd::bwd_kernel<0>) != cudaSuccess || bwd_attr(ar::bwd::bwd_kernel<1>) != cudaSuccess ||
                bwd_attr(ar::bwd::bwd_kernel<3>) != cudaSuccess ||
                cudaFuncSetAttribute(ar::dqk::dq_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -90,8 +88,8 @@ int device_setup(int* sms_out, int* prep_blocks_out = nullptr) {
       // cannot be met.  The backward kernel is checked for its own budget.
       if (!fwd_regs_ok(ar::fwd::fwd_kernel<true, false>) || !fwd_regs_ok(ar::fwd::fwd_kernel<false, false>) ||
           !fwd_regs_ok(ar::fwd::fwd_kernel<true, true>) || !fwd_regs_ok(ar::fwd::fwd_kernel<false, true>) ||
-          !fwd_regs_ok(ar::fwd::fwd_kernel<true, false, 1>) || !fwd_regs_ok(ar::fwd::fwd_kernel<false, false, 1>) ||
-          !fwd_regs_ok(ar::fwd::fwd_kernel<true, false, 3>) || !fwd_regs_ok(ar::fwd::fwd_kernel<false, false, 3>))
+          !fwd_regs_ok(ar::fwd::fwd_kernel<true, false, true>) ||
+          !fwd_regs_ok(ar::fwd::fwd_kernel<false, false, true>))
         d.status = AR_ERR_CUDA;
       for (BwdKernel f : {ar::bwd::bwd_kernel<0>, ar::bwd::bwd_kernel<1>, ar::bwd::bwd_kernel<3>}) {
         cudaFuncAttributes ba;
@@ -164,8 +162,7 @@ ar::FwdParams fwd_params(void* o, float* lse, const float* ck, int B, int T, int
                          float eps, float scale) {
   ar::FwdParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
-  p.rcos = p.rsin = p.ve = p.vg = nullptr;
-  p.wide_ve = 0;
+  p.rcos = p.rsin = nullptr;
   p.lse = lse;
   p.ck = ck;
   p.B = B;
@@ -186,20 +183,15 @@ ar::FwdParams fwd_params(void* o, float* lse, const float* ck, int B, int T, int
 
 // The forward with the fixed softmax offset when the logit bound allows it
 // (see fwd.cuh), else the running-max forward; key factors computed in the
-// kernel, or (ck_global) read from p.ck; pro: the prologue fusion (1: RoPE,
-// 3: RoPE and the value embedding).
+// kernel, or (ck_global) read from p.ck; rope_q: Q tiles rotated in the kernel.
 void launch_fwd(int grid, cudaStream_t s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                const ar::FwdParams& p, bool ck_global, int pro = 0) {
+                const ar::FwdParams& p, bool ck_global, bool rope_q = false) {
   using namespace ar::fwd;
   const bool fixed = p.bound <= kFixedBoundMax;
-  if (pro == 1 && fixed)
-    fwd_kernel<true, false, 1><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
-  else if (pro == 1)
-    fwd_kernel<false, false, 1><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
-  else if (pro == 3 && fixed)
-    fwd_kernel<true, false, 3><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
-  else if (pro == 3)
-    fwd_kernel<false, false, 3><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
+  if (rope_q && fixed)
+    fwd_kernel<true, false, true><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
+  else if (rope_q)
+    fwd_kernel<false, false, true><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
   else if (fixed && !ck_global)
     fwd_kernel<true, false><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
   else if (!fixed && !ck_global)
@@ -354,9 +346,15 @@ int ar_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float*
   return cudaGetLastError() == cudaSuccess ? AR_OK : AR_ERR_CUDA;
 }
 
+size_t ar_attn_fwd_rope_workspace_bytes(int B, int T, int Hkv, int D, int with_ve) {
+  if (check_shape(B, T, Hkv, D) != AR_OK) return 0;
+  return round_up((size_t)B * T * Hkv * kD * 2, 256) * (with_ve ? 2 : 1);
+}
+
 int ar_attn_fwd_rope(const void* q, const void* k, const void* v, void* o, float* lse, const void* rope_cos,
                      const void* rope_sin, int rope_rows, const void* ve, const void* ve_gate, int B, int T, int H,
-                     int Hkv, int D, int window, float eps, float scale, void* stream) {
+                     int Hkv, int D, int window, float eps, float scale, void* workspace, size_t workspace_bytes,
+                     void* stream) {
   if (!q || !k || !v || !o || !rope_cos || !rope_sin) return AR_ERR_NULL;  // lse may be NULL: not stored
   if ((ve == nullptr) != (ve_gate == nullptr)) return AR_ERR_NULL;
   int st = check_shape(B, T, H, D);
@@ -367,27 +365,48 @@ int ar_attn_fwd_rope(const void* q, const void* k, const void* v, void* o, float
       !aligned(rope_cos, 16) || !aligned(rope_sin, 16) || !aligned(ve, 16) || !aligned(ve_gate, 2))
     return AR_ERR_ALIGN;
   if ((st = check_args(eps, scale)) != AR_OK) return st;
-  int sms = 0;
-  if ((st = device_setup(&sms)) != AR_OK) return st;
+  const size_t need = ar_attn_fwd_rope_workspace_bytes(B, T, Hkv, D, ve != nullptr);
+  if (workspace && workspace_bytes < need) return AR_ERR_WORKSPACE;
+  if (workspace && !aligned(workspace, 256)) return AR_ERR_ALIGN;
+  int sms = 0, prep_blocks = 1;
+  if ((st = device_setup(&sms, &prep_blocks)) != AR_OK) return st;
 
-  CUtensorMap tq, tk, tv;
-  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, Hkv) != AR_OK ||
-      make_map(&tv, v, B, T, Hkv) != AR_OK)
-    return AR_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  if (!ws && cudaMallocAsync(&ws, need, s) != cudaSuccess) return AR_ERR_CUDA;
+  // the rotated k and the mixed v, once per layer (a K or V tile is read by every
+  // unit whose band covers it); Q is rotated in the kernel's tiles
+  __nv_bfloat16* kr = static_cast<__nv_bfloat16*>(ws);
+  __nv_bfloat16* vm = kr + round_up((size_t)B * T * Hkv * kD * 2, 256) / 2;
+  const __nv_bfloat16* rc = static_cast<const __nv_bfloat16*>(rope_cos);
+  const __nv_bfloat16* rs = static_cast<const __nv_bfloat16*>(rope_sin);
+  {
+    KernelTimer t(AR_KERNEL_ROPE_PREP, s);
+    const long long prows = (long long)B * T * Hkv * (ve ? 2 : 1);
+    ar::rope_ve_prep_kernel<<<bwd_prep_grid(prows, sms, prep_blocks), 256, 0, s>>>(
+        nullptr, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+        static_cast<const __nv_bfloat16*>(ve), static_cast<const __nv_bfloat16*>(ve_gate), rc, rs, nullptr, kr, vm,
+        B, T, H, Hkv);
+    t.stop();
+  }
+  CUtensorMap tq, tk, tv;
+  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, kr, B, T, Hkv) != AR_OK ||
+      make_map(&tv, ve ? static_cast<const void*>(vm) : v, B, T, Hkv) != AR_OK) {
+    if (!workspace) cudaFreeAsync(ws, s);
+    return AR_ERR_CUDA;
+  }
   ar::FwdParams p = fwd_params(o, lse, nullptr, B, T, H, Hkv, window, eps, scale);
-  p.rcos = static_cast<const __nv_bfloat16*>(rope_cos);
-  p.rsin = static_cast<const __nv_bfloat16*>(rope_sin);
-  p.ve = static_cast<const __nv_bfloat16*>(ve);
-  p.vg = static_cast<const __nv_bfloat16*>(ve_gate);
-  p.wide_ve = ve != nullptr && aligned(ve, 32);
+  p.rcos = rc;
+  p.rsin = rs;
   const int grid = p.n_units < sms ? p.n_units : sms;
   {
     KernelTimer t(AR_KERNEL_FWD, s);
-    launch_fwd(grid, s, tq, tk, tv, p, false, ve ? 3 : 1);
+    launch_fwd(grid, s, tq, tk, tv, p, false, true);
     t.stop();
   }
-  return cudaGetLastError() == cudaSuccess ? AR_OK : AR_ERR_CUDA;
+  cudaError_t e = cudaGetLastError();
+  if (!workspace) cudaFreeAsync(ws, s);
+  return e == cudaSuccess ? AR_OK : AR_ERR_CUDA;
 }
 
 int ar_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T, int H, int D,

@@ -135,20 +135,21 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_
   }
 }
 
-// The backward's pre-pass of the RoPE / value-embedding path: the rotated q
-// and k and the mixed v that the forward formed in its tiles, written out for
-// the backward kernels (the same arithmetic, so the same bf16 values).  Rows
-// [0, nq) are q rows [B, T, H], then nk k rows and nk v rows [B, T, Hkv]; one
-// row per 8 lanes.  RoPE: lane l rotates features 8l .. 8l+7 with their
-// partners 64 + 8l ..; value embedding (only when ve is given): lane l mixes
-// features 16l .. 16l+15.
+// The pre-pass of the RoPE / value-embedding path: the rotated q and k and the
+// mixed v (v + 2 sigmoid(g) ve) written out for the attention kernels, with the
+// arithmetic of sm100.cuh's helpers.  Rows [0, nq) are q rows [B, T, H] (none
+// when q is NULL: the forward rotates its Q tiles itself), then nk k rows and,
+// when ve is given, nk v rows [B, T, Hkv]; one row per 8 lanes.  RoPE: lane l
+// rotates features 8l .. 8l+7 with their partners 64 + 8l ..; value embedding:
+// lane l mixes features 16l .. 16l+15.
 __global__ void rope_ve_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                                     const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ ve,
                                     const __nv_bfloat16* __restrict__ vg, const __nv_bfloat16* __restrict__ rcos,
                                     const __nv_bfloat16* __restrict__ rsin, __nv_bfloat16* __restrict__ qr,
                                     __nv_bfloat16* __restrict__ kr, __nv_bfloat16* __restrict__ vm, int B, int T,
                                     int H, int Hkv) {
-  const long long nq = (long long)B * T * H, nk = (long long)B * T * Hkv, rows = nq + nk + (ve ? nk : 0);
+  const long long nq = q ? (long long)B * T * H : 0, nk = (long long)B * T * Hkv;
+  const long long rows = nq + nk + (ve ? nk : 0);
   const int sub = threadIdx.x & 7;
   const long long gstride = (long long)gridDim.x * (blockDim.x / 8);
   for (long long r = (long long)blockIdx.x * (blockDim.x / 8) + threadIdx.x / 8; r < rows; r += gstride) {
@@ -173,18 +174,14 @@ __global__ void rope_ve_prep_kernel(const __nv_bfloat16* __restrict__ q, const _
       const long long rr = r - nq - nk;
       const uint4* src = reinterpret_cast<const uint4*>(v + rr * 128 + 16 * sub);
       uint4* dst = reinterpret_cast<uint4*>(vm + rr * 128 + 16 * sub);
-      uint4 a = __ldg(src), b = __ldg(src + 1);
-      if (ve) {
-        const float gate = ve_gate(vg[rr]);
-        const uint4* e = reinterpret_cast<const uint4*>(ve + rr * 128 + 16 * sub);
-        const uint4 ea = __ldg(e), eb = __ldg(e + 1);
-        a = make_uint4(ve_mix_word(a.x, ea.x, gate), ve_mix_word(a.y, ea.y, gate), ve_mix_word(a.z, ea.z, gate),
-                       ve_mix_word(a.w, ea.w, gate));
-        b = make_uint4(ve_mix_word(b.x, eb.x, gate), ve_mix_word(b.y, eb.y, gate), ve_mix_word(b.z, eb.z, gate),
-                       ve_mix_word(b.w, eb.w, gate));
-      }
-      dst[0] = a;
-      dst[1] = b;
+      const uint4 a = __ldg(src), b = __ldg(src + 1);
+      const float gate = ve_gate(vg[rr]);
+      const uint4* e = reinterpret_cast<const uint4*>(ve + rr * 128 + 16 * sub);
+      const uint4 ea = __ldg(e), eb = __ldg(e + 1);
+      dst[0] = make_uint4(ve_mix_word(a.x, ea.x, gate), ve_mix_word(a.y, ea.y, gate), ve_mix_word(a.z, ea.z, gate),
+                          ve_mix_word(a.w, ea.w, gate));
+      dst[1] = make_uint4(ve_mix_word(b.x, eb.x, gate), ve_mix_word(b.y, eb.y, gate), ve_mix_word(b.z, eb.z, gate),
+                          ve_mix_word(b.w, eb.w, gate));
     }
   }
 }

@@ -56,12 +56,6 @@ struct BwdParams {
   const float* lse2;       // [B*H, T_pad] lse * log2(e), 0 on padding
   const float* delta;      // [B*H, T_pad] rowsum(dO * o), 0 on padding
   const float* rq;         // [B*H, T_pad] 1/rms(q_i), 0 on padding
-  const __nv_bfloat16* rcos;  // kPro & 1: rotary tables [>= T, 64], row t = position t
-  const __nv_bfloat16* rsin;
-  const __nv_bfloat16* ve;    // kPro & 2: value embedding [B, T, Hkv, 128] and gate logits [B, T, Hkv]
-  const __nv_bfloat16* vg;
-  __nv_bfloat16* dve;         // kPro & 2: outputs [B, T, Hkv, 128] and [B, T, Hkv]
-  float* dg;
   int B, T, H, T_pad;
   int Hkv, grp;  // K/V heads and query heads per K/V head (H = Hkv * grp; grp = 1: multi-head)
   int w;        // left window (w >= T means full causal)
@@ -75,6 +69,12 @@ struct BwdParams {
   int wide_k;  // k is 32-byte aligned: key rows are read with 256-bit loads
   int wide_ve;  // ve is 32-byte aligned
   unsigned long long wait_ns;  // limit of a device-side wait (kWaitLimitNs unless set otherwise)
+  const __nv_bfloat16* rcos;   // kPro & 1: rotary tables [>= T, 64], row t = position t
+  const __nv_bfloat16* rsin;
+  const __nv_bfloat16* ve;     // kPro & 2: value embedding [B, T, Hkv, 128] and gate logits [B, T, Hkv]
+  const __nv_bfloat16* vg;
+  __nv_bfloat16* dve;          // kPro & 2: outputs [B, T, Hkv, 128] and [B, T, Hkv]
+  float* dg;
 };
 
 // Slot of the G tile of (query tile qt, key tile kt) of the launch's query head
@@ -514,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // dk = scale (acc - coef k), coef = rk^2 (acc . k) / D, with acc . k summed by
         // the compute warpgroups as sum_i G_ij S_ij; the raw key row is loaded into
         // registers before the wait, so its latency is hidden by the unit's products
-        if constexpr (!kRope) {
+        {
           uint4 kv[16];
           {
             const uint4* krow = reinterpret_cast<const uint4*>(p.k + orow);
@@ -532,74 +532,67 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const float coef = lds_f32(sbase + kDot + 4 * row) + lds_f32(sbase + kDot + 4 * (128 + row));
           mbar_arrive(bar_addr(sbase, DOTFREE));
+          if constexpr (!kRope) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t x[32];
-            tmem_ld32(tDK + 32 * c, x);
-            tmem_wait_ld();
-            uint32_t pk[16];
+            for (int c = 0; c < 4; ++c) {
+              uint32_t x[32];
+              tmem_ld32(tDK + 32 * c, x);
+              tmem_wait_ld();
+              uint32_t pk[16];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const uint4 v = kv[4 * c + q4];
-              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+              for (int q4 = 0; q4 < 4; ++q4) {
+                const uint4 v = kv[4 * c + q4];
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float g0 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e]) - coef * bf16lo(w4[e]));
-                const float g1 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e + 1]) - coef * bf16hi(w4[e]));
-                pk[4 * q4 + e] = pack_bf16(g0, g1);
+                for (int e = 0; e < 4; ++e) {
+                  const float g0 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e]) - coef * bf16lo(w4[e]));
+                  const float g1 = p.scale * (__uint_as_float(x[8 * q4 + 2 * e + 1]) - coef * bf16hi(w4[e]));
+                  pk[4 * q4 + e] = pack_bf16(g0, g1);
+                }
+              }
+              if (jv) {
+                stg32B(p.dk + orow + 32 * c, pk, p.wide);
+                stg32B(p.dk + orow + 32 * c + 16, pk + 8, p.wide);
               }
             }
-            if (jv) {
-              stg32B(p.dk + orow + 32 * c, pk, p.wide);
-              stg32B(p.dk + orow + 32 * c + 16, pk + 8, p.wide);
-            }
-          }
-        } else {
-          // dk_rot = scale (acc - coef k_rot), then dk = R_j^T dk_rot: features
-          // 16c .. 16c+15 with their partners 64 + 16c .., the rotated key row and
-          // the table entries read as needed (L2)
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, DKDVDONE), uidx & 1, abort_flag, p.wait_ns))) break;
-          tc_fence_after();
-          const float coef = lds_f32(sbase + kDot + 4 * row) + lds_f32(sbase + kDot + 4 * (128 + row));
-          mbar_arrive(bar_addr(sbase, DOTFREE));
-          const __nv_bfloat16* cr = p.rcos + (size_t)(jv ? j : 0) * 64;
-          const __nv_bfloat16* sr = p.rsin + (size_t)(jv ? j : 0) * 64;
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t xl[16], xh[16];
-            tmem_ld16(tDK + 16 * c, xl);
-            tmem_ld16(tDK + 64 + 16 * c, xh);
-            uint4 kl[2], kh[2], cc[2], sc[2];
-            if (jv) {
-              ldg32B(p.k + orow + 16 * c, kl[0], kl[1], p.wide_k);
-              ldg32B(p.k + orow + 64 + 16 * c, kh[0], kh[1], p.wide_k);
-              cc[0] = __ldg(reinterpret_cast<const uint4*>(cr + 16 * c));
-              cc[1] = __ldg(reinterpret_cast<const uint4*>(cr + 16 * c + 8));
-              sc[0] = __ldg(reinterpret_cast<const uint4*>(sr + 16 * c));
-              sc[1] = __ldg(reinterpret_cast<const uint4*>(sr + 16 * c + 8));
-            } else {
-              kl[0] = kl[1] = kh[0] = kh[1] = cc[0] = cc[1] = sc[0] = sc[1] = make_uint4(0, 0, 0, 0);
-            }
-            tmem_wait_ld();
-            uint32_t pl[8], ph[8];
+          } else {
+            // dk_rot = scale (acc - coef k_rot) (k_rot: the rotated key row in kv),
+            // then dk = R_j^T dk_rot: features 16c .. 16c+15 with their partners
+            // 64 + 16c .., the table entries read as needed (the tables stay in L2)
+            const __nv_bfloat16* cr = p.rcos + (size_t)(jv ? j : 0) * 64;
+            const __nv_bfloat16* sr = p.rsin + (size_t)(jv ? j : 0) * 64;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const uint4& a = kl[e >> 2];
-              const uint4& b = kh[e >> 2];
-              const uint4& cv = cc[e >> 2];
-              const uint4& sv = sc[e >> 2];
-              const uint32_t kw1 = (&a.x)[e & 3], kw2 = (&b.x)[e & 3], cw = (&cv.x)[e & 3], sw = (&sv.x)[e & 3];
-              const float d10 = p.scale * (__uint_as_float(xl[2 * e]) - coef * bf16lo(kw1));
-              const float d11 = p.scale * (__uint_as_float(xl[2 * e + 1]) - coef * bf16hi(kw1));
-              const float d20 = p.scale * (__uint_as_float(xh[2 * e]) - coef * bf16lo(kw2));
-              const float d21 = p.scale * (__uint_as_float(xh[2 * e + 1]) - coef * bf16hi(kw2));
-              const float c0 = bf16lo(cw), c1 = bf16hi(cw), s0 = bf16lo(sw), s1 = bf16hi(sw);
-              pl[e] = pack_bf16(fmaf(d10, c0, -(d20 * s0)), fmaf(d11, c1, -(d21 * s1)));
-              ph[e] = pack_bf16(fmaf(d10, s0, d20 * c0), fmaf(d11, s1, d21 * c1));
-            }
-            if (jv) {
-              stg32B(p.dk + orow + 16 * c, pl, p.wide);
-              stg32B(p.dk + orow + 64 + 16 * c, ph, p.wide);
+            for (int c = 0; c < 4; ++c) {  // unrolled: kv is indexed by c
+              uint32_t xl[16], xh[16];
+              tmem_ld16(tDK + 16 * c, xl);
+              tmem_ld16(tDK + 64 + 16 * c, xh);
+              uint4 cc[2], sc[2];
+              if (jv) {
+                cc[0] = __ldg(reinterpret_cast<const uint4*>(cr + 16 * c));
+                cc[1] = __ldg(reinterpret_cast<const uint4*>(cr + 16 * c + 8));
+                sc[0] = __ldg(reinterpret_cast<const uint4*>(sr + 16 * c));
+                sc[1] = __ldg(reinterpret_cast<const uint4*>(sr + 16 * c + 8));
+              } else {
+                cc[0] = cc[1] = sc[0] = sc[1] = make_uint4(0, 0, 0, 0);
+              }
+              tmem_wait_ld();
+              uint32_t pl[8], ph[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const uint32_t kw1 = (&kv[2 * c + (e >> 2)].x)[e & 3], kw2 = (&kv[8 + 2 * c + (e >> 2)].x)[e & 3];
+                const uint32_t cw = (&cc[e >> 2].x)[e & 3], sw = (&sc[e >> 2].x)[e & 3];
+                const float d10 = p.scale * (__uint_as_float(xl[2 * e]) - coef * bf16lo(kw1));
+                const float d11 = p.scale * (__uint_as_float(xl[2 * e + 1]) - coef * bf16hi(kw1));
+                const float d20 = p.scale * (__uint_as_float(xh[2 * e]) - coef * bf16lo(kw2));
+                const float d21 = p.scale * (__uint_as_float(xh[2 * e + 1]) - coef * bf16hi(kw2));
+                const float c0 = bf16lo(cw), c1 = bf16hi(cw), s0 = bf16lo(sw), s1 = bf16hi(sw);
+                pl[e] = pack_bf16(fmaf(d10, c0, -(d20 * s0)), fmaf(d11, c1, -(d21 * s1)));
+                ph[e] = pack_bf16(fmaf(d10, s0, d20 * c0), fmaf(d11, s1, d21 * c1));
+              }
+              if (jv) {
+                stg32B(p.dk + orow + 16 * c, pl, p.wide);
+                stg32B(p.dk + orow + 64 + 16 * c, ph, p.wide);
+              }
             }
           }
         }

@@ -18,7 +18,7 @@
 //   warps 4-7  softmax warpgroup 1: query tile 1 (rows r0+128..r0+255)
 //   warp 8     TMA producer: Q tiles, K tiles (3 stages), V tiles (2 stages)
 //   warp 9     MMA issuer: S_k = Q_k K^T into TMEM, O_k += P_k V with P_k read from TMEM
-//   warps 10-11 idle; with the value-embedding prologue they mix ve into each V tile
+//   warps 10-11 idle
 //   warps 12-15 key factors: ck_j = rk_j * scale * log2(e) of each K tile, one key
 //              row per thread, from the tile in shared memory into a 4-slot ring
 //              read by the softmax.  One warp sits on each SM sub-partition, so
@@ -49,17 +49,18 @@
 // product has run: the next unit's Q tiles load under the last tile's softmax
 // and the epilogue.
 //
-// Prologue fusion (kPro != 0): the steps the pages run just before the core
-// happen here, on the tiles in shared memory, so no rotated or mixed tensor is
-// ever written.  RoPE ("autoresearch" README (gitee), section 7.4: the halves
-// x1 = x[:64], x2 = x[64:] of each row at position t become x1 cos_t + x2 sin_t
-// and -x1 sin_t + x2 cos_t, with bf16 tables): the key-factor warps rotate the
-// unit's two Q tiles when they land, and each K tile before its S products
-// (rotation keeps a row's length, so the norm factors are unchanged).  The
-// value embedding (section 5.2.3: v + 2 sigmoid(g) ve on the layers that have
-// one) is mixed into each V tile by the same warps before its P V product.
-// The MMA warp then waits for these rewritten tiles (QREADY, KREADY, VREADY)
-// instead of the TMA arrivals.
+// RoPE on Q in the tile (kRopeQ): the rotary position embedding of the
+// "autoresearch" README (gitee), section 7.4 (the halves x1 = x[:64],
+// x2 = x[64:] of each row at position t become x1 cos_t + x2 sin_t and
+// -x1 sin_t + x2 cos_t, with bf16 tables) is applied to the unit's two Q tiles
+// in shared memory by the key-factor warps when they land, and the MMA warp and
+// the softmax warpgroups wait for the rotated tiles (QREADY) instead of the TMA
+// arrival.  A Q tile is loaded once per unit, so this costs one pass over q.
+// K and V tiles are re-read by every unit whose band covers them (about 4.5
+// times per layer at T = 2048, window 1024), so the rotated k and the mixed v
+// (section 5.2.3) come from one pre-pass instead (aux.cuh): rotating them in
+// each tile was measured at 121 against 54 us per layer, bound by the latency
+// of the table and value-embedding loads.
 #pragma once
 #include <type_traits>
 
@@ -69,10 +70,8 @@ namespace ar {
 
 struct FwdParams {
   __nv_bfloat16* o;  // [B, T, H, 128]
-  const __nv_bfloat16* rcos;  // kPro & 1: rotary tables [>= T, 64] bf16, row t = position t
+  const __nv_bfloat16* rcos;  // kRopeQ: rotary tables [>= T, 64] bf16, row t = position t
   const __nv_bfloat16* rsin;
-  const __nv_bfloat16* ve;    // kPro & 2: value embedding [B, T, Hkv, 128] bf16
-  const __nv_bfloat16* vg;    // kPro & 2: gate logits g [B, T, Hkv] bf16
   float* lse;        // [B, H, T], or NULL: not stored (forward-only use)
   const float* ck;   // kCkGlobal only: [B*Hkv, T_pad] rk_j * scale * log2(e), 0 on padding
   int B, T, H, T_pad;
@@ -84,7 +83,6 @@ struct FwdParams {
   float bound;       // scale * D * log2(e): the largest |logit| in log2 units
   float cscale;      // scale * log2(e)
   int wide;          // o is 32-byte aligned: rows are written with 256-bit stores
-  int wide_ve;       // ve is 32-byte aligned: its rows are read with 256-bit loads
   unsigned long long wait_ns;  // limit of a device-side wait (kWaitLimitNs unless set otherwise)
 };
 
@@ -97,8 +95,8 @@ constexpr int kThreads = 512;
 constexpr int kRegsLow = 104, kRegsCk = 40, kRegsHigh = 184, kLaunchRegs = 128;
 static_assert(256 * kRegsHigh + 128 * kRegsLow + 128 * kRegsCk <= kLaunchRegs * kThreads,
               "register split exceeds the launch budget");
-// With the prologue fusion the key-factor warps also rotate and mix tiles and
-// take 56 registers; the softmax warpgroups give up the difference.
+// With the rotation of Q the key-factor warps take 56 registers; the softmax
+// warpgroups give up the difference.
 constexpr int kRegsLowPro = 104, kRegsCkPro = 56, kRegsHighPro = 176;
 static_assert(256 * kRegsHighPro + 128 * kRegsLowPro + 128 * kRegsCkPro <= kLaunchRegs * kThreads,
               "register split exceeds the launch budget");
@@ -118,8 +116,7 @@ constexpr float kFixedBoundMax = 32.0f;
 enum {
   QFULL = 0, QEMPTY, KFULL, KEMPTY = KFULL + kKStages, VFULL = KEMPTY + kKStages, VEMPTY = VFULL + kVStages,
   SFULL = VEMPTY + kVStages, PFULL = SFULL + 2, ODONE = PFULL + 2, OFREE = ODONE + 2,
-  CKFULL = OFREE + 2, FINAL = CKFULL + kCkSlots,
-  QREADY, KREADY, VREADY = KREADY + kKStages, NBAR = VREADY + kVStages  // prologue fusion only
+  CKFULL = OFREE + 2, FINAL = CKFULL + kCkSlots, QREADY /* kRopeQ only */, NBAR
 };
 constexpr int kCkThreads = 128;  // warps 12-15
 constexpr uint32_t kBar = kCK + kCkSlots * 512;
@@ -200,36 +197,12 @@ __device__ __forceinline__ void rope_row(uint32_t tile, int row, const __nv_bflo
   }
 }
 
-// v <- v + gate * ve for row `row` of a 128-byte-swizzled V tile; erow: the
-// row's 128 value-embedding entries in global memory (32-byte aligned when
-// `wide`), all loaded before the tile is touched.  The sums are rounded to
-// bf16 once.
-__device__ __forceinline__ void ve_row(uint32_t tile, int row, const __nv_bfloat16* erow, float gate, bool wide) {
-  uint4 e[16];
-#pragma unroll
-  for (int c = 0; c < 16; c += 2) ldg32B(erow + 8 * c, e[c], e[c + 1], wide);
-#pragma unroll
-  for (int pass = 0; pass < 4; ++pass) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int ch = 4 * pass + i;  // 16-byte chunk of the row: features 8ch .. 8ch + 7
-      const uint32_t a = tile + (ch >> 3) * kHalf + sw128(row, ch & 7);
-      const uint4 x = lds128(a);
-      const uint32_t xv[4] = {x.x, x.y, x.z, x.w}, ev[4] = {e[ch].x, e[ch].y, e[ch].z, e[ch].w};
-      uint32_t y[4];
-#pragma unroll
-      for (int w = 0; w < 4; ++w) y[w] = ve_mix_word(xv[w], ev[w], gate);
-      sts128(a, make_uint4(y[0], y[1], y[2], y[3]));
-    }
-  }
-}
-
-template <bool kFixed, bool kCkGlobal, int kPro = 0>
+template <bool kFixed, bool kCkGlobal, bool kRopeQ = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  constexpr bool kRope = (kPro & 1) != 0, kVe = (kPro & 2) != 0;
-  static_assert(!(kPro && kCkGlobal), "the prologue fusion runs on the key-factor warps");
+  constexpr bool kRope = kRopeQ;
+  static_assert(!(kRopeQ && kCkGlobal), "the rotation of Q runs on the key-factor warps");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
@@ -247,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (i == PFULL || i == PFULL + 1 || i == OFREE || i == OFREE + 1) cnt = 128;
       if (!kCkGlobal && i >= KEMPTY && i < KEMPTY + kKStages) cnt = 1 + kCkThreads;  // MMA commit + key-factor warps
       if (i >= CKFULL && i < CKFULL + kCkSlots) cnt = kCkThreads;
-      if (i >= QREADY) cnt = i >= VREADY ? 64 : kCkThreads;  // the warps that rewrite the tile
+      if (i == QREADY) cnt = kCkThreads;  // the key-factor warps, once the unit's Q tiles are rotated
       mbar_init(bar_addr(sbase, i), cnt);
     }
     *abort_flag = 0;
@@ -268,9 +241,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + kTmemPtr);
 
   if (warp >= 12) {
-    regs_dec<kPro ? kRegsCkPro : kRegsCk>();
+    regs_dec<kRope ? kRegsCkPro : kRegsCk>();
     if (!kCkGlobal) {
-      // ---------------------------------------------------------- key factors (and prologue)
+      // ---------------------------------------------------------- key factors (and Q rotation)
       // Tile kv's factors go to ring slot kv % kCkSlots (free: see kCkSlots).
       const int row = threadIdx.x - 384;  // key row within the tile
       uint32_t kv = 0;
@@ -301,13 +274,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t kt = sbase + kK + st * kTile;
           const int j = n * 128 + row;  // key position
-          if constexpr (kRope) {
-            // rotate first: the norm factor is taken from the rotated bf16 row the
-            // S product multiplies (as the backward's is)
-            if (j < p.T) rope_row(kt, row, p.rcos + (size_t)j * 64, p.rsin + (size_t)j * 64);
-            fence_proxy_async_smem();
-            mbar_arrive(bar_addr(sbase, KREADY + st));
-          }
           float s0 = 0.f, s1 = 0.f;
 #pragma unroll 1
           for (int c = 0; c < 16; ++c) {  // 16-byte chunk c of the row
@@ -326,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= 8) {
-    regs_dec<kPro ? kRegsLowPro : kRegsLow>();
+    regs_dec<kRope ? kRegsLowPro : kRegsLow>();
     if (warp == 8 && lane == 0) {
       // ---------------------------------------------------------- TMA producer
       uint32_t kv = 0;
@@ -376,35 +342,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (last_v_par[s] >= 0) mbar_drain(bar_addr(sbase, VFULL + s), last_v_par[s]);
         if (last_q_par >= 0) mbar_drain(bar_addr(sbase, QFULL), last_q_par);
       }
-    } else if (kVe && warp >= 10) {
-      // ---------------------------------------------------------- value embedding (warps 10-11)
-      // v <- v + 2 sigmoid(g) ve on each V tile, rows vr and vr + 64 per thread
-      const int vr = threadIdx.x - 320;
-      uint32_t kv = 0;
-      bool ok = true;
-      for (int r = 0; ok; ++r) {
-        const int u = unit_index(cta, r, G);
-        if (u >= p.n_units) break;
-        const Unit U = decode(p, u);
-        for (int it = 0; it < U.N; ++it, ++kv) {
-          const int n = U.hi_u - it;
-          const int vs = kv % kVStages, vph = (kv / kVStages) & 1;
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_addr(sbase, VFULL + vs), vph, abort_flag, p.wait_ns))) {
-            ok = false;
-            break;
-          }
-#pragma unroll 1
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int row = vr + 64 * h2, j = n * 128 + row;
-            if (j < p.T) {
-              const size_t tok = ((size_t)U.b * p.T + j) * (p.H / p.grp) + U.hk;
-              ve_row(sbase + kV + vs * kTile, row, p.ve + tok * 128, ve_gate(p.vg[tok]), p.wide_ve);
-            }
-          }
-          fence_proxy_async_smem();
-          mbar_arrive(bar_addr(sbase, VREADY + vs));
-        }
-      }
     } else if (warp == 9 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t id_qk = idesc_bf16(128, 128, 0, 0);
@@ -437,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(bar_addr(sbase, kRope ? QREADY : QFULL), uidx & 1, abort_flag, p.wait_ns)) break;
         {
           const int st = kv % kKStages, ph = (kv / kKStages) & 1;
-          if (!mbar_wait(bar_addr(sbase, (kRope ? KREADY : KFULL) + st), ph, abort_flag, p.wait_ns)) break;
+          if (!mbar_wait(bar_addr(sbase, KFULL + st), ph, abort_flag, p.wait_ns)) break;
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 2; ++k)
@@ -457,10 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int vsn = kvn % kVStages, vphn = (kvn / kVStages) & 1;
           const int stx = kvx % kKStages, phx = (kvx / kKStages) & 1;
           const bool has_next = it + 1 < U.N;
-          if (!mbar_wait(bar_addr(sbase, (kVe ? VREADY : VFULL) + vsn), vphn, abort_flag, p.wait_ns)) {
-            ok = false;
-            break;
-          }
+          if (!mbar_wait(bar_addr(sbase, VFULL + vsn), vphn, abort_flag, p.wait_ns)) { ok = false; break; }
           bool k_next_ready = false;
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
@@ -476,10 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (k == 1) mma_commit(bar_addr(sbase, VEMPTY + vsn));
             if (has_next && U.in(k, n - 1)) {
               if (!k_next_ready) {
-                if (!mbar_wait(bar_addr(sbase, (kRope ? KREADY : KFULL) + stx), phx, abort_flag, p.wait_ns)) {
-                  ok = false;
-                  break;
-                }
+                if (!mbar_wait(bar_addr(sbase, KFULL + stx), phx, abort_flag, p.wait_ns)) { ok = false; break; }
                 k_next_ready = true;
               }
               tc_fence_after();
@@ -505,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_drain(bar_addr(sbase, FINAL), 0);
     }
   } else {
-    regs_inc<kPro ? kRegsHighPro : kRegsHigh>();
+    regs_inc<kRope ? kRegsHighPro : kRegsHigh>();
     // ------------------------------------------------------------ softmax warpgroups
     const int k = warp / 4;
     const int row = threadIdx.x & 127;

@@ -55,28 +55,39 @@ class Stack:
             with_ve = any("ve" in L for L in layers)
             self.ws_bwd = torch.empty(attn.bwd_rope_workspace_bytes(B, T, H, D, Hkv, with_ve), dtype=torch.uint8,
                                       device=dev)
+            # the forward's pre-pass output fits in the backward's workspace, and the
+            # two run one after the other on the same stream
+            assert attn.fwd_rope_workspace_bytes(B, T, Hkv, D, with_ve) <= self.ws_bwd.numel()
             for L, O in zip(layers, self.out):
                 if "ve" in L:
                     O["dve"] = torch.empty_like(L["ve"])
                     O["dg"] = torch.empty((B, T, Hkv), dtype=torch.float32, device=dev)
 
+    def forward_layer(self, l: int):
+        L, O, w = self.layers[l], self.out[l], self.windows[l]
+        if self.rope is None:
+            attn.fwd(L["q"], L["k"], L["v"], w, self.eps, self.scale, out=O["o"], lse=O["lse"])
+        else:
+            attn.fwd_rope(L["q"], L["k"], L["v"], self.rope[0], self.rope[1], w, self.eps, self.scale,
+                          ve=L.get("ve"), ve_gate=L.get("g"), out=O["o"], lse=O["lse"], workspace=self.ws_bwd)
+
+    def backward_layer(self, l: int):
+        L, O, w = self.layers[l], self.out[l], self.windows[l]
+        if self.rope is None:
+            attn.bwd(L["q"], L["k"], L["v"], O["o"], L["dO"], O["lse"], w, self.eps, self.scale,
+                     dq=O["dq"], dk=O["dk"], dv=O["dv"], workspace=self.ws_bwd)
+        else:
+            attn.bwd_rope(L["q"], L["k"], L["v"], O["o"], L["dO"], O["lse"], self.rope[0], self.rope[1], w,
+                          self.eps, self.scale, ve=L.get("ve"), ve_gate=L.get("g"), dq=O["dq"], dk=O["dk"],
+                          dv=O["dv"], dve=O.get("dve"), dgate=O.get("dg"), workspace=self.ws_bwd)
+
     def forward(self):
-        for L, O, w in zip(self.layers, self.out, self.windows):
-            if self.rope is None:
-                attn.fwd(L["q"], L["k"], L["v"], w, self.eps, self.scale, out=O["o"], lse=O["lse"])
-            else:
-                attn.fwd_rope(L["q"], L["k"], L["v"], self.rope[0], self.rope[1], w, self.eps, self.scale,
-                              ve=L.get("ve"), ve_gate=L.get("g"), out=O["o"], lse=O["lse"])
+        for l in range(len(self.layers)):
+            self.forward_layer(l)
 
     def backward(self):
-        for L, O, w in zip(reversed(self.layers), reversed(self.out), reversed(self.windows)):
-            if self.rope is None:
-                attn.bwd(L["q"], L["k"], L["v"], O["o"], L["dO"], O["lse"], w, self.eps, self.scale,
-                         dq=O["dq"], dk=O["dk"], dv=O["dv"], workspace=self.ws_bwd)
-            else:
-                attn.bwd_rope(L["q"], L["k"], L["v"], O["o"], L["dO"], O["lse"], self.rope[0], self.rope[1], w,
-                              self.eps, self.scale, ve=L.get("ve"), ve_gate=L.get("g"), dq=O["dq"], dk=O["dk"],
-                              dv=O["dv"], dve=O.get("dve"), dgate=O.get("dg"), workspace=self.ws_bwd)
+        for l in reversed(range(len(self.layers))):
+            self.backward_layer(l)
 
     def step(self):
         self.forward()
