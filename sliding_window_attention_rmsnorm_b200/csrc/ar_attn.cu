@@ -23,7 +23,7 @@
 
 namespace {
 
-constexpr int kD = 128;
+constexpr int kD = 128;  // the head dimension of the RoPE and no-alloc paths; the others take 64 or 128
 constexpr int kMaxDevices = 64;
 
 struct DeviceInfo {
@@ -73,8 +73,12 @@ int device_setup(int* sms_out, int* prep_blocks_out = nullptr) {
                fwd_attr(ar::fwd::fwd_kernel<false, true>) != cudaSuccess ||
                fwd_attr(ar::fwd::fwd_kernel<true, false, true>) != cudaSuccess ||
                fwd_attr(ar::fwd::fwd_kernel<false, false, true>) != cudaSuccess ||
+               fwd_attr(ar::fwd::fwd_kernel<true, false, false, 64>) != cudaSuccess ||
+               fwd_attr(ar::fwd::fwd_kernel<false, false, false, 64>) != cudaSuccess ||
                bwd_attr(ar::bwd::bwd_kernel<0>) != cudaSuccess || bwd_attr(ar::bwd::bwd_kernel<1>) != cudaSuccess ||
-               bwd_attr(ar::bwd::bwd_kernel<3>) != cudaSuccess ||
+               bwd_attr(ar::bwd::bwd_kernel<3>) != cudaSuccess || bwd_attr(ar::bwd::bwd_kernel<0, 64>) != cudaSuccess ||
+               cudaFuncSetAttribute(ar::dqk::dq_kernel<false, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    ar::dqk::kSmemBytes) != cudaSuccess ||
                cudaFuncSetAttribute(ar::dqk::dq_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     ar::dqk::kSmemBytes) != cudaSuccess ||
                cudaFuncSetAttribute(ar::dqk::dq_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -89,15 +93,19 @@ int device_setup(int* sms_out, int* prep_blocks_out = nullptr) {
       if (!fwd_regs_ok(ar::fwd::fwd_kernel<true, false>) || !fwd_regs_ok(ar::fwd::fwd_kernel<false, false>) ||
           !fwd_regs_ok(ar::fwd::fwd_kernel<true, true>) || !fwd_regs_ok(ar::fwd::fwd_kernel<false, true>) ||
           !fwd_regs_ok(ar::fwd::fwd_kernel<true, false, true>) ||
-          !fwd_regs_ok(ar::fwd::fwd_kernel<false, false, true>))
+          !fwd_regs_ok(ar::fwd::fwd_kernel<false, false, true>) ||
+          !fwd_regs_ok(ar::fwd::fwd_kernel<true, false, false, 64>) ||
+          !fwd_regs_ok(ar::fwd::fwd_kernel<false, false, false, 64>))
         d.status = AR_ERR_CUDA;
-      for (BwdKernel f : {ar::bwd::bwd_kernel<0>, ar::bwd::bwd_kernel<1>, ar::bwd::bwd_kernel<3>}) {
+      for (BwdKernel f : {ar::bwd::bwd_kernel<0>, ar::bwd::bwd_kernel<1>, ar::bwd::bwd_kernel<3>,
+                          ar::bwd::bwd_kernel<0, 64>}) {
         cudaFuncAttributes ba;
         if (cudaFuncGetAttributes(&ba, f) != cudaSuccess || ba.numRegs != ar::bwd::kLaunchRegs) d.status = AR_ERR_CUDA;
       }
     }
     if (d.status == AR_OK &&
-        (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.prep_blocks, ar::bwd_prep_kernel, 256, 0) != cudaSuccess ||
+        (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.prep_blocks, ar::bwd_prep_kernel<128>, 256, 0) !=
+             cudaSuccess ||
          d.prep_blocks < 1))
       d.status = AR_ERR_CUDA;
     if (!g_encode && d.status == AR_OK) {
@@ -124,13 +132,14 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-int check_shape(int B, int T, int H, int D) {
+// Head dimensions 64 and 128 (d128_only: the paths built for 128 alone).
+int check_shape(int B, int T, int H, int D, bool d128_only = false) {
   if (B <= 0 || T <= 0 || H <= 0) return AR_ERR_SHAPE;
-  if (D != kD) return AR_ERR_UNSUPPORTED;
+  if (D != 128 && (d128_only || D != 64)) return AR_ERR_UNSUPPORTED;
   const long long T_pad = (T + 127LL) / 128 * 128;
   // all element indices must fit comfortably in 63 bits and unit counts in int
   if ((long long)B * H * T_pad > (1LL << 31) / 2) return AR_ERR_SHAPE;
-  if ((long long)B * T * H * kD > (1LL << 40)) return AR_ERR_SHAPE;
+  if ((long long)B * T * H * D > (1LL << 40)) return AR_ERR_SHAPE;
   return AR_OK;
 }
 
@@ -145,11 +154,12 @@ int effective_window(int window, int T) { return (window < 0 || window >= T - 1)
 // Grouped K/V heads: Hkv divides H (Hkv = H is multi-head attention).
 int check_kv_heads(int H, int Hkv) { return (Hkv >= 1 && Hkv <= H && H % Hkv == 0) ? AR_OK : AR_ERR_SHAPE; }
 
-// [B, T, H, 128] bf16 viewed as a 4-D tensor (d, h, t, b); boxes of 64 x 1 x 128 x 1
-// land as 128 rows of 128 bytes with the 128-byte swizzle the MMA descriptors expect.
-int make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
-  cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)T * H * kD * 2};
+// [B, T, H, D] bf16 viewed as a 4-D tensor (d, h, t, b); boxes of 64 x 1 x 128 x 1
+// land as 128 rows of 128 bytes with the 128-byte swizzle the MMA descriptors
+// expect (D / 64 boxes per tile).
+int make_map(CUtensorMap* m, const void* base, int B, int T, int H, int D = kD) {
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
   cuuint32_t box[4] = {64, 1, 128, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
@@ -159,7 +169,7 @@ int make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
 }
 
 ar::FwdParams fwd_params(void* o, float* lse, const float* ck, int B, int T, int H, int Hkv, int window,
-                         float eps, float scale) {
+                         float eps, float scale, int D = kD) {
   ar::FwdParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.rcos = p.rsin = nullptr;
@@ -174,7 +184,7 @@ ar::FwdParams fwd_params(void* o, float* lse, const float* ck, int B, int T, int
   p.nqp = (T + 255) / 256;
   p.n_units = B * H * p.nqp;
   p.eps = eps;
-  p.bound = scale * 128.0f * 1.4426950408889634f;
+  p.bound = scale * (float)D * 1.4426950408889634f;
   p.cscale = scale * 1.4426950408889634f;
   p.wide = aligned(o, 32);
   p.wait_ns = g_wait_ns.load();
@@ -185,10 +195,14 @@ ar::FwdParams fwd_params(void* o, float* lse, const float* ck, int B, int T, int
 // (see fwd.cuh), else the running-max forward; key factors computed in the
 // kernel, or (ck_global) read from p.ck; rope_q: Q tiles rotated in the kernel.
 void launch_fwd(int grid, cudaStream_t s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                const ar::FwdParams& p, bool ck_global, bool rope_q = false) {
+                const ar::FwdParams& p, bool ck_global, bool rope_q = false, int D = kD) {
   using namespace ar::fwd;
   const bool fixed = p.bound <= kFixedBoundMax;
-  if (rope_q && fixed)
+  if (D == 64 && fixed)
+    fwd_kernel<true, false, false, 64><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
+  else if (D == 64)
+    fwd_kernel<false, false, false, 64><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
+  else if (rope_q && fixed)
     fwd_kernel<true, false, true><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
   else if (rope_q)
     fwd_kernel<false, false, true><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
@@ -332,22 +346,22 @@ int ar_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float*
   if ((st = device_setup(&sms)) != AR_OK) return st;
 
   CUtensorMap tq, tk, tv;
-  if (make_map(&tq, q, B, T, H) != AR_OK || make_map(&tk, k, B, T, Hkv) != AR_OK ||
-      make_map(&tv, v, B, T, Hkv) != AR_OK)
+  if (make_map(&tq, q, B, T, H, D) != AR_OK || make_map(&tk, k, B, T, Hkv, D) != AR_OK ||
+      make_map(&tv, v, B, T, Hkv, D) != AR_OK)
     return AR_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const ar::FwdParams p = fwd_params(o, lse, nullptr, B, T, H, Hkv, window, eps, scale);
+  const ar::FwdParams p = fwd_params(o, lse, nullptr, B, T, H, Hkv, window, eps, scale, D);
   const int grid = p.n_units < sms ? p.n_units : sms;
   {
     KernelTimer t(AR_KERNEL_FWD, s);
-    launch_fwd(grid, s, tq, tk, tv, p, false);
+    launch_fwd(grid, s, tq, tk, tv, p, false, false, D);
     t.stop();
   }
   return cudaGetLastError() == cudaSuccess ? AR_OK : AR_ERR_CUDA;
 }
 
 size_t ar_attn_fwd_rope_workspace_bytes(int B, int T, int Hkv, int D, int with_ve) {
-  if (check_shape(B, T, Hkv, D) != AR_OK) return 0;
+  if (check_shape(B, T, Hkv, D, true) != AR_OK) return 0;
   return round_up((size_t)B * T * Hkv * kD * 2, 256) * (with_ve ? 2 : 1);
 }
 
@@ -357,7 +371,7 @@ int ar_attn_fwd_rope(const void* q, const void* k, const void* v, void* o, float
                      void* stream) {
   if (!q || !k || !v || !o || !rope_cos || !rope_sin) return AR_ERR_NULL;  // lse may be NULL: not stored
   if ((ve == nullptr) != (ve_gate == nullptr)) return AR_ERR_NULL;
-  int st = check_shape(B, T, H, D);
+  int st = check_shape(B, T, H, D, true);
   if (st != AR_OK) return st;
   if ((st = check_kv_heads(H, Hkv)) != AR_OK) return st;
   if (rope_rows < T) return AR_ERR_SHAPE;
@@ -433,8 +447,8 @@ size_t rope_bytes(int B, int T, int H, int Hkv, bool with_ve) {
 }
 
 int bwd_run(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
-            void* dk, void* dv, int B, int T, int H, int Hkv, int window, float eps, float scale, void* workspace,
-            size_t need, void* stream, const RopeArgs* ra) {
+            void* dk, void* dv, int B, int T, int H, int Hkv, int D, int window, float eps, float scale,
+            void* workspace, size_t need, void* stream, const RopeArgs* ra) {
   int sms = 0, prep_blocks = 1;
   int st = device_setup(&sms, &prep_blocks);
   if (st != AR_OK) return st;
@@ -472,18 +486,23 @@ int bwd_run(const void* q, const void* k, const void* v, const void* o, const vo
     if (ra->ve) vx = vm;
   }
   CUtensorMap tq, tk, tv, tdo;
-  if (make_map(&tq, qx, B, T, H) != AR_OK || make_map(&tk, kx, B, T, Hkv) != AR_OK ||
-      make_map(&tv, vx, B, T, Hkv) != AR_OK || make_map(&tdo, dO, B, T, H) != AR_OK) {
+  if (make_map(&tq, qx, B, T, H, D) != AR_OK || make_map(&tk, kx, B, T, Hkv, D) != AR_OK ||
+      make_map(&tv, vx, B, T, Hkv, D) != AR_OK || make_map(&tdo, dO, B, T, H, D) != AR_OK) {
     if (!workspace) cudaFreeAsync(ws, s);
     return AR_ERR_CUDA;
   }
 
   {
     KernelTimer t(AR_KERNEL_BWD_PREP, s);
-    ar::bwd_prep_kernel<<<bwd_prep_grid(rows, sms, prep_blocks), 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(qx), static_cast<const __nv_bfloat16*>(o),
-        static_cast<const __nv_bfloat16*>(dO), lse, lse2, delta, rq, B, T, H, T_pad, eps,
-        aligned(qx, 32) && aligned(o, 32) && aligned(dO, 32));
+    const int wide = aligned(qx, 32) && aligned(o, 32) && aligned(dO, 32);
+    if (D == 64)
+      ar::bwd_prep_kernel<64><<<bwd_prep_grid(rows, sms, prep_blocks), 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(qx), static_cast<const __nv_bfloat16*>(o),
+          static_cast<const __nv_bfloat16*>(dO), lse, lse2, delta, rq, B, T, H, T_pad, eps, wide);
+    else
+      ar::bwd_prep_kernel<128><<<bwd_prep_grid(rows, sms, prep_blocks), 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(qx), static_cast<const __nv_bfloat16*>(o),
+          static_cast<const __nv_bfloat16*>(dO), lse, lse2, delta, rq, B, T, H, T_pad, eps, wide);
     t.stop();
   }
   const int w = effective_window(window, T);
@@ -538,7 +557,9 @@ int bwd_run(const void* q, const void* k, const void* v, const void* o, const vo
     {
       KernelTimer t(AR_KERNEL_BWD, s);
       const int grid = std::min(p.n_units, sms);
-      if (pro == 0)
+      if (D == 64)
+        ar::bwd::bwd_kernel<0, 64><<<grid, ar::bwd::kThreads, ar::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo, tg, p);
+      else if (pro == 0)
         ar::bwd::bwd_kernel<0><<<grid, ar::bwd::kThreads, ar::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo, tg, p);
       else if (pro == 1)
         ar::bwd::bwd_kernel<1><<<grid, ar::bwd::kThreads, ar::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo, tg, p);
@@ -570,7 +591,9 @@ int bwd_run(const void* q, const void* k, const void* v, const void* o, const vo
     {
       KernelTimer t(AR_KERNEL_DQ, s);
       const int grid = std::min(d.n_units, sms);
-      if (ra)
+      if (D == 64)
+        ar::dqk::dq_kernel<false, 64><<<grid, ar::dqk::kThreads, ar::dqk::kSmemBytes, s>>>(tg, tk, d);
+      else if (ra)
         ar::dqk::dq_kernel<true><<<grid, ar::dqk::kThreads, ar::dqk::kSmemBytes, s>>>(tg, tk, d);
       else
         ar::dqk::dq_kernel<false><<<grid, ar::dqk::kThreads, ar::dqk::kSmemBytes, s>>>(tg, tk, d);
@@ -600,10 +623,12 @@ int ar_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, 
   const size_t need = ar_attn_bwd_gqa_workspace_bytes(B, T, H, Hkv, D);
   if (workspace && workspace_bytes < need) return AR_ERR_WORKSPACE;
   if (workspace && !aligned(workspace, 256)) return AR_ERR_ALIGN;
-  return bwd_run(q, k, v, o, dO, lse, dq, dk, dv, B, T, H, Hkv, window, eps, scale, workspace, need, stream, nullptr);
+  return bwd_run(q, k, v, o, dO, lse, dq, dk, dv, B, T, H, Hkv, D, window, eps, scale, workspace, need, stream,
+                 nullptr);
 }
 
 size_t ar_attn_bwd_rope_workspace_bytes(int B, int T, int H, int Hkv, int D, int with_ve) {
+  if (D != kD) return 0;
   const size_t base = ar_attn_bwd_gqa_workspace_bytes(B, T, H, Hkv, D);
   return base ? base + rope_bytes(B, T, H, Hkv, with_ve != 0) : 0;
 }
@@ -616,7 +641,7 @@ int ar_attn_bwd_rope(const void* q, const void* k, const void* v, const void* o,
   const bool with_ve = ve != nullptr;
   if (with_ve && (!ve_gate || !dve || !dgate)) return AR_ERR_NULL;
   if (!with_ve && (ve_gate || dve || dgate)) return AR_ERR_NULL;
-  int st = check_shape(B, T, H, D);
+  int st = check_shape(B, T, H, D, true);
   if (st != AR_OK) return st;
   if ((st = check_kv_heads(H, Hkv)) != AR_OK) return st;
   if (rope_rows < T) return AR_ERR_SHAPE;
@@ -636,7 +661,8 @@ int ar_attn_bwd_rope(const void* q, const void* k, const void* v, const void* o,
   ra.vg = static_cast<const __nv_bfloat16*>(ve_gate);
   ra.dve = static_cast<__nv_bfloat16*>(dve);
   ra.dg = dgate;
-  return bwd_run(q, k, v, o, dO, lse, dq, dk, dv, B, T, H, Hkv, window, eps, scale, workspace, need, stream, &ra);
+  return bwd_run(q, k, v, o, dO, lse, dq, dk, dv, B, T, H, Hkv, D, window, eps, scale, workspace, need, stream,
+                 &ra);
 }
 
 int ar_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
@@ -774,7 +800,7 @@ int noalloc_scratch(float** out) {
 extern "C" int ar_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T,
                                    int H, int D, int window, float eps, float scale, void* stream) {
   if (!q || !k || !v || !o) return AR_ERR_NULL;  // lse may be NULL: not stored
-  int st = check_shape(B, T, H, D);
+  int st = check_shape(B, T, H, D, true);
   if (st != AR_OK) return st;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return AR_ERR_ALIGN;

@@ -84,32 +84,45 @@ __device__ __forceinline__ void dot_bf16x8_f32(float& c0, float& c1, const uint4
         : "r"(wa[e]), "r"(wb[e]));
 }
 
-// One row (one token of one head, 128 elements) per 8 lanes, 32 bytes of each
-// of q, o and dO per lane: 256-bit loads when the tensors are 32-byte aligned.
+// One row (one token of one head, D = 128 or 64 elements) per 8 lanes, D / 4
+// bytes of each of q, o and dO per lane: 256-bit loads (D = 128) when the
+// tensors are 32-byte aligned, 128-bit loads otherwise.
+template <int kD>
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ o,
                                 const __nv_bfloat16* __restrict__ dO, const float* __restrict__ lse,
                                 float* __restrict__ lse2, float* __restrict__ delta, float* __restrict__ rq, int B,
                                 int T, int H, int T_pad, float eps, int wide) {
+  static_assert(kD == 64 || kD == 128, "head dimension 64 or 128");
   const long long rows = (long long)B * T * H;
   const int sub = threadIdx.x & 7;
   const long long gstride = (long long)gridDim.x * (blockDim.x / 8);
   const float kLog2e = 1.4426950408889634f;
   for (long long r = (long long)blockIdx.x * (blockDim.x / 8) + threadIdx.x / 8; r < rows; r += gstride) {
+    const long long base = r * kD + sub * (kD / 8);
     uint4 q0, q1, o0, o1, d0, d1;
-    ldg32B(q + r * 128 + sub * 16, q0, q1, wide);
-    ldg32B(o + r * 128 + sub * 16, o0, o1, wide);
-    ldg32B(dO + r * 128 + sub * 16, d0, d1, wide);
+    if (kD == 128) {
+      ldg32B(q + base, q0, q1, wide);
+      ldg32B(o + base, o0, o1, wide);
+      ldg32B(dO + base, d0, d1, wide);
+    } else {
+      q0 = __ldg(reinterpret_cast<const uint4*>(q + base));
+      o0 = __ldg(reinterpret_cast<const uint4*>(o + base));
+      d0 = __ldg(reinterpret_cast<const uint4*>(dO + base));
+      q1 = o1 = d1 = make_uint4(0, 0, 0, 0);
+    }
     float s0 = 0.f, s1 = 0.f, t0 = 0.f, t1 = 0.f;
     fma_sq_bf16x2_f32(s0, s1, q0.x);
     fma_sq_bf16x2_f32(s0, s1, q0.y);
     fma_sq_bf16x2_f32(s0, s1, q0.z);
     fma_sq_bf16x2_f32(s0, s1, q0.w);
-    fma_sq_bf16x2_f32(s0, s1, q1.x);
-    fma_sq_bf16x2_f32(s0, s1, q1.y);
-    fma_sq_bf16x2_f32(s0, s1, q1.z);
-    fma_sq_bf16x2_f32(s0, s1, q1.w);
     dot_bf16x8_f32(t0, t1, o0, d0);
-    dot_bf16x8_f32(t0, t1, o1, d1);
+    if (kD == 128) {
+      fma_sq_bf16x2_f32(s0, s1, q1.x);
+      fma_sq_bf16x2_f32(s0, s1, q1.y);
+      fma_sq_bf16x2_f32(s0, s1, q1.z);
+      fma_sq_bf16x2_f32(s0, s1, q1.w);
+      dot_bf16x8_f32(t0, t1, o1, d1);
+    }
     float ss = s0 + s1, dl = t0 + t1;
 #pragma unroll
     for (int m = 4; m > 0; m >>= 1) {
@@ -121,7 +134,7 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_
       split_row(r, T, H, b, t, h);
       const long long bh = (long long)b * H + h;
       delta[bh * T_pad + t] = dl;
-      rq[bh * T_pad + t] = rsqrtf(ss * (1.0f / 128.0f) + eps);
+      rq[bh * T_pad + t] = rsqrtf(ss * (1.0f / kD) + eps);
       lse2[bh * T_pad + t] = lse[bh * T + t] * kLog2e;
     }
   }

@@ -50,9 +50,9 @@
 namespace ar {
 
 struct BwdParams {
-  __nv_bfloat16* dk;       // [B, T, Hkv, 128]
-  __nv_bfloat16* dv;       // [B, T, Hkv, 128]
-  const __nv_bfloat16* k;  // [B, T, Hkv, 128] raw keys, for the dk epilogue
+  __nv_bfloat16* dk;       // [B, T, Hkv, D]
+  __nv_bfloat16* dv;       // [B, T, Hkv, D]
+  const __nv_bfloat16* k;  // [B, T, Hkv, D] raw keys, for the dk epilogue
   const float* lse2;       // [B*H, T_pad] lse * log2(e), 0 on padding
   const float* delta;      // [B*H, T_pad] rowsum(dO * o), 0 on padding
   const float* rq;         // [B*H, T_pad] 1/rms(q_i), 0 on padding
@@ -178,12 +178,20 @@ __device__ __forceinline__ void grad_chunk(const uint32_t (&sv)[32], const uint3
   }
 }
 
-template <int kPro>
+template <int kPro, int kD = 128>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                const __grid_constant__ CUtensorMap tm_g, const BwdParams p) {
   constexpr bool kRope = (kPro & 1) != 0, kVe = (kPro & 2) != 0;
+  // Head dimension kD (64 or 128): K, V, Q and dO tiles are kD / 64 swizzled
+  // halves of 128 rows x 64 elements in their 32 KB slots; S^T and dP^T take
+  // kD / 16 K-steps; dV and dK use kD of their 128 accumulator columns.
+  static_assert(kD == 64 || kD == 128, "head dimension 64 or 128");
+  static_assert(kD == 128 || kPro == 0, "the RoPE / value-embedding path takes head dimension 128");
+  constexpr int kHalves = kD / 64;
+  constexpr uint32_t kTileBytes = 128u * kD * 2;
+  constexpr float kInvD = 1.0f / kD;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
@@ -237,8 +245,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
         if (uidx > 0 && !mbar_wait(bar_addr(sbase, KVEMPTY), (uidx - 1) & 1, abort_flag, p.wait_ns)) break;
-        mbar_expect_tx(bar_addr(sbase, KVFULL), 2 * kTile);
-        for (int hf = 0; hf < 2; ++hf) {
+        mbar_expect_tx(bar_addr(sbase, KVFULL), 2 * kTileBytes);
+        for (int hf = 0; hf < kHalves; ++hf) {
           tma_load_4d(sbase + kK + hf * kHalf, &tm_k, bar_addr(sbase, KVFULL), hf * 64, U.h, U.kt * 128, U.b);
           tma_load_4d(sbase + kV + hf * kHalf, &tm_v, bar_addr(sbase, KVFULL), hf * 64, U.h, U.kt * 128, U.b);
         }
@@ -247,8 +255,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int qt = U.qtile(it), hq = U.h * p.grp + U.qhead(it);
           const int st = qc & 1, ph = (qc >> 1) & 1;
           if (!mbar_wait(bar_addr(sbase, QEMPTY + st), ph ^ 1, abort_flag, p.wait_ns)) { ok = false; break; }
-          mbar_expect_tx(bar_addr(sbase, QFULL + st), 2 * kTile);
-          for (int hf = 0; hf < 2; ++hf) {
+          mbar_expect_tx(bar_addr(sbase, QFULL + st), 2 * kTileBytes);
+          for (int hf = 0; hf < kHalves; ++hf) {
             tma_load_4d(sbase + kQ + st * kTile + hf * kHalf, &tm_q, bar_addr(sbase, QFULL + st), hf * 64, hq,
                         qt * 128, U.b);
             tma_load_4d(sbase + kDO + st * kTile + hf * kHalf, &tm_do, bar_addr(sbase, QFULL + st), hf * 64, hq,
@@ -294,12 +302,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 13 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t id_s = idesc_bf16(128, 64, 0, 0);     // S^T, dP^T: both K-major, N = 64 queries
-      constexpr uint32_t id_acc = idesc_bf16(128, 128, 0, 1);  // dV, dK: A K-major, B MN-major
+      constexpr uint32_t id_acc = idesc_bf16(128, kD, 0, 1);  // dV, dK: A K-major, B MN-major
       const uint32_t tDV = tbase + 256, tDK = tbase + 384;
       auto issue_s = [&](int a, int st) {  // S_a^T = K Q_a^T
         const uint32_t qa = sbase + kQ + st * kTile + a * 64 * 128;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
           mma_ss(tbase + 64 * a, sdesc_sw128(sbase + kK + off, 16, 1024), sdesc_sw128(qa + off, 16, 1024), id_s,
                  kk > 0);
@@ -308,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_dp = [&](int a, int st) {  // dP_a^T = V dO_a^T
         const uint32_t da = sbase + kDO + st * kTile + a * 64 * 128;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
           mma_ss(tbase + 128 + 64 * a, sdesc_sw128(sbase + kV + off, 16, 1024), sdesc_sw128(da + off, 16, 1024),
                  id_s, kk > 0);
@@ -404,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
           float ss[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf)
+          for (int hf = 0; hf < kHalves; ++hf)
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               const uint4 v = lds128(sbase + kK + hf * kHalf + sw128(row, c));
@@ -416,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ss[e] = fmaf(x1, x1, ss[e]);
               }
             }
-          rk = rsqrtf((ss[0] + ss[1] + ss[2] + ss[3]) * (1.0f / 128.0f) + p.eps);
+          rk = rsqrtf((ss[0] + ss[1] + ss[2] + ss[3]) * kInvD + p.eps);
         }
         mbar_arrive(bar_addr(sbase, KVEMPTY));  // done reading K from shared memory
         const float Cj = rk * p.scale * kLog2e;
@@ -486,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               ok = false;
               break;
             }
-            sts_f32(sbase + kDot + 4 * (128 * a + row), (dt0 + dt1) * rk * rk * (1.0f / 128.0f));
+            sts_f32(sbase + kDot + 4 * (128 * a + row), (dt0 + dt1) * rk * rk * kInvD);
           }
           tmem_wait_st();
           fence_proxy_async_smem();
@@ -509,17 +517,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Unit U = decode(p, u);
         // ------------------------------------------------------------ dK, dV epilogue
         const int j = U.kt * 128 + row;
-        const size_t orow = (((size_t)U.b * p.T + (j < p.T ? j : 0)) * p.Hkv + U.h) * 128;
+        const size_t orow = (((size_t)U.b * p.T + (j < p.T ? j : 0)) * p.Hkv + U.h) * kD;
         const bool jv = j < p.T;
         // dk = scale (acc - coef k), coef = rk^2 (acc . k) / D, with acc . k summed by
         // the compute warpgroups as sum_i G_ij S_ij; the raw key row is loaded into
         // registers before the wait, so its latency is hidden by the unit's products
         {
-          uint4 kv[16];
+          uint4 kv[kD / 8];
           {
             const uint4* krow = reinterpret_cast<const uint4*>(p.k + orow);
 #pragma unroll
-            for (int c = 0; c < 16; c += 2) {
+            for (int c = 0; c < kD / 8; c += 2) {
               if (jv) {
                 ldg32B(krow + c, kv[c], kv[c + 1], p.wide_k);
               } else {
@@ -534,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(bar_addr(sbase, DOTFREE));
           if constexpr (!kRope) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < kD / 32; ++c) {
               uint32_t x[32];
               tmem_ld32(tDK + 32 * c, x);
               tmem_wait_ld();
@@ -598,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if constexpr (!kVe) {
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < kD / 32; ++c) {
             uint32_t x[32];
             tmem_ld32(tDV + 32 * c, x);
             tmem_wait_ld();

@@ -36,10 +36,10 @@
 namespace ar {
 
 struct DqParams {
-  const __nv_bfloat16* q;  // [B, T, H, 128]
+  const __nv_bfloat16* q;  // [B, T, H, D]
   const __nv_bfloat16* rcos;  // kRope: rotary tables [>= T, 64], row t = position t
   const __nv_bfloat16* rsin;
-  __nv_bfloat16* dq;       // [B, T, H, 128]
+  __nv_bfloat16* dq;       // [B, T, H, D]
   int B, T, H;
   int grp;         // query heads per K/V head: k has H / grp heads (1: multi-head)
   int w;           // left window (w >= T means full causal)
@@ -101,9 +101,15 @@ __device__ __forceinline__ long long g_slot(const DqParams& p, int hl, int qt, i
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t sbase, int i) { return sbase + kBar + 8u * i; }
 
-template <bool kRope>
+template <bool kRope, int kD = 128>
 __global__ void __launch_bounds__(kThreads, 1)
     dq_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_k, const DqParams p) {
+  // Head dimension kD (64 or 128): K tiles are kD / 64 swizzled halves in their
+  // 32 KB slots and the accumulator uses kD of its 128 columns.
+  static_assert(kD == 64 || kD == 128, "head dimension 64 or 128");
+  static_assert(kD == 128 || !kRope, "the RoPE path takes head dimension 128");
+  constexpr int kHalves = kD / 64;
+  constexpr float kInvD = 1.0f / kD;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -149,14 +155,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          mbar_expect_tx(bar_addr(sbase, full + s), kTile);
+          mbar_expect_tx(bar_addr(sbase, full + s), is_g ? kTile : 128u * kD * 2);
           if (is_g) {
             const long long slot = g_slot(p, U.hl, U.qt, kt);
             for (int hf = 0; hf < 2; ++hf)
               tma_load_2d(sbase + kG + s * kTile + hf * kHalf, &tm_g, bar_addr(sbase, full + s), 0,
                           (int)((2 * slot + hf) * 128));
           } else {
-            for (int hf = 0; hf < 2; ++hf)
+            for (int hf = 0; hf < kHalves; ++hf)
               tma_load_4d(sbase + kK + s * kTile + hf * kHalf, &tm_k, bar_addr(sbase, full + s), hf * 64,
                           U.h / p.grp, kt * 128, U.b);
           }
@@ -173,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 5) {
     if (lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      constexpr uint32_t id = idesc_bf16(128, 128, 1, 1);  // A (G) and B (K) both MN-major
+      constexpr uint32_t id = idesc_bf16(128, kD, 1, 1);  // A (G) and B (K) both MN-major
       const uint64_t dA = sdesc_sw128(sbase + kG, kHalf, 1024), dB = sdesc_sw128(sbase + kK, kHalf, 1024);
       uint32_t cg = 0, ck = 0;
       int uidx = 0;
@@ -221,14 +227,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         const int i = U.qt * 128 + row;
         const bool iv = i < p.T;
-        const size_t orow = (((size_t)U.b * p.T + (iv ? i : 0)) * p.H + U.h) * 128;
+        const size_t orow = (((size_t)U.b * p.T + (iv ? i : 0)) * p.H + U.h) * kD;
         // the whole q row, loaded before the wait for the accumulator so that its
         // latency overlaps the products
-        uint4 qv[16];
+        uint4 qv[kD / 8];
         {
           const uint4* qrow = reinterpret_cast<const uint4*>(p.q + orow);
 #pragma unroll
-          for (int c = 0; c < 16; c += 2) {
+          for (int c = 0; c < kD / 8; c += 2) {
             if (iv) {
               ldg32B(qrow + c, qv[c], qv[c + 1], p.wide_q);
             } else {
@@ -246,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // pass 1: (acc . q) and sum q^2
         float ss = 0.f, dot = 0.f;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < kD / 32; ++cc) {
           uint32_t x[32];
           tmem_ld32(tA + 32 * cc, x);
           tmem_wait_ld();
@@ -262,11 +268,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        const float coef = dot * (1.0f / 128.0f) / (ss * (1.0f / 128.0f) + p.eps);
+        const float coef = dot * kInvD / (ss * kInvD + p.eps);
         if constexpr (!kRope) {
           // pass 2: dq = scale (acc - coef q)
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
+          for (int cc = 0; cc < kD / 32; ++cc) {
             uint32_t x[32];
             tmem_ld32(tA + 32 * cc, x);
             tmem_wait_ld();

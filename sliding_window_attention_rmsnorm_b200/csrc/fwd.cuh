@@ -69,7 +69,7 @@
 namespace ar {
 
 struct FwdParams {
-  __nv_bfloat16* o;  // [B, T, H, 128]
+  __nv_bfloat16* o;  // [B, T, H, D]
   const __nv_bfloat16* rcos;  // kRopeQ: rotary tables [>= T, 64] bf16, row t = position t
   const __nv_bfloat16* rsin;
   float* lse;        // [B, H, T], or NULL: not stored (forward-only use)
@@ -197,12 +197,20 @@ __device__ __forceinline__ void rope_row(uint32_t tile, int row, const __nv_bflo
   }
 }
 
-template <bool kFixed, bool kCkGlobal, bool kRopeQ = false>
+template <bool kFixed, bool kCkGlobal, bool kRopeQ = false, int kD = 128>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   constexpr bool kRope = kRopeQ;
   static_assert(!(kRopeQ && kCkGlobal), "the rotation of Q runs on the key-factor warps");
+  // Head dimension kD (64 or 128): a Q, K or V tile is kD / 64 swizzled halves of
+  // 128 rows x 64 elements in its 32 KB slot; QK^T takes kD / 16 K-steps and P V
+  // writes kD accumulator columns.
+  static_assert(kD == 64 || kD == 128, "head dimension 64 or 128");
+  static_assert(!(kD != 128 && (kRopeQ || kCkGlobal)), "RoPE and the no-alloc forward take head dimension 128");
+  constexpr int kHalves = kD / 64;
+  constexpr uint32_t kTileBytes = 128u * kD * 2;
+  constexpr float kInvD = 1.0f / kD;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
@@ -276,14 +284,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int j = n * 128 + row;  // key position
           float s0 = 0.f, s1 = 0.f;
 #pragma unroll 1
-          for (int c = 0; c < 16; ++c) {  // 16-byte chunk c of the row
+          for (int c = 0; c < kD / 8; ++c) {  // 16-byte chunk c of the row
             const uint4 x = lds128(kt + (c >> 3) * kHalf + sw128(row, c & 7));
             fma_sq_bf16x2_f32(s0, s1, x.x);
             fma_sq_bf16x2_f32(s0, s1, x.y);
             fma_sq_bf16x2_f32(s0, s1, x.z);
             fma_sq_bf16x2_f32(s0, s1, x.w);
           }
-          const float ck = (j < p.T) ? rsqrtf((s0 + s1) * (1.0f / 128.0f) + p.eps) * p.cscale : 0.f;
+          const float ck = (j < p.T) ? rsqrtf((s0 + s1) * kInvD + p.eps) * p.cscale : 0.f;
           sts_f32(sbase + kCK + (kv % kCkSlots) * 512 + 4 * row, ck);
           mbar_arrive(bar_addr(sbase, KEMPTY + st));  // done with the K tile
           mbar_arrive(bar_addr(sbase, CKFULL + kv % kCkSlots));
@@ -304,10 +312,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u >= p.n_units) break;
         const Unit U = decode(p, u);
         if (uidx > 0 && !mbar_wait(bar_addr(sbase, QEMPTY), (uidx - 1) & 1, abort_flag, p.wait_ns)) break;
-        mbar_expect_tx(bar_addr(sbase, QFULL), kTile * (U.valid[1] ? 2 : 1));
+        mbar_expect_tx(bar_addr(sbase, QFULL), kTileBytes * (U.valid[1] ? 2 : 1));
         for (int k = 0; k < 2; ++k)
           if (U.valid[k])
-            for (int hf = 0; hf < 2; ++hf)
+            for (int hf = 0; hf < kHalves; ++hf)
               tma_load_4d(sbase + kQ + k * kTile + hf * kHalf, &tm_q, bar_addr(sbase, QFULL), hf * 64, U.h,
                           U.r0[k], U.b);
         last_q_par = uidx & 1;
@@ -315,15 +323,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int n = U.hi_u - it;
           const int st = kv % kKStages, ph = (kv / kKStages) & 1;
           if (!mbar_wait(bar_addr(sbase, KEMPTY + st), ph ^ 1, abort_flag, p.wait_ns)) { ok = false; break; }
-          mbar_expect_tx(bar_addr(sbase, KFULL + st), kTile);
-          for (int hf = 0; hf < 2; ++hf)
+          mbar_expect_tx(bar_addr(sbase, KFULL + st), kTileBytes);
+          for (int hf = 0; hf < kHalves; ++hf)
             tma_load_4d(sbase + kK + st * kTile + hf * kHalf, &tm_k, bar_addr(sbase, KFULL + st), hf * 64, U.hk,
                         n * 128, U.b);
           last_k_par[st] = ph;
           const int vs = kv % kVStages, vph = (kv / kVStages) & 1;
           if (!mbar_wait(bar_addr(sbase, VEMPTY + vs), vph ^ 1, abort_flag, p.wait_ns)) { ok = false; break; }
-          mbar_expect_tx(bar_addr(sbase, VFULL + vs), kTile + (kCkGlobal ? 512 : 0));
-          for (int hf = 0; hf < 2; ++hf)
+          mbar_expect_tx(bar_addr(sbase, VFULL + vs), kTileBytes + (kCkGlobal ? 512 : 0));
+          for (int hf = 0; hf < kHalves; ++hf)
             tma_load_4d(sbase + kV + vs * kTile + hf * kHalf, &tm_v, bar_addr(sbase, VFULL + vs), hf * 64, U.hk,
                         n * 128, U.b);
           if (kCkGlobal)
@@ -345,14 +353,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 9 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t id_qk = idesc_bf16(128, 128, 0, 0);
-      constexpr uint32_t id_pv = idesc_bf16(128, 128, 0, 1);
+      constexpr uint32_t id_pv = idesc_bf16(128, kD, 0, 1);
       // Descriptor bases; every operand below is a base plus a constant byte offset.
       const uint64_t dQ_k = sdesc_sw128(sbase + kQ, 16, 1024), dK_k = sdesc_sw128(sbase + kK, 16, 1024);
       const uint64_t dV_m = sdesc_sw128(sbase + kV, kHalf, 1024);
       auto issue_s = [&](int k, int st) {
         const uint64_t qb = sdesc_add(dQ_k, k * kTile), kb = sdesc_add(dK_k, st * kTile);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
           mma_ss(tbase + 128 * k, sdesc_add(qb, off), sdesc_add(kb, off), id_qk, kk > 0);
         }
@@ -470,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         float ss[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
+        for (int hf = 0; hf < kHalves; ++hf)
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const uint4 v = lds128(qa + hf * kHalf + sw128(row, c));
@@ -482,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               ss[e] = fmaf(b2, b2, ss[e]);
             }
           }
-        rq = rsqrtf((ss[0] + ss[1] + ss[2] + ss[3]) * (1.0f / 128.0f) + p.eps);
+        rq = rsqrtf((ss[0] + ss[1] + ss[2] + ss[3]) * kInvD + p.eps);
       }
       // l: row sum of the exponentials (gives lse); lr: row sum of the same values
       // rounded to bf16 as the P V product sees them (normalises O in the
@@ -608,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               l1 *= alpha;
             }
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < kD / 32; ++c) {
               uint32_t ov[32];
               tmem_ld32(tO + 32 * c, ov);
               tmem_wait_ld();
@@ -652,9 +660,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float l = l0 + l1;
       const float inv = 1.0f / (kFixed ? lr0 + lr1 : l);
       const bool iv = i < p.T;
-      __nv_bfloat16* orow = p.o + (((size_t)U.b * p.T + (iv ? i : 0)) * p.H + U.h) * 128;
+      __nv_bfloat16* orow = p.o + (((size_t)U.b * p.T + (iv ? i : 0)) * p.H + U.h) * kD;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < kD / 32; ++c) {
         uint32_t ov[32];
         tmem_ld32(tO + 32 * c, ov);
         tmem_wait_ld();

@@ -80,7 +80,11 @@ def test_workspace_sizes(L):
     # head (68 MB), 15 heads per group
     assert attn.bwd_workspace_bytes(4, 8192, 8, 128) == 3 * 32 * 8192 * 4 + 15 * 2080 * 32768
     assert attn.bwd_workspace_bytes(0, 200, 1, 128) == 0
-    assert attn.bwd_workspace_bytes(1, 200, 1, 64) == 0
+    # head dimension 64: the same per-token vectors and G tiles (queries x keys)
+    assert attn.bwd_workspace_bytes(1, 200, 1, 64) == attn.bwd_workspace_bytes(1, 200, 1, 128)
+    assert attn.bwd_workspace_bytes(1, 200, 1, 96) == 0
+    # the RoPE paths take head dimension 128 only
+    assert attn.bwd_rope_workspace_bytes(1, 200, 1, 64) == 0 and attn.fwd_rope_workspace_bytes(1, 200, 1, 64) == 0
 
 
 P16 = 1 << 20  # a 16-byte aligned placeholder address; never dereferenced
@@ -108,7 +112,9 @@ def test_fwd_argument_errors(L):
     assert fwd_call(L, B=0) == -2
     assert fwd_call(L, T=-3) == -2
     assert fwd_call(L, H=0) == -2
-    assert fwd_call(L, D=64) == -3
+    assert fwd_call(L, D=96) == -3
+    assert fwd_call(L, D=256) == -3
+    assert fwd_call(L, D=64, B=0) == -2  # 64 is a supported head dimension: validation goes on
     assert fwd_call(L, k=P16 + 8) == -4
     assert fwd_call(L, eps=-1.0) == -5
     assert fwd_call(L, eps=float("nan")) == -5

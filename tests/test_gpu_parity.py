@@ -435,3 +435,32 @@ def test_grouped_kv_heads_equal_duplicated_heads_on_gpu():
         err = np.abs(g[n] - summed)
         assert (err - bound).max() <= 0, (n, err.max())
         assert np.linalg.norm(g[n] - summed) / np.linalg.norm(summed) <= REL_L2
+
+
+# ------------------------------------------------------------------ head dimension 64
+@pytest.mark.parametrize("B,T,H,Hkv,window", [(1, 256, 4, 4, 128), (1, 256, 4, 4, -1), (2, 300, 3, 3, 100),
+                                              (2, 384, 8, 2, 200), (1, 129, 2, 1, 0)])
+def test_head_dim_64(B, T, H, Hkv, window):
+    """HEAD_DIM = 64 ("autoresearch" README (gitee), section 10.1.1: the head
+    dimension is a model parameter; section 10.2.1 lists changing it): whole
+    tensors against the oracle (edge-case bound) and the kernel-arithmetic
+    model; scale 1/sqrt(64)."""
+    xq = synth.layer_inputs(26, 0, B, T, H, 64, roles=("q", "dO"))
+    xk = synth.layer_inputs(26, 1, B, T, Hkv, 64, roles=("k", "v"))
+    x = dict(q=xq["q"], dO=xq["dO"], k=xk["k"], v=xk["v"])
+    g, ref = run_gpu(x, window), run_oracle(x, window)
+    assert g["o"].shape == (B, T, H, 64) and g["dk"].shape == (B, T, Hkv, 64)
+    tag = "D=64 B=%d T=%d H=%d Hkv=%d w=%d" % (B, T, H, Hkv, window)
+    compare(g, ref, H, tag=tag, edge=True)
+    check_model(g, x, window, tag=tag, ref=ref)
+
+
+def test_head_dim_64_full_size_sampled():
+    """B=8, T=2048, H=8, D=64 (the depth-8 model's width 512 in heads of 64),
+    window 1024 and full causal, three whole heads each against the oracle
+    with the stated bar."""
+    B, T, H = 8, 2048, 8
+    for w in (1024, 2048):
+        x = synth.layer_inputs(27, 0 if w == 1024 else 1, B, T, H, 64)
+        heads = [0, 21, B * H - 1]
+        compare(run_gpu(x, w), run_oracle(x, w, heads=heads), H, heads, tag="D=64 full size w=%d" % w)
