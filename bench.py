@@ -30,8 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "attn fwd+bwd TFLOP/s (unmasked) at T=2048 SSSL; % of B200 BF16 peak"
-D = 128
-FWD_FLOPS_PER_PAIR = 4 * D
+D = 128  # head dimension of the stated workloads (a workload may set its own)
 BWD_FACTOR = 2.5
 
 WORKLOADS = {
@@ -55,6 +54,9 @@ WORKLOADS = {
     "layer_s_rope": dict(config=2, B=8, T=2048, H=4, n_layer=1, windows=[1024], rope=True,
                          name="single S layer fwd+bwd with fused RoPE and value embedding, B=8 T=2048 H=4 D=128, "
                               "window 1024"),
+    # head dimension 64 (width 512 in 8 heads of 64): not one of the stated workloads
+    "stack8_d64": dict(config=3, B=8, T=2048, H=8, D=64, n_layer=8, pattern="SSSL",
+                       name="8-layer SSSL attention stack fwd+bwd, B=8 T=2048 H=8 D=64 (windows 1024/full)"),
     # grouped K/V heads (n_kv_head = n_head / 2): not one of the stated workloads
     "stack8_gqa": dict(config=3, B=8, T=2048, H=4, Hkv=2, n_layer=8, pattern="SSSL",
                        name="8-layer SSSL attention stack fwd+bwd, B=8 T=2048 H=4 Hkv=2 D=128 (windows 1024/full)"),
@@ -101,9 +103,14 @@ def pairs(T, w):
     return n1 * (n1 + 1) // 2 + (T - n1) * (w + 1)
 
 
+def head_dim(wl):
+    return wl.get("D", D)
+
+
 def step_flops(wl, windows):
-    """(forward, backward) counted FLOPs of one step of the workload."""
-    f = sum(wl["B"] * wl["H"] * pairs(wl["T"], w) * FWD_FLOPS_PER_PAIR for w in windows)
+    """(forward, backward) counted FLOPs of one step of the workload: 4 D per
+    visible (query, key) pair forward, 2.5 times that backward."""
+    f = sum(wl["B"] * wl["H"] * pairs(wl["T"], w) * 4 * head_dim(wl) for w in windows)
     return f, BWD_FACTOR * f
 
 
@@ -116,11 +123,24 @@ def measured_peaks():
     return dict(bf16_burst=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
 
 
-# DRAM bytes (read + write) per launch from one ncu capture of each kernel on a
-# single layer of B=8 T=2048 H=4 (window 1024, and full causal), valid only
-# while the kernel's sources are byte-identical to the ones captured.  Keyed
-# by kernel, then by (B, T, H, window).
-CAPTURED_TRAFFIC = {}
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
+# ncu capture of each kernel on one S layer and one L layer (B=8 T=2048 H=4
+# D=128; windows 1024 and full), each record valid while the sha256 of every
+# source the kernel is built from still matches:
+#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum --clock-control none \
+#       -k regex:"fwd_kernel|bwd_kernel|dq_kernel|bwd_prep" -s 12 -c 4 --csv \
+#       python bench.py --workload layer_s|layer_l --steps 1 --warmup 3 --no-e2e --no-cpu-baseline
+# ncu flushes the caches before each launch: these are cold-L2 bytes.
+CAPTURED_TRAFFIC = {
+    "fwd": {"sources": {"fwd.cuh": "3238025202dbfa4b90f4191cc23f00fee4f82c3a8e466925ab65278e0af5173d", "sm100.cuh": "1111847c6474fba79ab804963ad60d50973f7689121be5d4af96fe31bc24aafe", "ar_attn.cu": "7833bea0879ccfffcebd2789594852d103d4a56c299b908fa5908aed02333a06"},
+           "bytes": {(8, 2048, 4, 1024): 52025088, (8, 2048, 4, 2048): 51795712}},
+    "bwd": {"sources": {"bwd.cuh": "7426e2685f4cdc42d91d97bbbef77aabcd18e68298d2d94892f6ff9d81a0ea60", "sm100.cuh": "1111847c6474fba79ab804963ad60d50973f7689121be5d4af96fe31bc24aafe", "ar_attn.cu": "7833bea0879ccfffcebd2789594852d103d4a56c299b908fa5908aed02333a06"},
+           "bytes": {(8, 2048, 4, 1024): 162741248, (8, 2048, 4, 2048): 202188032}},
+    "dq": {"sources": {"dq.cuh": "d28931aa90808a8e6071b2cc4d04d4d1900378b57cb50325525353d1fd32d1a1", "sm100.cuh": "1111847c6474fba79ab804963ad60d50973f7689121be5d4af96fe31bc24aafe", "ar_attn.cu": "7833bea0879ccfffcebd2789594852d103d4a56c299b908fa5908aed02333a06"},
+           "bytes": {(8, 2048, 4, 1024): 149252864, (8, 2048, 4, 2048): 179639808}},
+    "bwd_prep": {"sources": {"aux.cuh": "33022e858a94bb1b6c8139535df48e09484cecd14f8498239ca7397d16237c60", "sm100.cuh": "1111847c6474fba79ab804963ad60d50973f7689121be5d4af96fe31bc24aafe", "ar_attn.cu": "7833bea0879ccfffcebd2789594852d103d4a56c299b908fa5908aed02333a06"},
+           "bytes": {(8, 2048, 4, 1024): 50615808, (8, 2048, 4, 2048): 50615808}},
+}
 
 
 def captured_traffic(kind, wl, windows):
@@ -128,7 +148,9 @@ def captured_traffic(kind, wl, windows):
     None when a layer shape was not captured or a source changed since."""
     import hashlib
     rec = CAPTURED_TRAFFIC.get(kind)
-    if rec is None:
+    # captured: the plain multi-head path at head dimension 128 (the RoPE and
+    # value-embedding variants and D = 64 are other instantiations)
+    if rec is None or wl.get("rope") or head_dim(wl) != 128:
         return None
     csrc = os.path.join(ROOT, "sliding_window_attention_rmsnorm_b200", "csrc")
     for name, digest in rec["sources"].items():
@@ -203,12 +225,12 @@ def layer_host_inputs(wl, layer):
     """Seeded bf16 CPU inputs of one layer: q, dO with H heads, k, v with Hkv
     (and ve, g on the value-embedding layers of a RoPE workload)."""
     from sliding_window_attention_rmsnorm_b200 import synth
-    H, Hkv = wl["H"], wl.get("Hkv", wl["H"])
+    H, Hkv, Dh = wl["H"], wl.get("Hkv", wl["H"]), head_dim(wl)
     if Hkv == H:
-        x = synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], H, D)
+        x = synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], H, Dh)
     else:
-        x = synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], H, D, roles=("q", "dO"))
-        x.update(synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], Hkv, D, roles=("k", "v")))
+        x = synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], H, Dh, roles=("q", "dO"))
+        x.update(synth.layer_inputs(wl["config"], layer, wl["B"], wl["T"], Hkv, Dh, roles=("k", "v")))
     if wl.get("rope") and layer % 2 == (wl["n_layer"] - 1) % 2:
         x["ve"], x["g"] = synth.value_embedding(wl["config"], layer, wl["B"], wl["T"], Hkv, D)
     return x
@@ -246,7 +268,7 @@ def oracle_sample(wl, seconds, seed_layer_offset=0):
             orc.attn_fwd(xs["q"], xs["k"], xs["v"], ws[layer])
             orc.attn_bwd(xs["q"], xs["k"], xs["v"], xs["dO"], ws[layer])
         t_total += time.perf_counter() - t0
-        flops += pairs(T, ws[layer]) * FWD_FLOPS_PER_PAIR * (1 + BWD_FACTOR)
+        flops += pairs(T, ws[layer]) * 4 * head_dim(wl) * (1 + BWD_FACTOR)
         heads_done.append((layer, head))
         n += 1
     desc = "%d whole heads (T=%d) of the workload's layers, fwd+bwd in fp64 C/OpenMP" % (n, T)
@@ -389,13 +411,16 @@ def run_ours(args, wl, rank, world, dist):
     nq = -(-T // 128)
     g_pairs = sum(B * H * sum(min(qt + 1, min(nq, (min(w, T) + 127) // 128 + 1)) for qt in range(nq))
                   for w in windows) / L
-    algo_bytes = {"fwd_prep": tok * D * 2 + tok * 4,
-                  "bwd_prep": 3 * tok * D * 2 + tok * 4 * 4,
-                  "dq": g_pairs * 32768 + tok * D * 2 * 2}
+    Dh = head_dim(wl)
+    algo_bytes = {"fwd_prep": tok * Dh * 2 + tok * 4,
+                  "bwd_prep": 3 * tok * Dh * 2 + tok * 4 * 4,
+                  "dq": g_pairs * 32768 + tok * Dh * 2 * 2}
     for k, by in algo_bytes.items():
         if kern[k][1]:
             kernels[k]["gbs"] = by * kern[k][1] / (kern[k][0] * 1e-3) / 1e9
             kernels[k]["hbm_frac"] = kernels[k]["gbs"] / peaks["hbm"]
+    if kern["bwd_prep"][1]:
+        kernels["bwd_prep"]["traffic"] = captured_traffic("bwd_prep", wl, windows)
 
     # End to end: inputs from pinned host memory, results back to host, all inside
     # the timed region.  The copies run on their own streams, layer by layer: the
@@ -462,6 +487,7 @@ def run_ours(args, wl, rank, world, dist):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl["name"], "global_batch": B * world, "seq_len": T, "heads": H,
+                       "head_dim": head_dim(wl),
                        **({"kv_heads": wl["Hkv"]} if wl.get("Hkv", H) != H else {}),
                        "layers": L, "windows": windows, "parallelism": "replicas x%d" % world,
                        "l2": "inputs larger than L2 (%.0f MB of q,k,v,dO per step)"

@@ -312,10 +312,11 @@ int prep_grid(long long rows, int sms) {
   return (int)blocks;
 }
 
-// The delta pre-pass: 32 rows per 256-thread block and iteration, as many
-// blocks as are resident on the GPU at once, looping over the rows.
+// The memory-bound passes: 64 rows per 256-thread block and iteration (two per
+// lane group of 8), as many blocks as are resident on the GPU at once, looping
+// over the rows.
 int bwd_prep_grid(long long rows, int sms, int per_sm) {
-  long long blocks = (rows + 31) / 32;
+  long long blocks = (rows + 63) / 64;
   const long long cap = (long long)sms * per_sm;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;

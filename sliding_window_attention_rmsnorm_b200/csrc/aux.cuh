@@ -86,7 +86,50 @@ __device__ __forceinline__ void dot_bf16x8_f32(float& c0, float& c1, const uint4
 
 // One row (one token of one head, D = 128 or 64 elements) per 8 lanes, D / 4
 // bytes of each of q, o and dO per lane: 256-bit loads (D = 128) when the
-// tensors are 32-byte aligned, 128-bit loads otherwise.
+// tensors are 32-byte aligned, 128-bit loads otherwise.  Each lane group takes
+// two rows per iteration (rows r and r + half a block's stride) and issues all
+// their loads before it uses any, so that enough bytes are in flight.
+template <int kD>
+__device__ __forceinline__ void prep_load(const __nv_bfloat16* __restrict__ x, long long base, uint4& a, uint4& b,
+                                          int wide) {
+  if (kD == 128) {
+    ldg32B(x + base, a, b, wide);
+  } else {
+    a = __ldg(reinterpret_cast<const uint4*>(x + base));
+    b = make_uint4(0, 0, 0, 0);
+  }
+}
+
+template <int kD>
+__device__ __forceinline__ void prep_row(long long r, int sub, const uint4 (&qv)[2], const uint4 (&ov)[2],
+                                         const uint4 (&dv)[2], const float* __restrict__ lse,
+                                         float* __restrict__ lse2, float* __restrict__ delta, float* __restrict__ rq,
+                                         int T, int H, int T_pad, float eps) {
+  float s0 = 0.f, s1 = 0.f, t0 = 0.f, t1 = 0.f;
+#pragma unroll
+  for (int h = 0; h < kD / 64; ++h) {
+    fma_sq_bf16x2_f32(s0, s1, qv[h].x);
+    fma_sq_bf16x2_f32(s0, s1, qv[h].y);
+    fma_sq_bf16x2_f32(s0, s1, qv[h].z);
+    fma_sq_bf16x2_f32(s0, s1, qv[h].w);
+    dot_bf16x8_f32(t0, t1, ov[h], dv[h]);
+  }
+  float ss = s0 + s1, dl = t0 + t1;
+#pragma unroll
+  for (int m = 4; m > 0; m >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, m);
+    dl += __shfl_xor_sync(0xffffffffu, dl, m);
+  }
+  if (sub == 0) {
+    int b, t, h;
+    split_row(r, T, H, b, t, h);
+    const long long bh = (long long)b * H + h;
+    delta[bh * T_pad + t] = dl;
+    rq[bh * T_pad + t] = rsqrtf(ss * (1.0f / kD) + eps);
+    lse2[bh * T_pad + t] = lse[bh * T + t] * 1.4426950408889634f;
+  }
+}
+
 template <int kD>
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ o,
                                 const __nv_bfloat16* __restrict__ dO, const float* __restrict__ lse,
@@ -95,48 +138,23 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_
   static_assert(kD == 64 || kD == 128, "head dimension 64 or 128");
   const long long rows = (long long)B * T * H;
   const int sub = threadIdx.x & 7;
-  const long long gstride = (long long)gridDim.x * (blockDim.x / 8);
-  const float kLog2e = 1.4426950408889634f;
-  for (long long r = (long long)blockIdx.x * (blockDim.x / 8) + threadIdx.x / 8; r < rows; r += gstride) {
-    const long long base = r * kD + sub * (kD / 8);
-    uint4 q0, q1, o0, o1, d0, d1;
-    if (kD == 128) {
-      ldg32B(q + base, q0, q1, wide);
-      ldg32B(o + base, o0, o1, wide);
-      ldg32B(dO + base, d0, d1, wide);
-    } else {
-      q0 = __ldg(reinterpret_cast<const uint4*>(q + base));
-      o0 = __ldg(reinterpret_cast<const uint4*>(o + base));
-      d0 = __ldg(reinterpret_cast<const uint4*>(dO + base));
-      q1 = o1 = d1 = make_uint4(0, 0, 0, 0);
+  const long long per_block = blockDim.x / 8;  // lane groups per block
+  const long long gstride = (long long)gridDim.x * per_block * 2;
+  for (long long r0 = (long long)blockIdx.x * per_block * 2 + threadIdx.x / 8; r0 < rows; r0 += gstride) {
+    const long long r1 = r0 + per_block;
+    const bool two = r1 < rows;  // uniform over the lane group
+    uint4 q0[2], o0[2], d0[2], q1[2], o1[2], d1[2];
+    const long long b0 = r0 * kD + sub * (kD / 8), b1 = r1 * kD + sub * (kD / 8);
+    prep_load<kD>(q, b0, q0[0], q0[1], wide);
+    prep_load<kD>(o, b0, o0[0], o0[1], wide);
+    prep_load<kD>(dO, b0, d0[0], d0[1], wide);
+    if (two) {
+      prep_load<kD>(q, b1, q1[0], q1[1], wide);
+      prep_load<kD>(o, b1, o1[0], o1[1], wide);
+      prep_load<kD>(dO, b1, d1[0], d1[1], wide);
     }
-    float s0 = 0.f, s1 = 0.f, t0 = 0.f, t1 = 0.f;
-    fma_sq_bf16x2_f32(s0, s1, q0.x);
-    fma_sq_bf16x2_f32(s0, s1, q0.y);
-    fma_sq_bf16x2_f32(s0, s1, q0.z);
-    fma_sq_bf16x2_f32(s0, s1, q0.w);
-    dot_bf16x8_f32(t0, t1, o0, d0);
-    if (kD == 128) {
-      fma_sq_bf16x2_f32(s0, s1, q1.x);
-      fma_sq_bf16x2_f32(s0, s1, q1.y);
-      fma_sq_bf16x2_f32(s0, s1, q1.z);
-      fma_sq_bf16x2_f32(s0, s1, q1.w);
-      dot_bf16x8_f32(t0, t1, o1, d1);
-    }
-    float ss = s0 + s1, dl = t0 + t1;
-#pragma unroll
-    for (int m = 4; m > 0; m >>= 1) {
-      ss += __shfl_xor_sync(0xffffffffu, ss, m);
-      dl += __shfl_xor_sync(0xffffffffu, dl, m);
-    }
-    if (sub == 0) {
-      int b, t, h;
-      split_row(r, T, H, b, t, h);
-      const long long bh = (long long)b * H + h;
-      delta[bh * T_pad + t] = dl;
-      rq[bh * T_pad + t] = rsqrtf(ss * (1.0f / kD) + eps);
-      lse2[bh * T_pad + t] = lse[bh * T + t] * kLog2e;
-    }
+    prep_row<kD>(r0, sub, q0, o0, d0, lse, lse2, delta, rq, T, H, T_pad, eps);
+    if (two) prep_row<kD>(r1, sub, q1, o1, d1, lse, lse2, delta, rq, T, H, T_pad, eps);
   }
   const long long pads = (long long)B * H * (T_pad - T);
   for (long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x; x < pads; x += (long long)gridDim.x * blockDim.x) {
