@@ -3,8 +3,10 @@
 The pages run two steps just before the attention core ("autoresearch" README
 (gitee), section 7.4: rotary position embedding of q and k with bf16 cos/sin
 tables; section 5.2.3: v + 2 sigmoid(g) ve on the layers that have a value
-embedding).  ar_attn_fwd_rope does both inside the forward kernel's tile
-loads; ar_attn_bwd_rope finishes the chain rule in the backward's epilogues.
+embedding).  ar_attn_fwd_rope rotates k and mixes v once per layer in a
+pre-pass and rotates each Q tile inside the forward kernel;
+ar_attn_bwd_rope runs the backward kernels on the pre-pass's rotated and mixed
+operands and finishes the chain rule in their epilogues.
 
 The kernels round the rotated q, k and the mixed v to bf16 once before their
 products; in the pages' model those are bf16 tensors too (their rotation and
@@ -183,5 +185,30 @@ def test_backward_rope_ve_full_size_sampled():
         check(g[n], r[n], n, "rope bwd full size", heads, H)
     a = np.stack([g["dg"][h // H, :, h % H] for h in heads])
     b = np.stack([r["dg"][h // H, :, h % H] for h in heads])
+    err = np.abs(a - b)
+    assert (err - (MAX_ABS + ULP * np.abs(b))).max() <= 0 and np.linalg.norm(a - b) / np.linalg.norm(b) <= REL_L2
+
+
+def test_backward_rope_ve_several_head_groups():
+    """B=2, T=8192, H=8, Hkv=4, full causal, RoPE and the value embedding: the
+    G tiles of all 16 query heads exceed the 1 GiB buffer, so the backward runs
+    as two launches over disjoint K/V-head groups, on the rotated and mixed
+    operands the pre-pass writes after the G buffer.  One K/V head from each
+    launch (with its two query heads) against the oracle."""
+    B, T, H, Hkv, w = 2, 8192, 8, 4, -1
+    assert attn.bwd_workspace_bytes(B, T, H, 128, Hkv) < B * H * 2080 * 32768  # really split
+    x = inputs(36, B, T, H, Hkv, True)
+    g = gpu_fwd_bwd(x, w)
+    heads = [1, B * Hkv - 2]  # first launch: K/V heads 0-3; second: 4-7
+    grp = H // Hkv
+    qheads = [hk // Hkv * H + (hk % Hkv) * grp + m for hk in heads for m in range(grp)]
+    r = orv.attn_bwd(x["q"], x["k"], x["v"], x["dO"], x["cos"], x["sin"], w, ve=x["ve"], g=x["g"], heads=heads,
+                     round_operands=orv.bf16_round)
+    tag = "rope bwd head groups"
+    check(g["dq"], r["dq"], "dq", tag, qheads, H)
+    for n in ("dk", "dv", "dve"):
+        check(g[n], r[n], n, tag, heads, Hkv)
+    a = np.stack([g["dg"][h // Hkv, :, h % Hkv] for h in heads])
+    b = np.stack([r["dg"][h // Hkv, :, h % Hkv] for h in heads])
     err = np.abs(a - b)
     assert (err - (MAX_ABS + ULP * np.abs(b))).max() <= 0 and np.linalg.norm(a - b) / np.linalg.norm(b) <= REL_L2
