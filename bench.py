@@ -70,7 +70,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="stack8")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="--impl reference: oracle time budget for the whole run")
@@ -434,47 +434,97 @@ def run_ours(args, wl, rank, world, dist):
         outs_h = [{n: torch.empty(st.out[l][n].shape, dtype=st.out[l][n].dtype, pin_memory=True)
                    for n in out_names[l]} for l in range(L)]
         h2d_stream, d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
+        # Two stacks (inputs, outputs, scratch), alternating steps: while step i
+        # computes on one and its results cross back to the host, step i+1's
+        # inputs cross into the other, so the two directions of the host link
+        # overlap.  Within a step the forward operands of layer l cross before
+        # layer l+1's, dO last (last layer first, the backward's order), each
+        # layer's o goes back as soon as its forward is done and its gradients
+        # as soon as its backward is.
+        layers2 = [{r: torch.empty_like(t) for r, t in x.items()} for x in layers]
+        st2 = stack.Stack(layers2, wl.get("pattern", "SSSL"), windows=wl.get("windows"), rope=rope)
+        bufs = [(st, layers), (st2, layers2)]
+        inputs_free = [None, None]  # per stack: its previous step's last kernel
+        outputs_read = [None, None]  # per stack: its previous step's last copy to the host
 
-        def e2e_step():
-            h2d_stream.wait_stream(stream)  # the previous step is done with the device buffers
-            ev_in = []
+        def mark(strm):
+            ev = torch.cuda.Event()
+            ev.record(strm)
+            return ev
+
+        def issue_h2d(i):
+            _, lay = bufs[i % 2]
             with torch.cuda.stream(h2d_stream):
+                if inputs_free[i % 2] is not None:
+                    h2d_stream.wait_event(inputs_free[i % 2])
+                fwd_in = []
                 for l in range(L):
                     for r, t in pinned[l].items():
-                        layers[l][r].copy_(t, non_blocking=True)
-                    ev = torch.cuda.Event()
-                    ev.record(h2d_stream)
-                    ev_in.append(ev)
+                        if r != "dO":
+                            lay[l][r].copy_(t, non_blocking=True)
+                    fwd_in.append(mark(h2d_stream))
+                bwd_in = [None] * L
+                for l in reversed(range(L)):
+                    lay[l]["dO"].copy_(pinned[l]["dO"], non_blocking=True)
+                    bwd_in[l] = mark(h2d_stream)
+            return fwd_in, bwd_in
+
+        def compute(i, fwd_in, bwd_in):
+            s = bufs[i % 2][0]
+            if outputs_read[i % 2] is not None:
+                stream.wait_event(outputs_read[i % 2])
             for l in range(L):
-                stream.wait_event(ev_in[l])
-                st.forward_layer(l)
-            d2h_stream.wait_stream(stream)
-            with torch.cuda.stream(d2h_stream):
-                for l in range(L):
-                    outs_h[l]["o"].copy_(st.out[l]["o"], non_blocking=True)
+                stream.wait_event(fwd_in[l])
+                s.forward_layer(l)
+                d2h_stream.wait_event(mark(stream))
+                with torch.cuda.stream(d2h_stream):
+                    outs_h[l]["o"].copy_(s.out[l]["o"], non_blocking=True)
             for l in reversed(range(L)):
-                st.backward_layer(l)
-                d2h_stream.wait_stream(stream)
+                stream.wait_event(bwd_in[l])
+                s.backward_layer(l)
+                d2h_stream.wait_event(mark(stream))
                 with torch.cuda.stream(d2h_stream):
                     for n in out_names[l]:
                         if n != "o":
-                            outs_h[l][n].copy_(st.out[l][n], non_blocking=True)
+                            outs_h[l][n].copy_(s.out[l][n], non_blocking=True)
+            inputs_free[i % 2] = mark(stream)
+            outputs_read[i % 2] = mark(d2h_stream)
+
+        def run_steps(n):
+            h2d_stream.wait_stream(stream)
+            ins = issue_h2d(0)
+            for i in range(n):
+                nxt = issue_h2d(i + 1) if i + 1 < n else None
+                compute(i, *ins)
+                ins = nxt
             stream.wait_stream(d2h_stream)
-        e2e_step()
+
+        run_steps(2)
         torch.cuda.synchronize()
         barrier()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        run_steps(args.e2e_steps)
         a1.record(stream)
         torch.cuda.synchronize()
         ms_e2e = a0.elapsed_time(a1) / args.e2e_steps
+        # the pipelined copies must not change a result: the last step's outputs on
+        # the host equal, bit for bit, an ordinary step's on the device (the kernels
+        # are deterministic and both buffer sets hold the same inputs)
+        st.step()
+        torch.cuda.synchronize()
+        for l in range(L):
+            for n in out_names[l]:
+                if not torch.equal(outs_h[l][n], st.out[l][n].cpu()):
+                    raise RuntimeError("e2e: layer %d %s differs from an ordinary step" % (l, n))
         ms_e2e = max_over_ranks(dist, ms_e2e, "cuda")
         h2d = sum(t.numel() * t.element_size() for x in pinned for t in x.values())
         d2h = sum(t.numel() * t.element_size() for x in outs_h for t in x.values())
         e2e = {"value": job_tflops(world, fwd_f + bwd_f, ms_e2e), "unit": "TFLOP/s",
-               "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "copies": "every step's inputs from pinned host memory and all its outputs back, inside the timed "
+                         "region; two device buffer sets, so step i+1's uploads overlap step i's compute and "
+                         "downloads; outputs checked bitwise against an ordinary step"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
