@@ -166,6 +166,20 @@ int ar_attn_bwd_rope(const void* q, const void* k, const void* v, const void* o,
                      void* dq, void* dk, void* dv, void* dve, float* dgate, int B, int T, int H, int Hkv, int D,
                      int window, float eps, float scale, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ar_attn_bwd_rope given the forward's pre-pass output, as a training step
+ * keeps an activation: `saved` is the workspace that ar_attn_fwd_rope was given
+ * for the same k, v, ve, ve_gate and tables, not written since (it holds the
+ * rotated k and, with a value embedding, the mixed v: the bf16 values the
+ * backward's pre-pass would form again).  The pre-pass then rotates only q.
+ * Outputs are bitwise those of ar_attn_bwd_rope.  `saved` is read only and
+ * must be 256-byte aligned (AR_ERR_ALIGN otherwise); NULL means
+ * ar_attn_bwd_rope.  The workspace requirement is unchanged. */
+int ar_attn_bwd_rope_saved(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                           const float* lse, const void* rope_cos, const void* rope_sin, int rope_rows,
+                           const void* ve, const void* ve_gate, void* dq, void* dk, void* dv, void* dve,
+                           float* dgate, int B, int T, int H, int Hkv, int D, int window, float eps, float scale,
+                           const void* saved, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears this device's status word.
  * Returns AR_OK, AR_ERR_TIMEOUT if a kernel abandoned a wait since the last
  * call, AR_ERR_LAYOUT if a kernel refused to run, or AR_ERR_CUDA if the

@@ -74,6 +74,9 @@ def lib():
         L.ar_attn_bwd_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp,
                                        i, i, i, i, i, i, f, f, vp, sz, vp]
         L.ar_attn_bwd_rope.restype = i
+        L.ar_attn_bwd_rope_saved.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp,
+                                             i, i, i, i, i, i, f, f, vp, vp, sz, vp]
+        L.ar_attn_bwd_rope_saved.restype = i
         L.ar_attn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
         L.ar_attn_set_wait_limit_ns.restype = i
         L.ar_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, vp]
@@ -281,10 +284,12 @@ def bwd_rope_workspace_bytes(B, T, H, D, Hkv=None, with_ve=False) -> int:
 
 
 def bwd_rope(q, k, v, o, dO, lse, cos, sin, window: int, eps: float = 1e-6, scale=None, ve=None, ve_gate=None,
-             dq=None, dk=None, dv=None, dve=None, dgate=None, workspace=None):
+             dq=None, dk=None, dv=None, dve=None, dgate=None, workspace=None, saved=None):
     """Backward of fwd_rope: (dq, dk, dv) for the unrotated, unmixed q, k, v,
     plus (dve, dgate) when the forward mixed in a value embedding (dgate: the
-    gradient of the gate logits, fp32 [B, T, Hkv])."""
+    gradient of the gate logits, fp32 [B, T, Hkv]).  saved: the workspace the
+    forward was given for the same k, v, ve, ve_gate and tables, untouched since
+    (its rotated k and mixed v are then used instead of formed again)."""
     Hkv = _check_qkv(q, k, v)
     _check_inputs(q, o, dO)
     B, T, H, D = q.shape
@@ -312,11 +317,15 @@ def bwd_rope(q, k, v, o, dO, lse, cos, sin, window: int, eps: float = 1e-6, scal
     if workspace is None:
         workspace = torch.empty(bwd_rope_workspace_bytes(B, T, H, D, Hkv, with_ve), dtype=torch.uint8,
                                 device=q.device)
-    st = lib().ar_attn_bwd_rope(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(cos), _ptr(sin),
-                                int(cos.shape[0]), _ptr(ve), _ptr(ve_gate), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dve),
-                                _ptr(dgate), B, T, H, Hkv, D, int(window), float(eps), float(scale), _ptr(workspace),
-                                workspace.numel(), _stream())
-    _check(st, "ar_attn_bwd_rope")
+    if saved is not None:
+        need = fwd_rope_workspace_bytes(B, T, Hkv, D, with_ve)
+        if not (saved.is_cuda and saved.device == q.device and saved.numel() * saved.element_size() >= need):
+            raise ValueError("saved must be the forward's CUDA workspace (at least %d bytes)" % need)
+    st = lib().ar_attn_bwd_rope_saved(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(cos),
+                                      _ptr(sin), int(cos.shape[0]), _ptr(ve), _ptr(ve_gate), _ptr(dq), _ptr(dk),
+                                      _ptr(dv), _ptr(dve), _ptr(dgate), B, T, H, Hkv, D, int(window), float(eps),
+                                      float(scale), _ptr(saved), _ptr(workspace), workspace.numel(), _stream())
+    _check(st, "ar_attn_bwd_rope_saved")
     return (dq, dk, dv, dve, dgate) if with_ve else (dq, dk, dv)
 
 

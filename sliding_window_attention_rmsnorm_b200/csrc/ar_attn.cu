@@ -438,6 +438,9 @@ struct RopeArgs {
   const __nv_bfloat16 *rcos = nullptr, *rsin = nullptr, *ve = nullptr, *vg = nullptr;
   __nv_bfloat16* dve = nullptr;
   float* dg = nullptr;
+  // the forward's workspace for the same inputs: its rotated k (and mixed v),
+  // used instead of forming them again (NULL: the pre-pass forms them)
+  const __nv_bfloat16* saved = nullptr;
 };
 
 // Extra workspace of the RoPE path: the rotated q and k and (with a value
@@ -476,11 +479,17 @@ int bwd_run(const void* q, const void* k, const void* v, const void* o, const vo
     __nv_bfloat16* qr = reinterpret_cast<__nv_bfloat16*>(r8);
     __nv_bfloat16* kr = reinterpret_cast<__nv_bfloat16*>(r8 + round_up((size_t)B * T * H * kD * 2, 256));
     __nv_bfloat16* vm = kr + round_up((size_t)B * T * Hkv * kD * 2, 256) / 2;
-    const long long prows = rows + (long long)B * T * Hkv * (ra->ve ? 2 : 1);
+    if (ra->saved) {
+      // the forward's pre-pass output: rotated k at the start, mixed v after it
+      kr = const_cast<__nv_bfloat16*>(ra->saved);
+      vm = kr + round_up((size_t)B * T * Hkv * kD * 2, 256) / 2;
+    }
+    const long long prows = rows + (ra->saved ? 0 : (long long)B * T * Hkv * (ra->ve ? 2 : 1));
     KernelTimer t(AR_KERNEL_ROPE_PREP, s);
     ar::rope_ve_prep_kernel<<<bwd_prep_grid(prows, sms, prep_blocks), 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-        static_cast<const __nv_bfloat16*>(v), ra->ve, ra->vg, ra->rcos, ra->rsin, qr, kr, vm, B, T, H, Hkv);
+        static_cast<const __nv_bfloat16*>(q), ra->saved ? nullptr : static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), ra->saved ? nullptr : ra->ve, ra->vg, ra->rcos, ra->rsin, qr, kr, vm,
+        B, T, H, Hkv);
     t.stop();
     qx = qr;
     kx = kr;
@@ -638,6 +647,16 @@ int ar_attn_bwd_rope(const void* q, const void* k, const void* v, const void* o,
                      const void* rope_cos, const void* rope_sin, int rope_rows, const void* ve, const void* ve_gate,
                      void* dq, void* dk, void* dv, void* dve, float* dgate, int B, int T, int H, int Hkv, int D,
                      int window, float eps, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  return ar_attn_bwd_rope_saved(q, k, v, o, dO, lse, rope_cos, rope_sin, rope_rows, ve, ve_gate, dq, dk, dv, dve,
+                                dgate, B, T, H, Hkv, D, window, eps, scale, nullptr, workspace, workspace_bytes,
+                                stream);
+}
+
+int ar_attn_bwd_rope_saved(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                           const float* lse, const void* rope_cos, const void* rope_sin, int rope_rows,
+                           const void* ve, const void* ve_gate, void* dq, void* dk, void* dv, void* dve,
+                           float* dgate, int B, int T, int H, int Hkv, int D, int window, float eps, float scale,
+                           const void* saved, void* workspace, size_t workspace_bytes, void* stream) {
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !rope_cos || !rope_sin) return AR_ERR_NULL;
   const bool with_ve = ve != nullptr;
   if (with_ve && (!ve_gate || !dve || !dgate)) return AR_ERR_NULL;
@@ -655,7 +674,9 @@ int ar_attn_bwd_rope(const void* q, const void* k, const void* v, const void* o,
   const size_t need = ar_attn_bwd_rope_workspace_bytes(B, T, H, Hkv, D, with_ve);
   if (workspace && workspace_bytes < need) return AR_ERR_WORKSPACE;
   if (workspace && !aligned(workspace, 256)) return AR_ERR_ALIGN;
+  if (saved && !aligned(saved, 256)) return AR_ERR_ALIGN;
   RopeArgs ra;
+  ra.saved = static_cast<const __nv_bfloat16*>(saved);
   ra.rcos = static_cast<const __nv_bfloat16*>(rope_cos);
   ra.rsin = static_cast<const __nv_bfloat16*>(rope_sin);
   ra.ve = static_cast<const __nv_bfloat16*>(ve);

@@ -170,7 +170,8 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_
 // mixed v (v + 2 sigmoid(g) ve) written out for the attention kernels, with the
 // arithmetic of sm100.cuh's helpers.  Rows [0, nq) are q rows [B, T, H] (none
 // when q is NULL: the forward rotates its Q tiles itself), then nk k rows and,
-// when ve is given, nk v rows [B, T, Hkv]; one row per 8 lanes.  RoPE: lane l
+// when ve is given, nk v rows [B, T, Hkv] (no k or v rows when k is NULL: the
+// backward given the forward's rotated k and mixed v); one row per 8 lanes.  RoPE: lane l
 // rotates features 8l .. 8l+7 with their partners 64 + 8l ..; value embedding:
 // lane l mixes features 16l .. 16l+15.
 __global__ void rope_ve_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
@@ -179,8 +180,8 @@ __global__ void rope_ve_prep_kernel(const __nv_bfloat16* __restrict__ q, const _
                                     const __nv_bfloat16* __restrict__ rsin, __nv_bfloat16* __restrict__ qr,
                                     __nv_bfloat16* __restrict__ kr, __nv_bfloat16* __restrict__ vm, int B, int T,
                                     int H, int Hkv) {
-  const long long nq = q ? (long long)B * T * H : 0, nk = (long long)B * T * Hkv;
-  const long long rows = nq + nk + (ve ? nk : 0);
+  const long long nq = q ? (long long)B * T * H : 0, nk = k ? (long long)B * T * Hkv : 0;
+  const long long rows = nq + nk + (ve && k ? nk : 0);
   const int sub = threadIdx.x & 7;
   const long long gstride = (long long)gridDim.x * (blockDim.x / 8);
   for (long long r = (long long)blockIdx.x * (blockDim.x / 8) + threadIdx.x / 8; r < rows; r += gstride) {

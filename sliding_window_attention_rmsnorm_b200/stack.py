@@ -33,7 +33,9 @@ class Stack:
     with a value embedding, ve [B, T, Hkv, 128] and g [B, T, Hkv].
     rope: optional (cos, sin) tables; with them every layer runs the fused RoPE
     path (fwd_rope / bwd_rope), with the value embedding where a layer has one.
-    Outputs (o, lse, dq, dk, dv[, dve, dg]) and scratch are allocated once and reused.
+    Outputs (o, lse, dq, dk, dv[, dve, dg]) and scratch are allocated once and reused;
+    with rope, each layer's forward workspace (its rotated k and mixed v) is kept
+    for that layer's backward, which then rotates only q.
     """
 
     def __init__(self, layers, pattern: str = "SSSL", eps: float = 1e-6, scale=None, windows=None, rope=None):
@@ -55,9 +57,10 @@ class Stack:
             with_ve = any("ve" in L for L in layers)
             self.ws_bwd = torch.empty(attn.bwd_rope_workspace_bytes(B, T, H, D, Hkv, with_ve), dtype=torch.uint8,
                                       device=dev)
-            # the forward's pre-pass output fits in the backward's workspace, and the
-            # two run one after the other on the same stream
-            assert attn.fwd_rope_workspace_bytes(B, T, Hkv, D, with_ve) <= self.ws_bwd.numel()
+            # each layer's forward pre-pass output (rotated k, mixed v) is kept, as
+            # an activation, for that layer's backward
+            self.ws_fwd = [torch.empty(attn.fwd_rope_workspace_bytes(B, T, Hkv, D, "ve" in L), dtype=torch.uint8,
+                                       device=dev) for L in layers]
             for L, O in zip(layers, self.out):
                 if "ve" in L:
                     O["dve"] = torch.empty_like(L["ve"])
@@ -69,7 +72,7 @@ class Stack:
             attn.fwd(L["q"], L["k"], L["v"], w, self.eps, self.scale, out=O["o"], lse=O["lse"])
         else:
             attn.fwd_rope(L["q"], L["k"], L["v"], self.rope[0], self.rope[1], w, self.eps, self.scale,
-                          ve=L.get("ve"), ve_gate=L.get("g"), out=O["o"], lse=O["lse"], workspace=self.ws_bwd)
+                          ve=L.get("ve"), ve_gate=L.get("g"), out=O["o"], lse=O["lse"], workspace=self.ws_fwd[l])
 
     def backward_layer(self, l: int):
         L, O, w = self.layers[l], self.out[l], self.windows[l]
@@ -79,7 +82,8 @@ class Stack:
         else:
             attn.bwd_rope(L["q"], L["k"], L["v"], O["o"], L["dO"], O["lse"], self.rope[0], self.rope[1], w,
                           self.eps, self.scale, ve=L.get("ve"), ve_gate=L.get("g"), dq=O["dq"], dk=O["dk"],
-                          dv=O["dv"], dve=O.get("dve"), dgate=O.get("dg"), workspace=self.ws_bwd)
+                          dv=O["dv"], dve=O.get("dve"), dgate=O.get("dg"), workspace=self.ws_bwd,
+                          saved=self.ws_fwd[l])
 
     def forward(self):
         for l in range(len(self.layers)):

@@ -172,6 +172,42 @@ def test_stack_buffers_follow_kv_heads(L):
         assert st.ws_bwd.numel() == attn.bwd_workspace_bytes(B, T, H, D, Hkv) > 0
 
 
+def test_stack_keeps_rope_forward_workspaces(L):
+    """With RoPE each layer keeps its own forward workspace (its rotated k and
+    mixed v) for its backward, sized by whether the layer has a value embedding."""
+    import torch
+    from sliding_window_attention_rmsnorm_b200 import stack
+    B, T, H, Hkv, D = 1, 200, 4, 2, 128
+    z = lambda h: torch.zeros(B, T, h, D, dtype=torch.bfloat16)  # noqa: E731
+    plain = dict(q=z(H), dO=z(H), k=z(Hkv), v=z(Hkv))
+    with_ve = dict(plain, ve=z(Hkv), g=torch.zeros(B, T, Hkv, dtype=torch.bfloat16))
+    cos = torch.zeros(T, 64, dtype=torch.bfloat16)
+    st = stack.Stack([plain, with_ve], windows=[100, 200], rope=(cos, cos))
+    assert [w.numel() for w in st.ws_fwd] == [attn.fwd_rope_workspace_bytes(B, T, Hkv, D, False),
+                                              attn.fwd_rope_workspace_bytes(B, T, Hkv, D, True)]
+    assert st.ws_fwd[0].data_ptr() != st.ws_fwd[1].data_ptr()
+
+
+def test_bwd_rope_saved_argument_errors(L):
+    """ar_attn_bwd_rope_saved validates like ar_attn_bwd_rope, and `saved` must
+    be 256-byte aligned; every call here fails before touching the device."""
+    vp, P = ctypes.c_void_p, lambda a: ctypes.c_void_p(a)  # noqa: E731
+    B, T, H, Hkv, D = 1, 256, 4, 2, 128
+    args = dict(q=P(0x100000), k=P(0x200000), v=P(0x300000), o=P(0x400000), dO=P(0x500000), lse=P(0x600000),
+                cos=P(0x700000), sin=P(0x800000), dq=P(0x900000), dk=P(0xa00000), dv=P(0xb00000))
+
+    def call(saved, **over):
+        a = dict(args, **over)
+        return L.ar_attn_bwd_rope_saved(a["q"], a["k"], a["v"], a["o"], a["dO"], a["lse"], a["cos"], a["sin"], T,
+                                        None, None, a["dq"], a["dk"], a["dv"], None, None, B, T, H, Hkv, D, 128,
+                                        ctypes.c_float(1e-6), ctypes.c_float(0.088), saved, P(0xc00000),
+                                        ctypes.c_size_t(1 << 40), None)
+    assert call(P(0xd00010)) == -4                    # saved not 256-byte aligned
+    assert call(P(0xd00000), q=None) == -1            # a required pointer missing
+    assert call(P(0xd00000), dq=P(0x900008)) == -4    # an output not 16-byte aligned
+    assert call(None, q=None) == -1                   # saved = NULL: ar_attn_bwd_rope's checks
+
+
 def test_wait_limit_setter(L):
     """Host-side only: the setter accepts any limit and 0 restores the default."""
     assert L.ar_attn_set_wait_limit_ns(ctypes.c_ulonglong(1)) == 0

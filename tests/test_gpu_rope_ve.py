@@ -212,3 +212,24 @@ def test_backward_rope_ve_several_head_groups():
     b = np.stack([r["dg"][h // Hkv, :, h % Hkv] for h in heads])
     err = np.abs(a - b)
     assert (err - (MAX_ABS + ULP * np.abs(b))).max() <= 0 and np.linalg.norm(a - b) / np.linalg.norm(b) <= REL_L2
+
+
+@pytest.mark.parametrize("B,T,H,Hkv,w,with_ve", [(2, 300, 4, 2, 100, True), (1, 640, 4, 4, 256, False),
+                                                 (2, 2048, 4, 4, 1024, True)])
+def test_backward_with_saved_forward_operands(B, T, H, Hkv, w, with_ve):
+    """ar_attn_bwd_rope_saved, given the forward's workspace (its rotated k and
+    mixed v), rotates only q and returns bitwise the outputs of ar_attn_bwd_rope,
+    which forms them again."""
+    x = inputs(38, B, T, H, Hkv, with_ve)
+    d = {n: t.cuda() for n, t in x.items()}
+    ws = torch.empty(attn.fwd_rope_workspace_bytes(B, T, Hkv, 128, with_ve), dtype=torch.uint8, device="cuda")
+    o, lse = attn.fwd_rope(d["q"], d["k"], d["v"], d["cos"], d["sin"], w, ve=d.get("ve"), ve_gate=d.get("g"),
+                           workspace=ws)
+    a = attn.bwd_rope(d["q"], d["k"], d["v"], o, d["dO"], lse, d["cos"], d["sin"], w, ve=d.get("ve"),
+                      ve_gate=d.get("g"))
+    b = attn.bwd_rope(d["q"], d["k"], d["v"], o, d["dO"], lse, d["cos"], d["sin"], w, ve=d.get("ve"),
+                      ve_gate=d.get("g"), saved=ws)
+    attn.sync_status()
+    assert len(a) == len(b) == (5 if with_ve else 3)
+    for n, ta, tb in zip(("dq", "dk", "dv", "dve", "dg"), a, b):
+        assert torch.equal(ta, tb), n
