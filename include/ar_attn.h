@@ -136,7 +136,9 @@ int ar_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, 
  *   ve, ve_gate: both NULL (no value embedding), or ve bf16 [B, T, Hkv, D] and
  *     the gate logits g bf16 [B, T, Hkv]: v becomes v + 2 sigmoid(g) ve.
  *   workspace: at least ar_attn_fwd_rope_workspace_bytes(B, T, Hkv, D, ve != NULL)
- *     bytes, 256-byte aligned (NULL: allocated stream-ordered on `stream`).
+ *     bytes, 256-byte aligned (NULL: allocated stream-ordered on `stream`).  It
+ *     keeps the rotated k and mixed v after the call: a caller that keeps it
+ *     until the backward can pass it to ar_attn_bwd_rope_saved.
  * The rotated and mixed values are rounded to bf16 once, as the pages hold
  * them.  Everything else (layouts, lse optional, grouped K/V heads, errors) is
  * as for ar_attn_fwd_gqa.  AR_ERR_NULL if a table is NULL or only one of ve,
