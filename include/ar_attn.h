@@ -15,7 +15,8 @@
  * web3.okx.com code review, paragraphs on the QK norm and on the window pattern.
  *
  * Conventions shared by every entry point
- *   - q, k, v, o, dO, dq, dk, dv: bf16, layout [B, T, H, D] contiguous, D = 128.
+ *   - q, k, v, o, dO, dq, dk, dv: bf16, layout [B, T, H, D] contiguous, D = 64 or
+ *     128 (128 on the RoPE and no-alloc entry points).
  *   - lse: fp32 [B, H, T], natural logarithm.
  *   - window: a key j is visible to query i iff 0 <= i - j <= window.  window < 0
  *     or window >= T - 1 means full causal attention.  window = 0: each query
@@ -32,11 +33,13 @@
  *     abort crosses the ABI.  Argument errors are detected before any work is
  *     enqueued.  A device-side wait that gives up (AR_ERR_TIMEOUT) is reported
  *     by ar_attn_sync_status().
- *   - Workspace (ar_attn_bwd only; the forward needs none): if `workspace` is NULL
+ *   - Workspace (the backward entry points and the RoPE forward; ar_attn_fwd
+ *     needs none): if `workspace` is NULL
  *     the library allocates it stream-ordered (cudaMallocAsync / cudaFreeAsync
  *     on `stream`); otherwise it must hold at least the bytes returned by
- *     ar_attn_bwd_workspace_bytes() and be 256-byte aligned.  It is scratch:
- *     its contents on entry do not matter.
+ *     entry point's *_workspace_bytes() and be 256-byte aligned.  It is scratch:
+ *     its contents on entry do not matter (ar_attn_bwd_rope_saved also reads a
+ *     RoPE forward's workspace, as its `saved` argument).
  */
 #ifndef AR_ATTN_H
 #define AR_ATTN_H
@@ -51,7 +54,7 @@ enum {
   AR_OK = 0,
   AR_ERR_NULL = -1,        /* a required pointer is NULL */
   AR_ERR_SHAPE = -2,       /* B, T or H <= 0, or sizes overflow the index range */
-  AR_ERR_UNSUPPORTED = -3, /* D != 128 */
+  AR_ERR_UNSUPPORTED = -3, /* D other than 64 or 128 (or than 128 where only 128 is built) */
   AR_ERR_ALIGN = -4,       /* a pointer is not 16-byte aligned (workspace: 256) */
   AR_ERR_ARG = -5,         /* eps < 0, scale <= 0, or either is not finite */
   AR_ERR_DEVICE = -6,      /* current device is not compute capability 10.0 (B200) */
