@@ -168,6 +168,17 @@ def captured_traffic(kind, wl, windows):
     return sum(per_layer) / len(per_layer)
 
 
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or None."""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples nvidia-smi clocks and throttle reasons while the GPU is timed."""
@@ -295,7 +306,7 @@ def run_reference(args, wl, rank, world):
         "config": {"workload": wl["name"], "global_batch": wl["B"], "seq_len": wl["T"], "heads": wl["H"],
                    "layers": wl["n_layer"], "parallelism": "replicas"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                         "sample": "per step: " + desc},
+                         "sample": "per step: " + desc, "cpu_model": cpu_model(), "nproc": os.cpu_count()},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -529,7 +540,8 @@ def run_ours(args, wl, rank, world, dist):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, secs, desc, threads = oracle_sample(wl, args.cpu_seconds)
-        cpu = {"value": f / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+        cpu = {"value": f / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "cpu_model": cpu_model(), "nproc": os.cpu_count()}
 
     if rank == 0:
         line = {
